@@ -1,0 +1,25 @@
+"""B200 (sm_100a) block-causal gated linear attention: a C-ABI CUDA library
+(libgla.so) with a thin Python binding.  See include/gla.h for the ABI."""
+
+from ._binding import (  # noqa: F401
+    EXPORTED,
+    GLA_ERR_ALIGN,
+    GLA_ERR_ALLOC,
+    GLA_ERR_DEVICE,
+    GLA_ERR_LAUNCH,
+    GLA_ERR_NULL,
+    GLA_ERR_SHAPE,
+    GLA_ERR_UNSUPPORTED_D,
+    GLA_OK,
+    GLAError,
+    forward,
+    gla_device_fault,
+    gla_error_string,
+    gla_forward,
+    gla_forward_timed,
+    gla_version,
+    load_library,
+)
+
+# Every entry point loads libgla.so on first use and raises ImportError when
+# it is missing; there is no other implementation to fall back on.

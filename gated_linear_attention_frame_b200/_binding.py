@@ -1,0 +1,166 @@
+"""ctypes binding of libgla.so, with the same names as the C ABI (include/gla.h).
+
+Only argument marshalling happens here: tensors become device pointers and
+the stream becomes a raw cudaStream_t; every step of the computation runs in
+the library's CUDA kernels.  If the shared library is missing or cannot be
+loaded, importing the package raises -- there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
+
+GLA_OK = 0
+GLA_ERR_NULL = 1
+GLA_ERR_ALIGN = 2
+GLA_ERR_SHAPE = 3
+GLA_ERR_UNSUPPORTED_D = 4
+GLA_ERR_ALLOC = 5
+GLA_ERR_LAUNCH = 6
+GLA_ERR_DEVICE = 7
+
+EXPORTED = ("gla_forward", "gla_forward_timed", "gla_error_string", "gla_device_fault",
+            "gla_version")
+
+
+class GLAError(RuntimeError):
+    def __init__(self, status: int, where: str = "gla_forward"):
+        self.status = int(status)
+        super().__init__("%s failed: %s (status %d)" % (where, gla_error_string(status), status))
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libgla.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(
+            "libgla.so not found at %s; build it with "
+            "`python -m gated_linear_attention_frame_b200.build`" % p)
+    lib = ctypes.CDLL(p)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fwd = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
+    lib.gla_forward.argtypes = fwd
+    lib.gla_forward.restype = i32
+    lib.gla_forward_timed.argtypes = fwd + [ctypes.POINTER(vp)]
+    lib.gla_forward_timed.restype = i32
+    lib.gla_error_string.argtypes = [i32]
+    lib.gla_error_string.restype = ctypes.c_char_p
+    lib.gla_device_fault.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.gla_device_fault.restype = i32
+    lib.gla_version.argtypes = []
+    lib.gla_version.restype = i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(x) -> int | None:
+    """Device pointer of a CUDA tensor, an int address, or None (-> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if x.numel() == 0:
+            return x.data_ptr() or None
+        if not x.is_cuda:
+            raise ValueError("gla: tensors must be on a CUDA device (got %s)" % x.device)
+        if not x.is_contiguous():
+            raise ValueError("gla: tensors must be contiguous")
+        return x.data_ptr()
+    raise TypeError("gla: expected a torch.Tensor, an int address or None, got %r" % type(x))
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check_dtypes(q, k, v, gate_logits, state_in, state_out, out):
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
+                        ("v", v, torch.bfloat16), ("out", out, torch.bfloat16),
+                        ("gate_logits", gate_logits, torch.float32),
+                        ("state_in", state_in, torch.float32),
+                        ("state_out", state_out, torch.float32)):
+        if isinstance(t, torch.Tensor) and t.dtype != dt:
+            raise TypeError("gla: %s must be %s, got %s" % (name, dt, t.dtype))
+
+
+def gla_forward(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
+                tokens_per_frame, d, eps, stream=None) -> None:
+    """Enqueue one layer call (see include/gla.h).  Tensors or raw device
+    addresses; raises GLAError on a nonzero status."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    st = lib.gla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in),
+                         _ptr(state_out), _ptr(out), int(B), int(H), int(frames),
+                         int(tokens_per_frame), int(d), float(eps), _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st)
+
+
+def gla_forward_timed(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
+                      tokens_per_frame, d, eps, stream, events) -> None:
+    """gla_forward that records 4 CUDA events around the three kernels
+    (`events`: 4 torch.cuda.Event(enable_timing=True))."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+    st = lib.gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in),
+                               _ptr(state_out), _ptr(out), int(B), int(H), int(frames),
+                               int(tokens_per_frame), int(d), float(eps), _stream(stream),
+                               ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_timed")
+
+
+def gla_error_string(status: int) -> str:
+    return load_library().gla_error_string(int(status)).decode()
+
+
+def gla_device_fault(stream=None) -> int:
+    """Synchronise `stream`, then read and clear the device fault word."""
+    code = ctypes.c_uint(0)
+    st = load_library().gla_device_fault(_stream(stream), ctypes.byref(code))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_device_fault")
+    return code.value
+
+
+def gla_version() -> int:
+    return load_library().gla_version()
+
+
+def forward(q, k, v, gate_logits, state_in=None, eps: float = 1e-6, out=None, state_out=None,
+            stream=None):
+    """Convenience wrapper: shapes from q [B, N, H, d] and gate_logits
+    [B, frames, H]; allocates `out` and `state_out` if not given.  Returns
+    (out, state_out)."""
+    B, N, H, d = q.shape
+    frames = gate_logits.shape[1]
+    if frames == 0:
+        T = 0
+    else:
+        if N % frames:
+            raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+        T = N // frames
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None:
+        state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
+    gla_forward(q, k, v, gate_logits, state_in, state_out, out, B, H, frames, T, d, eps, stream)
+    return out, state_out

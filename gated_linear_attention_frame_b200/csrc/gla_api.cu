@@ -1,0 +1,277 @@
+// gla_api.cu -- C ABI of the gated linear attention library (see gla.h).
+//
+// gla_forward validates its arguments (no CUDA call before that), takes a
+// stream-ordered workspace, builds the TMA tensor maps of q, k, v and out,
+// and enqueues the three kernels on the caller's stream:
+//   1. gla_increment_kernel  dS_f partials  (tcgen05, TMA, ReLU fused)
+//   2. gla_scan_kernel       S_f = a_f S_{f-1} + dS_f, state_out, bf16 S_f^T images
+//   3. gla_output_kernel     out = phi(q) S_f / (phi(q) S_f[:, d] + eps)   (tcgen05)
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gla.h"
+#include "gla_common.cuh"
+#include "gla_increment.cuh"
+#include "gla_output.cuh"
+#include "gla_scan.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+using gla::Geo;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int major = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <int D>
+cudaError_t set_smem_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(gla::gla_increment_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       gla::IncCfg<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gla::gla_output_kernel<D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gla::OutCfg<D>::kSmemBytes);
+}
+
+// Per-device one-time set-up: SM count, architecture check, kernel attributes,
+// the driver's tensor-map encoder.
+int device_setup(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GLA_ERR_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return GLA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return GLA_ERR_DEVICE;
+    if (prop.major != 10) return GLA_ERR_DEVICE;
+    if (set_smem_attrs<32>() != cudaSuccess || set_smem_attrs<64>() != cudaSuccess ||
+        set_smem_attrs<128>() != cudaSuccess)
+      return GLA_ERR_LAUNCH;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return GLA_ERR_DEVICE;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    di.sms = prop.multiProcessorCount;
+    di.major = prop.major;
+    di.ready = true;
+  }
+  *out = di;
+  return GLA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 5-D view (d, H, T, F, B) of a bf16 [B, F*T, H, d] tensor; box = one swizzle
+// atom of features x `box_rows` tokens of one head of one frame.
+int encode_map(CUtensorMap* m, const void* base, int d, int H, int T, int F, int B, int box_rows) {
+  const int atom = d >= 64 ? 64 : 32;
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(F),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[4] = {d * e, static_cast<cuuint64_t>(H) * d * e,
+                           static_cast<cuuint64_t>(T) * H * d * e,
+                           static_cast<cuuint64_t>(F) * T * H * d * e};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(atom), 1, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GLA_OK : GLA_ERR_LAUNCH;
+}
+
+struct Args {
+  const void *q, *k, *v;
+  const float* g;
+  const float* s_in;
+  float* s_out;
+  void* out;
+  int B, H, F, T, d;
+  float eps;
+  cudaStream_t stream;
+};
+
+// Host-only checks; no CUDA call.
+int validate(const Args& a) {
+  if (a.d != 32 && a.d != 64 && a.d != 128) return GLA_ERR_UNSUPPORTED_D;
+  if (a.B < 0 || a.H < 0 || a.F < 0 || a.T < 0) return GLA_ERR_SHAPE;
+  const int64_t tokens = static_cast<int64_t>(a.F) * a.T;
+  // TMA coordinates and per-frame token offsets are 32-bit.
+  if (tokens > INT32_MAX || static_cast<int64_t>(a.B) * a.H > (int64_t(1) << 24) ||
+      static_cast<int64_t>(a.T) + gla::kTileTokens > INT32_MAX)
+    return GLA_ERR_SHAPE;
+  const int64_t elems = static_cast<int64_t>(a.B) * tokens * a.H * a.d;
+  const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
+  if (elems > (int64_t(1) << 46)) return GLA_ERR_SHAPE;
+  if (elems > 0 && (a.q == nullptr || a.k == nullptr || a.v == nullptr || a.out == nullptr))
+    return GLA_ERR_NULL;
+  if (units > 0 && a.g == nullptr) return GLA_ERR_NULL;
+  if (elems > 0 && (!aligned(a.q, 16) || !aligned(a.k, 16) || !aligned(a.v, 16) ||
+                    !aligned(a.out, 16)))
+    return GLA_ERR_ALIGN;
+  if ((a.g && !aligned(a.g, 4)) || (a.s_in && !aligned(a.s_in, 4)) ||
+      (a.s_out && !aligned(a.s_out, 4)))
+    return GLA_ERR_ALIGN;
+  return GLA_OK;
+}
+
+inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+template <int D>
+int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
+  using G = Geo<D>;
+  const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
+  const int tpu = (a.T + gla::kTileTokens - 1) / gla::kTileTokens;
+  const int64_t W = units * tpu;
+  const int32_t G1 = static_cast<int32_t>(W < di.sms ? W : di.sms);
+  const int32_t G3 = G1;
+
+  const int64_t partial_bytes =
+      W > 0 ? align256((units + G1) * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4) : 0;
+  const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
+  const int64_t ws_bytes = partial_bytes + image_bytes;
+
+  CUtensorMap tm_q, tm_k, tm_v, tm_out;
+  if (W > 0) {
+    int st;
+    if ((st = encode_map(&tm_q, a.q, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_k, a.k, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_v, a.v, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_out, a.out, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+  }
+
+  uint8_t* ws = nullptr;
+  if (ws_bytes > 0) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), a.stream) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return GLA_ERR_ALLOC;
+    }
+  }
+  float* partial = reinterpret_cast<float*>(ws);
+  uint8_t* image = ws ? ws + partial_bytes : nullptr;
+
+  int status = GLA_OK;
+  auto check = [&]() {
+    if (cudaGetLastError() != cudaSuccess) status = GLA_ERR_LAUNCH;
+  };
+  auto record = [&](int i) {
+    if (ev != nullptr && status == GLA_OK && cudaEventRecord(ev[i], a.stream) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+  };
+
+  record(0);
+  if (W > 0 && status == GLA_OK) {
+    gla::IncParams ip{partial, a.H, a.F, tpu, W};
+    gla::gla_increment_kernel<D>
+        <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    check();
+  }
+  record(1);
+  if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
+    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, a.H, a.F, tpu, W, G1};
+    constexpr int NT = (D + 1) * (D / 8);
+    const unsigned grid = static_cast<unsigned>((NT + 255) / 256) * static_cast<unsigned>(a.B * a.H);
+    gla::gla_scan_kernel<D><<<grid, 256, 0, a.stream>>>(sp);
+    check();
+  }
+  record(2);
+  if (W > 0 && status == GLA_OK) {
+    gla::OutParams op{image, a.eps, a.H, a.F, a.T, tpu, W};
+    gla::gla_output_kernel<D>
+        <<<G3, gla::OutCfg<D>::kThreads, gla::OutCfg<D>::kSmemBytes, a.stream>>>(tm_q, tm_out, op);
+    check();
+  }
+  record(3);
+  if (ws != nullptr && cudaFreeAsync(ws, a.stream) != cudaSuccess) {
+    cudaGetLastError();
+    if (status == GLA_OK) status = GLA_ERR_LAUNCH;
+  }
+  return status;
+}
+
+int forward_impl(const Args& a, cudaEvent_t* ev) {
+  int st = validate(a);
+  if (st != GLA_OK) return st;
+  if (static_cast<int64_t>(a.B) * a.H == 0) return GLA_OK;  // nothing to compute or write
+  DeviceInfo di;
+  if ((st = device_setup(&di)) != GLA_OK) return st;
+  switch (a.d) {
+    case 32: return run<32>(a, di, ev);
+    case 64: return run<64>(a, di, ev);
+    default: return run<128>(a, di, ev);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int gla_forward(const void* q, const void* k, const void* v, const float* gate_logits,
+                const float* state_in, float* state_out, void* out, int B, int H, int frames,
+                int tokens_per_frame, int d, float eps, cudaStream_t stream) {
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream};
+  return forward_impl(a, nullptr);
+}
+
+int gla_forward_timed(const void* q, const void* k, const void* v, const float* gate_logits,
+                      const float* state_in, float* state_out, void* out, int B, int H, int frames,
+                      int tokens_per_frame, int d, float eps, cudaStream_t stream,
+                      cudaEvent_t* events) {
+  if (events == nullptr) return GLA_ERR_NULL;
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream};
+  return forward_impl(a, events);
+}
+
+const char* gla_error_string(int status) {
+  switch (status) {
+    case GLA_OK: return "ok";
+    case GLA_ERR_NULL: return "a required pointer is NULL";
+    case GLA_ERR_ALIGN: return "a pointer is not aligned (q, k, v, out: 16 bytes; others: 4)";
+    case GLA_ERR_SHAPE: return "negative or too large size";
+    case GLA_ERR_UNSUPPORTED_D: return "head dim must be 32, 64 or 128";
+    case GLA_ERR_ALLOC: return "workspace allocation failed";
+    case GLA_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
+    case GLA_ERR_DEVICE: return "no CUDA device of compute capability 10.x";
+    default: return "unknown status";
+  }
+}
+
+int gla_device_fault(cudaStream_t stream, unsigned int* code) {
+  if (code == nullptr) return GLA_ERR_NULL;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return GLA_ERR_LAUNCH;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, gla::g_gla_fault, sizeof(v)) != cudaSuccess) return GLA_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(gla::g_gla_fault, &zero, sizeof(zero)) != cudaSuccess)
+    return GLA_ERR_LAUNCH;
+  *code = v;
+  return GLA_OK;
+}
+
+int gla_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,281 @@
+// gla_increment.cuh -- per-frame state increment on tcgen05 tensor cores.
+//
+// For every unit u = (b, f, h) it forms dS_f = phi(K_f)^T [V_f | 1], the
+// block's own key-value contribution that the SANA-Video talk (block KV cache
+// segment) adds to the cached state, as a bf16 x bf16 -> fp32 contraction
+// over the frame's tokens:
+//   A = phi(K_f)^T  [M = 128 key features (rows >= d are zero), K = tokens]
+//   B = V_f         [N = d value features,                     K = tokens]
+// Both operands are MN-major in memory (token rows of d contiguous features),
+// loaded by TMA in 128-token tiles with 128-byte (64-byte for d = 32)
+// swizzle; ReLU is applied in shared memory between the TMA landing and the
+// MMA, and the same pass sums phi(K) over tokens for the normaliser column.
+//
+// Work split: the units' token tiles (W = units * ceil(T / 128)) are divided
+// into contiguous ranges, one per persistent CTA.  A CTA accumulates the
+// tiles of one unit in TMEM and, when the unit or its range ends, writes an
+// fp32 partial [d + 4][d] (transposed: row j = value column, column i = key
+// feature; rows d..d+3 = the four ReLU warps' normaliser sums) to slot
+// (u + cta).  The scan kernel sums a unit's partials.
+//
+// Warp roles (320 threads): warps 0-3 drain TMEM (epilogue), warps 4-7 apply
+// ReLU, warp 8 issues TMA, warp 9 issues MMAs.
+#pragma once
+
+#include "gla_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gla {
+
+template <int D>
+struct IncCfg {
+  using G = Geo<D>;
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kAAtoms = 128 / G::kAtomElems;           // A spans M = 128 rows
+  static constexpr int kABytes = kAAtoms * G::kAtomTileBytes;   // 32 KB
+  static constexpr int kVBytes = G::kTileBytes;
+  static constexpr int kStageBytes = kABytes + kVBytes;
+  static constexpr int kTmemCols = 2 * D;                       // two fp32 accumulators of N = D
+  static constexpr int kPartialRows = D + 4;
+  static constexpr int kPartialFloats = kPartialRows * D;
+  static constexpr int kThreads = 320;
+  static constexpr int kBarBytes = (3 * kStages + 5) * 8;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
+};
+
+struct IncParams {
+  float* partial;   // [(units + gridDim.x) slots][d + 4][d] fp32
+  int H, F, tpu;    // heads, frames, token tiles per frame
+  int64_t W;        // units * tpu
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned int code) {
+  const int lane = threadIdx.x & 31;
+  int ok = 0;
+  if (lane == 0) ok = mbar_wait(bar, parity, abort, code) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_try_wait(bar, parity);  // completed phase: acquire for every lane
+  return ok != 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    gla_increment_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const IncParams p) {
+  using G = Geo<D>;
+  using C = IncCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr unsigned kCode = 1u;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  auto accf = [&](int a) { return bar0 + 8u * (3 * S + a); };
+  auto acce = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (3 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto a_buf = [&](int s) { return sbase + s * C::kStageBytes; };
+  auto v_buf = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const TileSplit split{p.W, static_cast<int32_t>(gridDim.x)};
+  const int64_t lo = split.lo(blockIdx.x);
+  const int64_t hi = split.lo(blockIdx.x + 1);
+  const int tpu = p.tpu;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(relu_done(s), 4);
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf(a), 1);
+      mbar_init(acce(a), 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if constexpr (C::kAAtoms > G::kAtoms) {
+    // Rows d..127 of A: zero atoms that TMA never writes.
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    constexpr int kPadBytes = (C::kAAtoms - G::kAtoms) * G::kAtomTileBytes;
+    for (int s = 0; s < S; ++s)
+      for (int o = threadIdx.x * 16; o < kPadBytes; o += C::kThreads * 16)
+        st_shared_v4(a_buf(s) + G::kAtoms * G::kAtomTileBytes + o, z);
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int64_t issued = 0;
+      for (int64_t x = lo; x < hi; ++x, ++issued) {
+        const int s = static_cast<int>(issued % S);
+        const uint32_t ph = static_cast<uint32_t>((issued / S) & 1);
+        if (!mbar_wait(empty(s), ph ^ 1u, abort, kCode)) break;
+        const int64_t u = x / tpu;
+        const int t = static_cast<int>(x - u * tpu);
+        const int h = static_cast<int>(u % p.H);
+        const int64_t bf = u / p.H;
+        const int f = static_cast<int>(bf % p.F);
+        const int b = static_cast<int>(bf / p.F);
+        mbar_arrive_expect_tx(full(s), 2u * G::kTileBytes);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a) {
+          tma_load_5d(a_buf(s) + a * G::kAtomTileBytes, &tm_k, full(s), a * G::kAtomElems, h,
+                      t * kTileTokens, f, b);
+          tma_load_5d(v_buf(s) + a * G::kAtomTileBytes, &tm_v, full(s), a * G::kAtomElems, h,
+                      t * kTileTokens, f, b);
+        }
+      }
+      // Let every load still in flight land before the CTA can exit.
+      for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+      int64_t i = 0, seg = 0;
+      for (int64_t x = lo; x < hi; ++x, ++i) {
+        const int64_t u = x / tpu;
+        const int t = static_cast<int>(x - u * tpu);
+        const bool first = (x == lo) || (t == 0);
+        const bool last = (x == hi - 1) || (t == tpu - 1);
+        const int ab = static_cast<int>(seg & 1);
+        if (first && !mbar_wait(acce(ab), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort, kCode))
+          break;
+        const int s = static_cast<int>(i % S);
+        if (!mbar_wait(relu_done(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+          const uint64_t ad = smem_desc(a_buf(s) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                        G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(v_buf(s) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                        G::kGroupBytes, G::kLayout);
+          mma_bf16(tmem + ab * D, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(empty(s));
+        if (last) {
+          mma_commit(accf(ab));
+          ++seg;
+        }
+      }
+      mma_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- ReLU + normaliser sums
+    constexpr int CPR = G::kChunksPerRow;     // 16-byte chunks per token row
+    constexpr int RPP = kTileTokens / CPR;    // rows covered per pass of 128 threads
+    constexpr int CPA = G::kAtomElems / 8;    // chunks per swizzle row
+    const int rt = threadIdx.x - 128;
+    const int c = rt % CPR;
+    const int r0 = rt / CPR;
+    const uint32_t off0 = (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes +
+                          G::swz(r0, c % CPA) * 16;  // same swizzle slot for r0 + RPP*m
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = 0.f;
+    int64_t i = 0;
+    for (int64_t x = lo; x < hi; ++x, ++i) {
+      const int s = static_cast<int>(i % S);
+      if (!warp_wait(full(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+      const uint32_t base = a_buf(s) + off0;
+#pragma unroll
+      for (int m = 0; m < CPR; ++m) {
+        const uint32_t addr = base + m * RPP * G::kRowBytes;
+        uint4 w = ld_shared_v4(addr);
+        relu8(w);
+        st_shared_v4(addr, w);
+        z[0] += bf16lo_to_f32(w.x);
+        z[1] += bf16hi_to_f32(w.x);
+        z[2] += bf16lo_to_f32(w.y);
+        z[3] += bf16hi_to_f32(w.y);
+        z[4] += bf16lo_to_f32(w.z);
+        z[5] += bf16hi_to_f32(w.z);
+        z[6] += bf16lo_to_f32(w.w);
+        z[7] += bf16hi_to_f32(w.w);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(relu_done(s));
+      const int64_t u = x / tpu;
+      const int t = static_cast<int>(x - u * tpu);
+      if (x == hi - 1 || t == tpu - 1) {
+        // Unit range ends: this warp's column sums of phi(K) go to row d + (warp - 4).
+#pragma unroll
+        for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) z[e] += __shfl_xor_sync(0xffffffffu, z[e], o);
+        if (lane < CPR) {
+          float* dst = p.partial + (u + blockIdx.x) * static_cast<int64_t>(C::kPartialFloats) +
+                       static_cast<int64_t>(D + warp - 4) * D + lane * 8;
+          reinterpret_cast<float4*>(dst)[0] = make_float4(z[0], z[1], z[2], z[3]);
+          reinterpret_cast<float4*>(dst)[1] = make_float4(z[4], z[5], z[6], z[7]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] = 0.f;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // key feature i
+    int64_t seg = 0;
+    for (int64_t x = lo; x < hi; ++seg) {
+      const int64_t u = x / tpu;
+      const int64_t xe = ((u + 1) * tpu < hi) ? (u + 1) * tpu : hi;
+      const int ab = static_cast<int>(seg & 1);
+      if (!warp_wait(accf(ab), static_cast<uint32_t>((seg >> 1) & 1), abort, kCode)) break;
+      tc_fence_after();
+      if (q4 * 32 < D) {
+        float* dst = p.partial + (u + blockIdx.x) * static_cast<int64_t>(C::kPartialFloats) + row;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * D + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce(ab));
+      x = xe;
+    }
+  }
+
+  __syncwarp();  // producer / MMA roles ran on lane 0 only
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace gla

@@ -1,0 +1,127 @@
+/*
+ * gla.h -- C ABI of the B200 (sm_100a) gated linear attention library.
+ *
+ * Operation (block-causal gated linear attention, one latent video frame per
+ * block).  The SANA-Video pages describe the layer's structure: gated linear
+ * attention is the O(N) mixer of the hybrid DiT (SANA-Video 2.0 project page,
+ * "Hybrid Linear-Softmax Attention"); the state is a fixed-size D x D matrix
+ * to which each block adds its own key-value contribution, cached between
+ * blocks (SANA-Video ICLR 2026 oral talk, block KV cache segment); decay gates
+ * on the recurrent state stop the drift of plain cumulative linear attention
+ * and the attention is applied frame-wise (SANA-WM paper analysis, method
+ * components).  This library fixes the formulas as follows, per batch entry b
+ * and head h, frames f = 0..frames-1, tokens t of frame f:
+ *
+ *   phi(x) = max(x, 0)
+ *   a_f    = 1 / (1 + exp(-gate_logits[b, f, h]))
+ *   S_f    = a_f * S_{f-1} + phi(K_f)^T [V_f | 1]      (d x (d+1), fp32; S_{-1} = state_in)
+ *   out_t  = (phi(q_t) S_f[:, :d]) / (phi(q_t) S_f[:, d] + eps)
+ *   state_out = S_{frames-1}
+ *
+ * Queries of frame f read S_f: attention is bidirectional inside a frame and
+ * causal across frames.  A long sequence can be streamed through several
+ * calls by passing one call's state_out as the next call's state_in; the
+ * result equals one call over all frames up to fp32 rounding.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller; the library keeps no reference after the call.
+ *   - Work is enqueued on `stream` and the call returns without waiting.
+ *     Errors found before launch are returned; faults inside the kernels
+ *     surface at the caller's next synchronisation, and bounded waits that
+ *     gave up are reported by gla_device_fault().
+ *   - Supported head dims: d in {32, 64, 128}.  B, H, frames,
+ *     tokens_per_frame may be 0 (nothing to attend; see gla_forward).
+ *   - Requires a compute capability 10.0 device (B200, sm_100a).
+ */
+#ifndef GLA_H_
+#define GLA_H_
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+typedef enum {
+  GLA_OK = 0,
+  GLA_ERR_NULL = 1,            /* a required pointer is NULL */
+  GLA_ERR_ALIGN = 2,           /* a pointer violates its alignment rule */
+  GLA_ERR_SHAPE = 3,           /* negative or too-large size */
+  GLA_ERR_UNSUPPORTED_D = 4,   /* d not in {32, 64, 128} */
+  GLA_ERR_ALLOC = 5,           /* stream-ordered workspace allocation failed */
+  GLA_ERR_LAUNCH = 6,          /* a CUDA runtime call or kernel launch failed */
+  GLA_ERR_DEVICE = 7           /* no CUDA device, or not compute capability 10.x */
+} gla_status;
+
+/*
+ * gla_forward -- one block-causal gated linear attention layer call.
+ *
+ * Arguments (device pointers unless stated):
+ *   q, k, v      bf16 [B, frames * tokens_per_frame, H, d], contiguous; token
+ *                n = f * tokens_per_frame + t.  16-byte aligned.
+ *   gate_logits  fp32 [B, frames, H]; a = sigmoid(logit).  +inf gives a = 1,
+ *                -inf gives a = 0.  4-byte aligned.  Must not be NULL when
+ *                B * H * frames > 0.
+ *   state_in     fp32 [B, H, d, d + 1] (row i = key feature, column d = the
+ *                normaliser); NULL means the zero state.  4-byte aligned.
+ *   state_out    fp32 [B, H, d, d + 1]; NULL means "not written".  May be the
+ *                same pointer as state_in (updated in place).
+ *   out          bf16 [B, frames * tokens_per_frame, H, d], 16-byte aligned,
+ *                rounded to nearest even.  Must not overlap q, k, v.
+ *   B, H, frames, tokens_per_frame   sizes, each >= 0.  frames == 0 copies
+ *                state_in to state_out; tokens_per_frame == 0 applies only
+ *                the decays to the state.
+ *   d            head dim: 32, 64 or 128.
+ *   eps          added to the normaliser before the division.
+ *   stream       CUDA stream for all work (0 = legacy default stream).
+ *
+ * Memory: takes a workspace of about (B*H*frames*6 + #SMs*4) * (d+1)*d bytes
+ * (per-frame fp32 state increments and bf16 prefix states) with
+ * cudaMallocAsync on `stream` and frees it with cudaFreeAsync on the same
+ * stream.
+ * Returns GLA_OK or a gla_status code; on error nothing was enqueued, except
+ * GLA_ERR_LAUNCH, after which part of the work may have been enqueued.
+ */
+int gla_forward(const void* q, const void* k, const void* v,
+                const float* gate_logits,
+                const float* state_in, float* state_out,
+                void* out,
+                int B, int H, int frames, int tokens_per_frame, int d,
+                float eps, cudaStream_t stream);
+
+/*
+ * gla_forward_timed -- gla_forward that also records four caller-created CUDA
+ * events on `stream`: events[0] before the state-increment kernel, events[1]
+ * after it, events[2] after the gated scan, events[3] after the output
+ * kernel.  Used to time each kernel in place; the computation is identical.
+ * `events` is a host array of 4 cudaEvent_t.
+ */
+int gla_forward_timed(const void* q, const void* k, const void* v,
+                      const float* gate_logits,
+                      const float* state_in, float* state_out,
+                      void* out,
+                      int B, int H, int frames, int tokens_per_frame, int d,
+                      float eps, cudaStream_t stream, cudaEvent_t* events);
+
+/* Static string for a gla_status code (never NULL). Host only, no CUDA call. */
+const char* gla_error_string(int status);
+
+/*
+ * gla_device_fault -- synchronises `stream`, then reads and clears the
+ * library's device-side fault word of the current device.  Nonzero means a
+ * kernel gave up a bounded wait (about one second) and returned early; its
+ * output is then invalid.  Bit 0: state-increment kernel, bit 1: output
+ * kernel.  `code` is a host pointer.  Returns GLA_OK or GLA_ERR_LAUNCH.
+ */
+int gla_device_fault(cudaStream_t stream, unsigned int* code);
+
+/* Library version as major * 10000 + minor * 100 + patch.  Host only. */
+int gla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_H_ */

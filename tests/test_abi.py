@@ -1,0 +1,118 @@
+"""The C-ABI library: builds, loads without a GPU, exports every function that
+include/gla.h declares, and rejects bad arguments before any CUDA call."""
+
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_linear_attention_frame_b200.build import build
+
+    build()
+    import gated_linear_attention_frame_b200 as g
+
+    return g.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(gla_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gla_forward", "gla_error_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    import gated_linear_attention_frame_b200 as g
+
+    assert set(names) == set(g.EXPORTED)
+
+
+def test_error_strings(lib):
+    import gated_linear_attention_frame_b200 as g
+
+    seen = set()
+    for st in range(0, 8):
+        s = g.gla_error_string(st)
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 8
+    assert g.gla_error_string(99) == "unknown status"
+    assert g.gla_version() >= 100
+
+
+def _call(lib, q=None, k=None, v=None, g=None, s_in=None, s_out=None, out=None,
+          B=1, H=1, F=1, T=16, d=32, eps=1e-6):
+    return lib.gla_forward(q, k, v, g, s_in, s_out, out, B, H, F, T, d, eps, None)
+
+
+FAKE = 1 << 20  # never dereferenced: validation fails first
+
+
+def test_validation_before_any_cuda_call(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    ok = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, out=FAKE)
+    assert _call(lib, d=48, **ok) == gl.GLA_ERR_UNSUPPORTED_D
+    assert _call(lib, d=256, **ok) == gl.GLA_ERR_UNSUPPORTED_D
+    assert _call(lib, B=-1, **ok) == gl.GLA_ERR_SHAPE
+    assert _call(lib, T=-5, **ok) == gl.GLA_ERR_SHAPE
+    assert _call(lib, F=1 << 20, T=1 << 12, **ok) == gl.GLA_ERR_SHAPE
+    assert _call(lib, **dict(ok, q=None)) == gl.GLA_ERR_NULL
+    assert _call(lib, **dict(ok, out=None)) == gl.GLA_ERR_NULL
+    assert _call(lib, **dict(ok, g=None)) == gl.GLA_ERR_NULL
+    assert _call(lib, **dict(ok, v=FAKE + 8)) == gl.GLA_ERR_ALIGN
+    assert _call(lib, **dict(ok, out=FAKE + 2)) == gl.GLA_ERR_ALIGN
+    assert _call(lib, **dict(ok, s_in=FAKE + 2)) == gl.GLA_ERR_ALIGN
+    # empty batch or heads: nothing to do, no device needed
+    assert _call(lib, B=0, **ok) == gl.GLA_OK
+    assert _call(lib, H=0) == gl.GLA_OK
+
+
+def test_timed_variant_requires_events(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    st = lib.gla_forward_timed(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 1, 16, 32, 1e-6,
+                               None, None)
+    assert st == gl.GLA_ERR_NULL
+
+
+def test_device_fault_rejects_null(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    assert lib.gla_device_fault(None, None) == gl.GLA_ERR_NULL
+
+
+def test_binding_marshalling_errors():
+    import torch
+
+    import gated_linear_attention_frame_b200 as gl
+
+    q = torch.zeros(1, 16, 1, 32, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        gl.gla_forward(q, q, q, None, None, None, q, 1, 1, 1, 16, 32, 1e-6, 0)
+    qb = torch.zeros(1, 16, 1, 32, dtype=torch.bfloat16)  # CPU tensor: not a device pointer
+    g = torch.zeros(1, 1, 1)
+    with pytest.raises(ValueError):
+        gl.gla_forward(qb, qb, qb, g, None, None, qb, 1, 1, 1, 16, 32, 1e-6, 0)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from gated_linear_attention_frame_b200._binding import load_library
+
+    with pytest.raises(ImportError):
+        load_library(str(tmp_path / "libgla.so"))
