@@ -1,0 +1,463 @@
+"""Benchmark of the gated linear attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+One step = one gla_forward call (increment -> gated scan -> output kernels)
+over one batch of the workload, inputs resident in HBM.  With N > 1 (torchrun,
+one process per GPU) every rank runs its own independent copy of the workload
+(heads and sequences are independent: weak scaling, no data-path
+collective); the timed region is bracketed by a barrier and a device
+synchronisation and the time is the maximum over ranks.  Rank 0 prints one
+JSON line.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (one
+(batch, head) slice of the workload per step), on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, make_inputs, make_state  # noqa: E402
+
+METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "720p-5s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture, valid
+# only while the kernel source is unchanged (hash of the .cuh files below).
+NCU_TRAFFIC = {}
+KERNEL_SOURCES = ["gla_increment.cuh", "gla_output.cuh", "gla_scan.cuh", "gla_common.cuh",
+                  "sm100_ptx.cuh", "gla_api.cu"]
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for n in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "gated_linear_attention_frame_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def algorithmic_work(w, state_in: bool, state_out: bool = True) -> dict:
+    """Bytes and flops the layer must move / compute (no workspace traffic).
+    Per token-head: q, k, v read and out written in bf16 = 8d bytes;
+    flops 2d(d+1) (increment) + 2d(d+1) (output) + d (divide).
+    Per (b, h): state_in read / state_out written, d(d+1) fp32 each.
+    Per (b, f, h): one fp32 gate and 2d(d+1) scan flops."""
+    d = w.d
+    th = w.B * w.tokens * w.H
+    bh = w.B * w.H
+    units = w.B * w.frames * w.H
+    k1_bytes = th * 4 * d
+    k3_bytes = th * 4 * d
+    k2_bytes = units * 4 + bh * d * (d + 1) * 4 * (int(state_in) + int(state_out))
+    flops = th * (4 * d * (d + 1) + d) + units * 2 * d * (d + 1)
+    return {"increment": k1_bytes, "scan": k2_bytes, "output": k3_bytes,
+            "bytes": k1_bytes + k2_bytes + k3_bytes, "flops": flops}
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML (read only)
+    in a background thread while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML unavailable: report no clocks
+            self.ok = False
+        self._t = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                pw = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((sm, rs, pw))
+            except Exception:
+                pass
+            self._stop.wait(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self) -> dict | None:
+        if not self.ok:
+            return None
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        sm = [s[0] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= int(s[1])
+        reasons = [n for n, b in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sm), "power_w_max": round(max(s[2] for s in self.samples), 1)}
+
+
+# ------------------------------------------------------------ distributed
+
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def dist_init(world: int, backend: str):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(x: float, dist, device) -> float:
+    """Maximum of a float over ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is None:
+        return
+    if device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+# --------------------------------------------------------------- CPU oracle
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def oracle_head_slices(w, heads, seed_device="cpu"):
+    """Host copies of (q, k, v, g) for the sampled (b, h) slices of call 0."""
+    q, k, v, g = make_inputs(w, device=seed_device)
+    out = []
+    for (b, h) in heads:
+        out.append(tuple(x.cpu() for x in (q[b, :, h], k[b, :, h], v[b, :, h], g[b, :, h])))
+    del q, k, v, g
+    return out
+
+
+def time_oracle(w, budget_s: float, max_heads: int | None = None, device="cpu") -> dict:
+    """Time the fp64 oracle on (b, h) slices of the workload until `budget_s`
+    of CPU work has been done; tokens/s counts full-layer tokens (all heads)."""
+    import oracle
+
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if max_heads:
+        pairs = pairs[:max_heads]
+    slices = oracle_head_slices(w, pairs[: min(len(pairs), 8)], device)
+    s_in = make_state(w)
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        i = done % len(slices)
+        b, h = pairs[i]
+        q, k, v, g = slices[i]
+        oracle.gla_head(q, k, v, g, w.tokens_per_frame,
+                        None if s_in is None else s_in[b, h], w.eps)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 4 * len(pairs):
+            break
+    tokens = done * w.tokens / w.H * 1.0  # head-slices -> full-layer tokens
+    return {"value": tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": "%d (batch, head) slices of %s (%d frames x %d tokens each), fp64 numpy, "
+                      "%.1f s wall" % (done, w.name, w.frames, w.tokens_per_frame, el),
+            "seconds": round(el, 3)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def run_gpu(args, w, dist, rank, local_rank, world):
+    import gated_linear_attention_frame_b200 as gla
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+
+    # inputs: a ring of input sets (fresh frames for the streaming workload)
+    nsets = 4 if w.name == "stream" else 1
+    sets = [make_inputs(w, call=c, device=dev) for c in range(nsets)]
+    state = make_state(w, device=dev)
+    state_buf = state.clone() if state is not None else None
+    out = torch.empty_like(sets[0][0])
+    so = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev, dtype=torch.float32)
+    work = algorithmic_work(w, state_in=state is not None)
+
+    def step(i, events=None):
+        q, k, v, g = sets[i % nsets]
+        s_in = state_buf  # streaming: the state carries from call to call
+        s_out = state_buf if state_buf is not None else so
+        a = (q, k, v, g, s_in, s_out, out, w.B, w.H, w.frames, w.tokens_per_frame, w.d, w.eps,
+             stream)
+        if events is None:
+            gla.gla_forward(*a)
+        else:
+            gla.gla_forward_timed(*a, events)
+
+    warm = max(3, args.warmup)
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert gla.gla_device_fault(stream) == 0
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e4 in evs:
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with clocks:
+        for i in range(K):
+            step(i, evs[i])
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    fault = gla.gla_device_fault(stream)
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                    for e in evs])
+    total_ms = reduce_max(total_ms, dist, dev)
+    ms_step = total_ms / K
+    value = world * w.total_tokens / (ms_step * 1e-3)
+
+    names = ["increment", "scan", "output"]
+    avg = per.mean(axis=0)
+    dom = int(np.argmax(avg))
+    achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
+    traffic = None
+    if NCU_TRAFFIC.get("kernel") == names[dom] and NCU_TRAFFIC.get("src") == kernel_source_hash():
+        traffic = NCU_TRAFFIC.get("bytes_per_launch")
+    roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "peak_source": peaks["source"] + " (hbm_gbs)"}
+    t_roof = max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                 work["flops"] / (peaks["bf16_tflops"] * 1e12))
+    layer = {"algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
+             "roofline_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_step, 4),
+             "achieved_GBps": round(work["bytes"] / (ms_step * 1e-3) / 1e9, 1),
+             "kernel_ms": {n: round(float(a), 4) for n, a in zip(names, avg)}}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        E = max(1, min(K, args.e2e_steps))
+        host = [x.cpu().pin_memory() for x in sets[0]]
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        host_so = torch.empty(so.shape, dtype=so.dtype).pin_memory()
+        dq, dk, dv, dg = (torch.empty_like(x) for x in sets[0])
+        h2d = sum(x.numel() * x.element_size() for x in host)
+        d2h = host_out.numel() * host_out.element_size() + host_so.numel() * 4
+        if state_buf is not None:
+            h2d += state_buf.numel() * 4
+            host_state = state_buf.cpu().pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            for d_, h_ in zip((dq, dk, dv, dg), host):
+                d_.copy_(h_, non_blocking=True)
+            s_in = None
+            if state_buf is not None:
+                state_buf.copy_(host_state, non_blocking=True)
+                s_in = state_buf
+            gla.gla_forward(dq, dk, dv, dg, s_in, so, out, w.B, w.H, w.frames,
+                            w.tokens_per_frame, w.d, w.eps, stream)
+            host_out.copy_(out, non_blocking=True)
+            host_so.copy_(so, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(dist, dev)
+        e0.record(stream)
+        for _ in range(E):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / E
+        e2e = {"value": round(world * w.total_tokens / (e_ms * 1e-3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E,
+               "ms_per_step": round(e_ms, 3)}
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": warm, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.frames,
+                   "tokens_per_frame": w.tokens_per_frame, "tokens_per_step_per_gpu": w.total_tokens,
+                   "state_in": "carried fp32" if state is not None else "zero",
+                   "l2": "inputs larger than L2 (%.2f GB read+written per step); no flush"
+                         % (work["bytes"] / 1e9),
+                   "parallelism": "dp%d (independent sequences per GPU)" % world},
+        "roofline": roof, "layer_roofline": layer, "gpu_launches": 3 * K, "e2e": e2e,
+        "clocks": clocks.summary(), "device_fault": fault,
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+    return res
+
+
+def run_reference(args, w):
+    """fp64 CPU oracle, one (batch, head) slice per step."""
+    import oracle
+
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    slices = oracle_head_slices(w, pairs[:4])
+    s_in = make_state(w)
+
+    def step(i):
+        b, h = pairs[i % 4]
+        q, k, v, g = slices[i % 4]
+        oracle.gla_head(q, k, v, g, w.tokens_per_frame, None if s_in is None else s_in[b, h],
+                        w.eps)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = args.steps * w.tokens / w.H / el
+    sample = ("one (batch, head) slice of %s per step (%d frames x %d tokens), fp64 numpy oracle"
+              % (w.name, w.frames, w.tokens_per_frame))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.frames,
+                   "tokens_per_frame": w.tokens_per_frame},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--frames", type=int, default=0,
+                    help="override the workload's frame count (small profiling cases)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for cpu_baseline (0 = skip)")
+    args = ap.parse_args(argv)
+    w = WORKLOADS[args.workload]
+    if args.frames > 0:
+        w = w.with_(frames=args.frames, name="%s-%dframes" % (w.name, args.frames))
+    rank, local_rank, world = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+
+    if world != args.gpus and world > 1:
+        print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
+    dist = dist_init(world, "nccl")
+    try:
+        res = run_gpu(args, w, dist, rank, local_rank, world)
+        if rank == 0 and world == 1 and args.cpu_budget > 0:
+            res["cpu_baseline"] = time_oracle(w, args.cpu_budget)
+        elif rank == 0:
+            res["cpu_baseline"] = None
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -119,6 +119,9 @@ def gla_forward_timed(q, k, v, gate_logits, state_in, state_out, out, B, H, fram
     (`events`: 4 torch.cuda.Event(enable_timing=True))."""
     _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
     lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the CUDA event at its first record
+            e.record()
     arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
     st = lib.gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in),
                                _ptr(state_out), _ptr(out), int(B), int(H), int(frames),
