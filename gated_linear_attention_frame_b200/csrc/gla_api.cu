@@ -124,7 +124,7 @@ int validate(const Args& a) {
     return GLA_ERR_SHAPE;
   const int64_t elems = static_cast<int64_t>(a.B) * tokens * a.H * a.d;
   const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
-  if (elems > (int64_t(1) << 46)) return GLA_ERR_SHAPE;
+  if (elems > (int64_t(1) << 46) || units > INT32_MAX / 2) return GLA_ERR_SHAPE;
   if (elems > 0 && (a.q == nullptr || a.k == nullptr || a.v == nullptr || a.out == nullptr))
     return GLA_ERR_NULL;
   if (units > 0 && a.g == nullptr) return GLA_ERR_NULL;
@@ -139,6 +139,25 @@ int validate(const Args& a) {
 
 inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
+// Launch as a programmatic dependent of the previous kernel in the stream:
+// the grid may be scheduled before its predecessor finishes and must execute
+// griddepcontrol.wait before reading anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block,
+                             size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int D>
 int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   using G = Geo<D>;
@@ -147,6 +166,7 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   const int64_t W = units * tpu;
   const int32_t G1 = static_cast<int32_t>(W < di.sms ? W : di.sms);
   const int32_t G3 = G1;
+  const gla::WorkPlan wp = W > 0 ? gla::WorkPlan::make(units, tpu, G1) : gla::WorkPlan{};
 
   const int64_t partial_bytes =
       W > 0 ? align256((units + G1) * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4) : 0;
@@ -184,24 +204,31 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
 
   record(0);
   if (W > 0 && status == GLA_OK) {
-    gla::IncParams ip{partial, a.H, a.F, tpu, W};
+    gla::IncParams ip{partial, wp, a.H, a.F};
     gla::gla_increment_kernel<D>
         <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
     check();
   }
   record(1);
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
-    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, a.H, a.F, tpu, W, G1};
-    constexpr int NT = (D + 1) * (D / 8);
-    const unsigned grid = static_cast<unsigned>((NT + 255) / 256) * static_cast<unsigned>(a.B * a.H);
-    gla::gla_scan_kernel<D><<<grid, 256, 0, a.stream>>>(sp);
+    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, wp, a.H, a.F, tpu};
+    using SC = gla::ScanCfg<D>;
+    const unsigned grid = static_cast<unsigned>(SC::kGroups) * static_cast<unsigned>(a.B * a.H);
+    // Few blocks per SM (long sequences, few heads): keep more frames of
+    // loads in flight per thread; otherwise fewer registers, more blocks.
+    const bool deep = grid <= 2u * static_cast<unsigned>(di.sms);
+    const cudaError_t e =
+        deep ? launch_dependent(gla::gla_scan_kernel<D, 4>, grid, SC::kBlock, 0, a.stream, sp)
+             : launch_dependent(gla::gla_scan_kernel<D, 2>, grid, SC::kBlock, 0, a.stream, sp);
+    if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
   }
   record(2);
   if (W > 0 && status == GLA_OK) {
-    gla::OutParams op{image, a.eps, a.H, a.F, a.T, tpu, W};
-    gla::gla_output_kernel<D>
-        <<<G3, gla::OutCfg<D>::kThreads, gla::OutCfg<D>::kSmemBytes, a.stream>>>(tm_q, tm_out, op);
+    gla::OutParams op{image, a.eps, wp, a.H, a.F, a.T};
+    if (launch_dependent(gla::gla_output_kernel<D>, G3, gla::OutCfg<D>::kThreads,
+                         gla::OutCfg<D>::kSmemBytes, a.stream, tm_q, tm_out, op) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
     check();
   }
   record(3);

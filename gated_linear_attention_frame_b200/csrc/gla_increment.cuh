@@ -11,12 +11,13 @@
 // swizzle; ReLU is applied in shared memory between the TMA landing and the
 // MMA, and the same pass sums phi(K) over tokens for the normaliser column.
 //
-// Work split: the units' token tiles (W = units * ceil(T / 128)) are divided
-// into contiguous ranges, one per persistent CTA.  A CTA accumulates the
-// tiles of one unit in TMEM and, when the unit or its range ends, writes an
-// fp32 partial [d + 4][d] (transposed: row j = value column, column i = key
-// feature; rows d..d+3 = the four ReLU warps' normaliser sums) to slot
-// (u + cta).  The scan kernel sums a unit's partials.
+// Work split: the token tiles of all units go to the persistent CTAs as the
+// WorkPlan describes (whole units in full rounds, then a contiguous split of
+// the remainder).  A CTA accumulates the tiles of one unit in TMEM and, when
+// the unit or its share of it ends, writes an fp32 partial [d + 1][d]
+// (transposed: row j = value column, column i = key feature; row d = the
+// normaliser column, the four ReLU warps' sums added in a fixed order) to the
+// plan's slot.  The scan kernel sums a unit's partials.
 //
 // Warp roles (320 threads): warps 0-3 drain TMEM (epilogue), warps 4-7 apply
 // ReLU, warp 8 issues TMA, warp 9 issues MMAs.
@@ -36,18 +37,27 @@ struct IncCfg {
   static constexpr int kVBytes = G::kTileBytes;
   static constexpr int kStageBytes = kABytes + kVBytes;
   static constexpr int kTmemCols = 2 * D;                       // two fp32 accumulators of N = D
-  static constexpr int kPartialRows = D + 4;
+  static constexpr int kPartialRows = D + 1;
   static constexpr int kPartialFloats = kPartialRows * D;
   static constexpr int kThreads = 320;
-  static constexpr int kBarBytes = (3 * kStages + 5) * 8;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
+  static constexpr int kBarBytes = (3 * kStages + 7) * 8;
+  static constexpr int kZBytes = 4 * D * 4;  // per-ReLU-warp normaliser sums
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kZBytes + kBarBytes + 16;
 };
 
 struct IncParams {
-  float* partial;   // [(units + gridDim.x) slots][d + 4][d] fp32
-  int H, F, tpu;    // heads, frames, token tiles per frame
-  int64_t W;        // units * tpu
+  float* partial;   // [(units + gridDim.x) slots][d + 1][d] fp32
+  WorkPlan wp;      // tile assignment (gridDim.x == wp.G)
+  int H, F;         // heads, frames
 };
+
+// (b, f, h) of unit u = (b * F + f) * H + h.
+__device__ __forceinline__ void unit_coords(int32_t u, int H, int F, int& b, int& f, int& h) {
+  h = u % H;
+  const int32_t bf = u / H;
+  f = bf % F;
+  b = bf / F;
+}
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned int code) {
@@ -72,7 +82,8 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  float* zpart = reinterpret_cast<float*>(smem + S * C::kStageBytes);  // [4][D]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kZBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
@@ -80,17 +91,17 @@ __global__ void __launch_bounds__(320, 1)
   auto accf = [&](int a) { return bar0 + 8u * (3 * S + a); };
   auto acce = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (3 * S + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  const uint32_t zfull = bar0 + 8u * (3 * S + 5);  // 4 ReLU warps wrote zpart
+  const uint32_t zfree = bar0 + 8u * (3 * S + 6);  // warp 4 consumed zpart
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 7);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto a_buf = [&](int s) { return sbase + s * C::kStageBytes; };
   auto v_buf = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TileSplit split{p.W, static_cast<int32_t>(gridDim.x)};
-  const int64_t lo = split.lo(blockIdx.x);
-  const int64_t hi = split.lo(blockIdx.x + 1);
-  const int tpu = p.tpu;
+  TileCursor cur;
+  cur.init(p.wp, blockIdx.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -103,6 +114,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(acce(a), 4);
     }
     mbar_init(done_bar, 1);
+    mbar_init(zfull, 4);
+    mbar_init(zfree, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -130,16 +143,13 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       int64_t issued = 0;
-      for (int64_t x = lo; x < hi; ++x, ++issued) {
+      int b = 0, f = 0, h = 0;
+      for (; cur.valid(); cur.advance(), ++issued) {
         const int s = static_cast<int>(issued % S);
         const uint32_t ph = static_cast<uint32_t>((issued / S) & 1);
         if (!mbar_wait(empty(s), ph ^ 1u, abort, kCode)) break;
-        const int64_t u = x / tpu;
-        const int t = static_cast<int>(x - u * tpu);
-        const int h = static_cast<int>(u % p.H);
-        const int64_t bf = u / p.H;
-        const int f = static_cast<int>(bf % p.F);
-        const int b = static_cast<int>(bf / p.F);
+        if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+        const int t = cur.t;
         mbar_arrive_expect_tx(full(s), 2u * G::kTileBytes);
 #pragma unroll
         for (int a = 0; a < G::kAtoms; ++a) {
@@ -158,11 +168,9 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
       int64_t i = 0, seg = 0;
-      for (int64_t x = lo; x < hi; ++x, ++i) {
-        const int64_t u = x / tpu;
-        const int t = static_cast<int>(x - u * tpu);
-        const bool first = (x == lo) || (t == 0);
-        const bool last = (x == hi - 1) || (t == tpu - 1);
+      for (; cur.valid(); cur.advance(), ++i) {
+        const bool first = cur.first;
+        const bool last = cur.last;
         const int ab = static_cast<int>(seg & 1);
         if (first && !mbar_wait(acce(ab), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort, kCode))
           break;
@@ -200,7 +208,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
     for (int e = 0; e < 8; ++e) z[e] = 0.f;
     int64_t i = 0;
-    for (int64_t x = lo; x < hi; ++x, ++i) {
+    uint32_t zround = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
       if (!warp_wait(full(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
       const uint32_t base = a_buf(s) + off0;
@@ -222,20 +231,32 @@ __global__ void __launch_bounds__(320, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(relu_done(s));
-      const int64_t u = x / tpu;
-      const int t = static_cast<int>(x - u * tpu);
-      if (x == hi - 1 || t == tpu - 1) {
-        // Unit range ends: this warp's column sums of phi(K) go to row d + (warp - 4).
+      if (cur.last) {
+        // Unit range ends: the column sums of phi(K) become row d of the
+        // partial.  Each warp reduces its lanes, parks its sums in zpart[warp];
+        // warp 4 adds the four in a fixed order and writes the row.
 #pragma unroll
         for (int o = CPR; o < 32; o <<= 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) z[e] += __shfl_xor_sync(0xffffffffu, z[e], o);
+        if (zround > 0 && !warp_wait(zfree, (zround - 1) & 1u, abort, kCode)) break;
         if (lane < CPR) {
-          float* dst = p.partial + (u + blockIdx.x) * static_cast<int64_t>(C::kPartialFloats) +
-                       static_cast<int64_t>(D + warp - 4) * D + lane * 8;
-          reinterpret_cast<float4*>(dst)[0] = make_float4(z[0], z[1], z[2], z[3]);
-          reinterpret_cast<float4*>(dst)[1] = make_float4(z[4], z[5], z[6], z[7]);
+          float4* zp = reinterpret_cast<float4*>(zpart + (warp - 4) * D + lane * 8);
+          zp[0] = make_float4(z[0], z[1], z[2], z[3]);
+          zp[1] = make_float4(z[4], z[5], z[6], z[7]);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zfull);
+        if (warp == 4) {
+          if (!warp_wait(zfull, zround & 1u, abort, kCode)) break;
+          float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) +
+                       static_cast<int64_t>(D) * D;
+          for (int col = lane; col < D; col += 32)
+            dst[col] = ((zpart[col] + zpart[D + col]) + zpart[2 * D + col]) + zpart[3 * D + col];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(zfree);
+        }
+        ++zround;
 #pragma unroll
         for (int e = 0; e < 8; ++e) z[e] = 0.f;
       }
@@ -245,14 +266,13 @@ __global__ void __launch_bounds__(320, 1)
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // key feature i
     int64_t seg = 0;
-    for (int64_t x = lo; x < hi; ++seg) {
-      const int64_t u = x / tpu;
-      const int64_t xe = ((u + 1) * tpu < hi) ? (u + 1) * tpu : hi;
+    for (; cur.valid(); cur.advance()) {
+      if (!cur.last) continue;
       const int ab = static_cast<int>(seg & 1);
       if (!warp_wait(accf(ab), static_cast<uint32_t>((seg >> 1) & 1), abort, kCode)) break;
       tc_fence_after();
       if (q4 * 32 < D) {
-        float* dst = p.partial + (u + blockIdx.x) * static_cast<int64_t>(C::kPartialFloats) + row;
+        float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) + row;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
@@ -265,7 +285,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce(ab));
-      x = xe;
+      ++seg;
     }
   }
 

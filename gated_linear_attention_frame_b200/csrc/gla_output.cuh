@@ -41,8 +41,8 @@ struct OutCfg {
 struct OutParams {
   const uint8_t* image;  // [units][Geo<D>::kImageBytes] bf16 S_f^T images
   float eps;
-  int H, F, T, tpu;
-  int64_t W;
+  WorkPlan wp;           // tile assignment (gridDim.x == wp.G)
+  int H, F, T;
 };
 
 template <int D>
@@ -79,10 +79,8 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TileSplit split{p.W, static_cast<int32_t>(gridDim.x)};
-  const int64_t lo = split.lo(blockIdx.x);
-  const int64_t hi = split.lo(blockIdx.x + 1);
-  const int tpu = p.tpu;
+  TileCursor cur;
+  cur.init(p.wp, blockIdx.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -129,10 +127,27 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       int64_t issued = 0, seg = 0;
-      for (int64_t x = lo; x < hi; ++x, ++issued) {
-        const int64_t u = x / tpu;
-        const int t = static_cast<int>(x - u * tpu);
-        if (x == lo || t == 0) {
+      bool waited = false;
+      int b = 0, f = 0, h = 0;
+      for (; cur.valid(); cur.advance(), ++issued) {
+        const int64_t u = cur.u;
+        const int t = cur.t;
+        const int s = static_cast<int>(issued % S);
+        if (!mbar_wait(qempty(s), static_cast<uint32_t>(((issued / S) & 1) ^ 1), abort, kCode))
+          break;
+        if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+        mbar_arrive_expect_tx(qfull(s), G::kTileBytes);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a)
+          tma_load_5d(q_buf(s) + a * G::kAtomTileBytes, &tm_q, qfull(s), a * G::kAtomElems, h,
+                      t * kTileTokens, f, b);
+        if (cur.first) {
+          if (!waited) {
+            // q is a caller input; the state images come from the scan kernel,
+            // which this grid may have started alongside.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+          }
           const int sb = static_cast<int>(seg & 1);
           if (!mbar_wait(sempty(sb), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort, kCode))
             break;
@@ -144,18 +159,6 @@ __global__ void __launch_bounds__(320, 1)
                       G::kImageAtomBytes, sfull(sb));
           ++seg;
         }
-        const int s = static_cast<int>(issued % S);
-        if (!mbar_wait(qempty(s), static_cast<uint32_t>(((issued / S) & 1) ^ 1), abort, kCode))
-          break;
-        const int h = static_cast<int>(u % p.H);
-        const int64_t bf = u / p.H;
-        const int f = static_cast<int>(bf % p.F);
-        const int b = static_cast<int>(bf / p.F);
-        mbar_arrive_expect_tx(qfull(s), G::kTileBytes);
-#pragma unroll
-        for (int a = 0; a < G::kAtoms; ++a)
-          tma_load_5d(q_buf(s) + a * G::kAtomTileBytes, &tm_q, qfull(s), a * G::kAtomElems, h,
-                      t * kTileTokens, f, b);
       }
       for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
         mbar_wait_drain(qfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
@@ -169,11 +172,9 @@ __global__ void __launch_bounds__(320, 1)
       constexpr int KPA = G::kAtomElems / 16;  // 16-wide K steps per swizzle row
       int64_t i = 0, seg = 0;
       int sb = 0;
-      for (int64_t x = lo; x < hi; ++x, ++i) {
-        const int64_t u = x / tpu;
-        const int t = static_cast<int>(x - u * tpu);
-        const bool first = (x == lo) || (t == 0);
-        const bool last = (x == hi - 1) || (t == tpu - 1);
+      for (; cur.valid(); cur.advance(), ++i) {
+        const bool first = cur.first;
+        const bool last = cur.last;
         if (first) {
           sb = static_cast<int>(seg & 1);
           if (!mbar_wait(sfull(sb), static_cast<uint32_t>((seg >> 1) & 1), abort, kCode)) break;
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t off0 =
         (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes + G::swz(r0, c % CPA) * 16;
     int64_t i = 0;
-    for (int64_t x = lo; x < hi; ++x, ++i) {
+    for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
       if (!warp_wait(qfull(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
       const uint32_t base = q_buf(s) + off0;
@@ -234,7 +235,8 @@ __global__ void __launch_bounds__(320, 1)
     const int row = q4 * 32 + lane;  // token within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     int64_t i = 0;
-    for (int64_t x = lo; x < hi; ++x, ++i) {
+    int b = 0, f = 0, h = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
       const int ab = static_cast<int>(i & 1);
       if (!warp_wait(accf(ab), static_cast<uint32_t>((i >> 1) & 1), abort, kCode)) break;
       tc_fence_after();
@@ -243,13 +245,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld_1col(tb + D, dr);
       tmem_wait_ld();
       const float rinv = 1.0f / (__uint_as_float(dr) + p.eps);
-      const int64_t u = x / tpu;
-      const int t = static_cast<int>(x - u * tpu);
-      const int h = static_cast<int>(u % p.H);
-      const int64_t bf = u / p.H;
-      const int f = static_cast<int>(bf % p.F);
-      const int b = static_cast<int>(bf / p.F);
-      const int tok0 = t * kTileTokens + q4 * 32;  // first token of this warp's rows
+      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+      const int tok0 = cur.t * kTileTokens + q4 * 32;  // first token of this warp's rows  // first token of this warp's rows
 #pragma unroll
       for (int a = 0; a < G::kAtoms; ++a) {
         const int buf = static_cast<int>((i * G::kAtoms + a) & 1);

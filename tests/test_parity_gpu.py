@@ -95,6 +95,11 @@ SMALL = [
     (1, 3, 7, 255, 128, True),
     (2, 1, 3, 1000, 128, False),
     (1, 2, 9, 77, 64, True),
+    # schedule edges on 148 SMs: a tail of one unit, an exact multiple of the
+    # CTA count, a tail with fewer tiles than CTAs
+    (1, 149, 1, 200, 64, True),
+    (2, 37, 4, 130, 32, False),
+    (1, 150, 1, 1, 32, False),
 ]
 
 
