@@ -8,6 +8,7 @@ from ._binding import (  # noqa: F401
     GLA_ERR_DEVICE,
     GLA_ERR_LAUNCH,
     GLA_ERR_NULL,
+    GLA_ERR_SCRATCH,
     GLA_ERR_SHAPE,
     GLA_ERR_UNSUPPORTED_D,
     GLA_OK,
@@ -16,7 +17,9 @@ from ._binding import (  # noqa: F401
     gla_device_fault,
     gla_error_string,
     gla_forward,
+    gla_forward_noalloc,
     gla_forward_timed,
+    gla_noalloc_scratch_bytes,
     gla_version,
     load_library,
 )

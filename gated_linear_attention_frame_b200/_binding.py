@@ -23,9 +23,10 @@ GLA_ERR_UNSUPPORTED_D = 4
 GLA_ERR_ALLOC = 5
 GLA_ERR_LAUNCH = 6
 GLA_ERR_DEVICE = 7
+GLA_ERR_SCRATCH = 8
 
-EXPORTED = ("gla_forward", "gla_forward_timed", "gla_error_string", "gla_device_fault",
-            "gla_version")
+EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
+            "gla_error_string", "gla_device_fault", "gla_version")
 
 
 class GLAError(RuntimeError):
@@ -54,6 +55,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward.restype = i32
     lib.gla_forward_timed.argtypes = fwd + [ctypes.POINTER(vp)]
     lib.gla_forward_timed.restype = i32
+    lib.gla_forward_noalloc.argtypes = fwd
+    lib.gla_forward_noalloc.restype = i32
+    lib.gla_noalloc_scratch_bytes.argtypes = []
+    lib.gla_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.gla_error_string.argtypes = [i32]
     lib.gla_error_string.restype = ctypes.c_char_p
     lib.gla_device_fault.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -129,6 +134,25 @@ def gla_forward_timed(q, k, v, gate_logits, state_in, state_out, out, B, H, fram
                                ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
     if st != GLA_OK:
         raise GLAError(st, "gla_forward_timed")
+
+
+def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
+                        tokens_per_frame, d, eps, stream=None) -> None:
+    """gla_forward with its workspace in the library's fixed device scratch
+    array instead of a fresh allocation (see include/gla.h).  For callers
+    that must not allocate device memory; problems whose workspace exceeds
+    gla_noalloc_scratch_bytes() raise GLAError(GLA_ERR_SCRATCH)."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    st = lib.gla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in),
+                                 _ptr(state_out), _ptr(out), int(B), int(H), int(frames),
+                                 int(tokens_per_frame), int(d), float(eps), _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_noalloc")
+
+
+def gla_noalloc_scratch_bytes() -> int:
+    return int(load_library().gla_noalloc_scratch_bytes())
 
 
 def gla_error_string(status: int) -> str:

@@ -31,6 +31,19 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int major = 0;
+  void* scratch = nullptr;  // device address of g_gla_scratch (gla_forward_noalloc)
+};
+
+// Fixed scratch of gla_forward_noalloc: a file-scope device array that every
+// device which loads this library holds until the process exits.  In host
+// code its name is only a stand-in; the kernels get the device address that
+// cudaGetSymbolAddress returns for the current device.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_gla_scratch[kNoAllocScratchBytes];
+
+struct FixedScratch {
+  uint8_t* ptr;
+  size_t bytes;
 };
 
 std::mutex g_mu;
@@ -159,7 +172,8 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned b
 }
 
 template <int D>
-int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
+int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
+        const FixedScratch* fixed = nullptr) {
   using G = Geo<D>;
   const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
   const int tpu = (a.T + gla::kTileTokens - 1) / gla::kTileTokens;
@@ -183,7 +197,10 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
 
   uint8_t* ws = nullptr;
-  if (ws_bytes > 0) {
+  if (fixed != nullptr) {
+    if (static_cast<size_t>(ws_bytes) > fixed->bytes) return GLA_ERR_SCRATCH;
+    ws = ws_bytes > 0 ? fixed->ptr : nullptr;
+  } else if (ws_bytes > 0) {
     if (cudaMallocAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), a.stream) !=
         cudaSuccess) {
       cudaGetLastError();
@@ -232,7 +249,7 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
     check();
   }
   record(3);
-  if (ws != nullptr && cudaFreeAsync(ws, a.stream) != cudaSuccess) {
+  if (fixed == nullptr && ws != nullptr && cudaFreeAsync(ws, a.stream) != cudaSuccess) {
     cudaGetLastError();
     if (status == GLA_OK) status = GLA_ERR_LAUNCH;
   }
@@ -249,6 +266,41 @@ int forward_impl(const Args& a, cudaEvent_t* ev) {
     case 32: return run<32>(a, di, ev);
     case 64: return run<64>(a, di, ev);
     default: return run<128>(a, di, ev);
+  }
+}
+
+// One-time per-device lookup of g_gla_scratch's device address, made with
+// that device current (the caller's current device).
+int noalloc_setup(DeviceInfo* out) {
+  int st = device_setup(out);
+  if (st != GLA_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GLA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.scratch == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gla_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return GLA_ERR_LAUNCH;
+    }
+    di.scratch = p;
+  }
+  *out = di;
+  return GLA_OK;
+}
+
+int forward_noalloc_impl(const Args& a) {
+  int st = validate(a);
+  if (st != GLA_OK) return st;
+  if (static_cast<int64_t>(a.B) * a.H == 0) return GLA_OK;
+  DeviceInfo di;
+  if ((st = noalloc_setup(&di)) != GLA_OK) return st;
+  const FixedScratch fs{static_cast<uint8_t*>(di.scratch), kNoAllocScratchBytes};
+  switch (a.d) {
+    case 32: return run<32>(a, di, nullptr, &fs);
+    case 64: return run<64>(a, di, nullptr, &fs);
+    default: return run<128>(a, di, nullptr, &fs);
   }
 }
 
@@ -274,6 +326,16 @@ int gla_forward_timed(const void* q, const void* k, const void* v, const float* 
   return forward_impl(a, events);
 }
 
+int gla_forward_noalloc(const void* q, const void* k, const void* v, const float* gate_logits,
+                        const float* state_in, float* state_out, void* out, int B, int H,
+                        int frames, int tokens_per_frame, int d, float eps, cudaStream_t stream) {
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream};
+  return forward_noalloc_impl(a);
+}
+
+size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
 const char* gla_error_string(int status) {
   switch (status) {
     case GLA_OK: return "ok";
@@ -284,6 +346,8 @@ const char* gla_error_string(int status) {
     case GLA_ERR_ALLOC: return "workspace allocation failed";
     case GLA_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
     case GLA_ERR_DEVICE: return "no CUDA device of compute capability 10.x";
+    case GLA_ERR_SCRATCH:
+      return "problem needs more scratch than gla_forward_noalloc's fixed 32 MiB buffer";
     default: return "unknown status";
   }
 }

@@ -52,7 +52,8 @@ typedef enum {
   GLA_ERR_UNSUPPORTED_D = 4,   /* d not in {32, 64, 128} */
   GLA_ERR_ALLOC = 5,           /* stream-ordered workspace allocation failed */
   GLA_ERR_LAUNCH = 6,          /* a CUDA runtime call or kernel launch failed */
-  GLA_ERR_DEVICE = 7           /* no CUDA device, or not compute capability 10.x */
+  GLA_ERR_DEVICE = 7,          /* no CUDA device, or not compute capability 10.x */
+  GLA_ERR_SCRATCH = 8          /* gla_forward_noalloc: problem exceeds the fixed scratch */
 } gla_status;
 
 /*
@@ -104,6 +105,45 @@ int gla_forward_timed(const void* q, const void* k, const void* v,
                       void* out,
                       int B, int H, int frames, int tokens_per_frame, int d,
                       float eps, cudaStream_t stream, cudaEvent_t* events);
+
+/*
+ * gla_forward_noalloc -- gla_forward that allocates no device memory.
+ *
+ * No counterpart in the paper: this is a deployment variant.  Some callers
+ * cannot allocate device memory while they run the layer: a serving process
+ * whose own allocator reserves all free HBM at start-up (so a library
+ * cudaMallocAsync fails or fragments that reserve), or a per-frame streaming
+ * loop that must not enter the CUDA allocator, whose calls can block and
+ * whose failures are hard to recover from mid-stream.  This entry point takes
+ * the same arguments and computes the same result as gla_forward, with its
+ * workspace in a fixed 32 MiB device array inside the library instead.
+ *
+ *   - Limit: the workspace must fit in 32 MiB (gla_noalloc_scratch_bytes()),
+ *     i.e. about (B*H*frames*6 + #SMs*4)*(d+1)*d bytes <= 32 MiB.  At d = 128
+ *     on a 148-SM B200 that is up to 240 (batch, frame, head) units per call,
+ *     e.g. the one-frame streaming step of 8 sequences x 24 heads.  Larger
+ *     problems return GLA_ERR_SCRATCH and nothing is enqueued.
+ *   - The array exists on every device that loads the library, until exit.
+ *   - The first call on each device performs a one-time set-up (it looks up
+ *     the array's device address with that device current, and sets kernel
+ *     attributes); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Nothing in it needs to start at zero: every byte the kernels read was
+ *     written earlier in the same call.  Calls that overlap on the GPU (for
+ *     example on two streams at once) race on the array and give wrong
+ *     results: serialise them.
+ *   - Never calls cudaMalloc, cudaMallocAsync, cudaFree or any allocating
+ *     routine.  Returns the gla_forward codes plus GLA_ERR_SCRATCH.
+ */
+int gla_forward_noalloc(const void* q, const void* k, const void* v,
+                        const float* gate_logits,
+                        const float* state_in, float* state_out,
+                        void* out,
+                        int B, int H, int frames, int tokens_per_frame, int d,
+                        float eps, cudaStream_t stream);
+
+/* Size in bytes of gla_forward_noalloc's fixed scratch array.  Host only. */
+size_t gla_noalloc_scratch_bytes(void);
 
 /* Static string for a gla_status code (never NULL). Host only, no CUDA call. */
 const char* gla_error_string(int status);

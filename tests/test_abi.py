@@ -46,11 +46,11 @@ def test_error_strings(lib):
     import gated_linear_attention_frame_b200 as g
 
     seen = set()
-    for st in range(0, 8):
+    for st in range(0, 9):
         s = g.gla_error_string(st)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 8
+    assert len(seen) == 9
     assert g.gla_error_string(99) == "unknown status"
     assert g.gla_version() >= 100
 
