@@ -56,9 +56,12 @@ cudaError_t set_smem_attrs() {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        gla::IncCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(gla::gla_output_kernel<D>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gla::OutCfg<D>::kSmemBytes);
+  e = cudaFuncSetAttribute(gla::gla_output_kernel<D>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::OutCfg<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gla::gla_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gla::ScanCfg<D>::kSmemBytes);
 }
 
 // Per-device one-time set-up: SM count, architecture check, kernel attributes,
@@ -231,12 +234,8 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
     gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, wp, a.H, a.F, tpu};
     using SC = gla::ScanCfg<D>;
     const unsigned grid = static_cast<unsigned>(SC::kGroups) * static_cast<unsigned>(a.B * a.H);
-    // Few blocks per SM (long sequences, few heads): keep more frames of
-    // loads in flight per thread; otherwise fewer registers, more blocks.
-    const bool deep = grid <= 2u * static_cast<unsigned>(di.sms);
-    const cudaError_t e =
-        deep ? launch_dependent(gla::gla_scan_kernel<D, 4>, grid, SC::kBlock, 0, a.stream, sp)
-             : launch_dependent(gla::gla_scan_kernel<D, 2>, grid, SC::kBlock, 0, a.stream, sp);
+    const cudaError_t e = launch_dependent(gla::gla_scan_kernel<D>, grid, SC::kThreads,
+                                           SC::kSmemBytes, a.stream, sp);
     if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
   }

@@ -13,12 +13,13 @@
 //   * writes S_f^T rounded to bf16 into the swizzled K-major image that the
 //     output kernel bulk-copies into shared memory as its B operand.
 // After the last frame it writes state_out in the caller's [d][d+1] layout.
-// Each thread keeps the partial loads of its next kAhead frames (up to two
-// partials per frame, the common case) in flight in registers, issued before
-// the current frame is consumed.  Which increment CTAs hold a unit's partials
-// is tabulated once per block and chunk of frames in shared memory.  state_in
-// and state_out, stored [d][d+1] by the caller, are moved through a shared-
-// memory tile so that global accesses are row-contiguous.
+// A producer warp streams each frame's partial increments into a ring of
+// shared-memory stages with plain bulk copies (one copy per partial: the
+// block's rows of it are contiguous), so several frames are in flight without
+// holding them in registers; eight consumer warps take one stage per frame.
+// Which increment CTAs hold a unit's partials travels with the stage.
+// state_in and state_out, stored [d][d+1] by the caller, are moved through a
+// shared-memory tile so that global accesses run along rows.
 #pragma once
 
 #include "gla_common.cuh"
@@ -40,10 +41,15 @@ struct ScanParams {
 template <int D>
 struct ScanCfg {
   static constexpr int kOcts = D / 8;                          // 8-float chunks per state row
-  static constexpr int kBlock = 256;
-  static constexpr int kRows = kBlock / kOcts;                  // state rows per block
+  static constexpr int kConsumers = 256;                        // 8 consumer warps
+  static constexpr int kThreads = kConsumers + 32;              // + 1 producer warp
+  static constexpr int kRows = kConsumers / kOcts;              // state rows per block
   static constexpr int kGroups = (D + 1 + kRows - 1) / kRows;   // blocks per (b, h)
-  static constexpr int kChunk = 256;                            // frames tabulated at once
+  static constexpr int kStages = 3;
+  static constexpr int kSlotBytes = kRows * D * 4;              // one partial's rows: 8 KB
+  static constexpr int kStageBytes = 2 * kSlotBytes + 16;       // two partials + header
+  static constexpr int kTileBytes = kRows * (D + 1) * 4;        // state_in / state_out tile
+  static constexpr int kSmemBytes = 128 + kStages * kStageBytes + kTileBytes + 2 * kStages * 8 + 16;
 };
 
 __device__ __forceinline__ void add8(float (&acc)[8], const float4& a, const float4& b) {
@@ -51,134 +57,141 @@ __device__ __forceinline__ void add8(float (&acc)[8], const float4& a, const flo
   acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
 }
 
-// Grid: kGroups blocks of 256 threads per (b, h), flattened; block g owns
+// Grid: kGroups blocks of 288 threads per (b, h), flattened; block g owns
 // state rows j in [g*kRows, (g+1)*kRows) (row d = normaliser).  Launched as a
 // programmatic dependent of the increment kernel: only caller inputs
-// (state_in, gate logits) are read before griddepcontrol.wait.
-template <int D, int kAhead>
-__global__ void __launch_bounds__(256, (kAhead <= 2) ? 3 : 2) gla_scan_kernel(const ScanParams p) {
+// (state_in) are read before griddepcontrol.wait.
+template <int D>
+__global__ void __launch_bounds__(288) gla_scan_kernel(const ScanParams p) {
   using G = Geo<D>;
   using C = ScanCfg<D>;
   constexpr int PF = IncCfg<D>::kPartialFloats;
-  __shared__ int2 slot_tab[C::kChunk];  // per frame: slots u + x .. u + y of the unit
-  __shared__ __align__(16) float st[C::kRows][D + 1];      // state tile [j - j0][i]
+  constexpr int S = C::kStages;
+  constexpr unsigned kCode = 4u;
 
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~uintptr_t(127));
+  auto stage = [&](int s) { return smem + s * C::kStageBytes; };  // [slot0 | slot1 | header]
+  float(*st)[D + 1] = reinterpret_cast<float(*)[D + 1]>(smem + S * C::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kTileBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 2 * S);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x / C::kGroups;
   const int j0 = (blockIdx.x % C::kGroups) * C::kRows;
-  const int r = threadIdx.x / C::kOcts;
-  const int c = threadIdx.x % C::kOcts;  // key features 8c .. 8c+7
-  const int j = j0 + r;                  // value column (j == D: normaliser)
-  const bool active = j <= D;
   const int nrows = (D + 1 - j0 < C::kRows) ? D + 1 - j0 : C::kRows;
+  const int r = threadIdx.x / C::kOcts;  // consumer: row within the block
+  const int c = threadIdx.x % C::kOcts;  // consumer: key features 8c .. 8c+7
+  const int j = j0 + r;                  // value column (j == D: normaliser)
+  const bool consumer = warp < 8;
+  const bool active = consumer && r < nrows;
   const int b = bh / p.H;
   const int h = bh - b * p.H;
   const int64_t u0 = static_cast<int64_t>(b) * p.F * p.H + h;  // unit of frame 0; frame f: + f*H
   const int64_t srow = static_cast<int64_t>(bh) * D * (D + 1);  // this (b, h)'s state
 
-  // state_in -> registers, through the shared tile (global reads along j)
-  float S[8];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 8);
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
   if (p.state_in != nullptr) {
-    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kBlock) {
+    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kThreads) {
       const int jj = idx % C::kRows, i = idx / C::kRows;
       if (jj < nrows) st[jj][i] = p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jj];
     }
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < 8; ++e) S[e] = active ? st[r][c * 8 + e] : 0.f;
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) S[e] = 0.f;
   }
+  __syncthreads();
+  float S8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) S8[e] = (active && p.state_in != nullptr) ? st[r][c * 8 + e] : 0.f;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
 
-  const float* col = p.partial + static_cast<int64_t>(j) * D + c * 8;
-  constexpr int CPA = G::kAtomElems / 8;
-  const int64_t img_off = (c / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
-                          G::swz(j, c % CPA) * 16;
-  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  bool waited = false;
-
-  for (int fc = 0; fc < p.F; fc += C::kChunk) {
-    const int nf = (p.F - fc < C::kChunk) ? p.F - fc : C::kChunk;
-    __syncthreads();  // the previous chunk's table is no longer read
-    if (p.tpu > 0) {
-      for (int k = threadIdx.x; k < nf; k += C::kBlock) {
+  const bool stream_partials = p.tpu > 0 && p.F > 0;
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && stream_partials) {
+      const uint32_t bytes = static_cast<uint32_t>(nrows) * D * 4;
+      int f = 0;
+      for (; f < p.F; ++f) {
+        const int s = f % S;
+        if (!mbar_wait(empty(s), static_cast<uint32_t>(((f / S) & 1) ^ 1), abort, kCode)) break;
+        const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
         int32_t c0, c1;
-        p.wp.slot_range(u0 + static_cast<int64_t>(fc + k) * p.H, c0, c1);
-        slot_tab[k] = make_int2(c0, c1);
+        p.wp.slot_range(u, c0, c1);
+        int2* hdr = reinterpret_cast<int2*>(stage(s) + 2 * C::kSlotBytes);
+        *hdr = make_int2(c0, c1);
+        const float* src = p.partial + (u + c0) * PF + static_cast<int64_t>(j0) * D;
+        mbar_arrive_expect_tx(full(s), (c1 > c0 ? 2u : 1u) * bytes);
+        bulk_load(smem_u32(stage(s)), src, bytes, full(s));
+        if (c1 > c0) bulk_load(smem_u32(stage(s)) + C::kSlotBytes, src + PF, bytes, full(s));
       }
+      for (int k = (f > S ? f - S : 0); k < f; ++k)
+        mbar_wait_drain(full(k % S), static_cast<uint32_t>((k / S) & 1));
     }
-    __syncthreads();
-    if (!waited) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
-      waited = true;
-    }
-    if (!active) continue;
-
-    // Loads of frame fc + k: slot c0 and, if the unit was split, c0 + 1.
-    auto issue = [&](int k, float4 (&x)[4]) {
-      if (p.tpu == 0) {
-        x[0] = x[1] = x[2] = x[3] = zero4;
-        return;
-      }
-      const int64_t u = u0 + static_cast<int64_t>(fc + k) * p.H;
-      const int2 cr = slot_tab[k];
-      const float4* s0 = reinterpret_cast<const float4*>(col + (u + cr.x) * PF);
-      x[0] = __ldg(s0);
-      x[1] = __ldg(s0 + 1);
-      if (cr.y > cr.x) {
-        x[2] = __ldg(s0 + PF / 4);
-        x[3] = __ldg(s0 + PF / 4 + 1);
-      } else {
-        x[2] = x[3] = zero4;
-      }
-    };
-    float4 x[kAhead][4];
-#pragma unroll
-    for (int k = 0; k < kAhead; ++k)
-      if (k < nf) issue(k, x[k]);
-    for (int k0 = 0; k0 < nf; k0 += kAhead) {
-#pragma unroll
-      for (int kk = 0; kk < kAhead; ++kk) {
-        const int k = k0 + kk;
-        if (k < nf) {
-          const int64_t u = u0 + static_cast<int64_t>(fc + k) * p.H;
-          float dS[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          add8(dS, x[kk][0], x[kk][1]);
-          add8(dS, x[kk][2], x[kk][3]);
-          if (p.tpu > 0) {
-            const int2 cr = slot_tab[k];
-            for (int cc = cr.x + 2; cc <= cr.y; ++cc) {
-              const float4* sx = reinterpret_cast<const float4*>(col + (u + cc) * PF);
-              add8(dS, __ldg(sx), __ldg(sx + 1));
+  } else {
+    // --------------------------------------------------------------- consumers
+    const float* gcol = p.partial + static_cast<int64_t>(j) * D + c * 8;
+    constexpr int CPA = G::kAtomElems / 8;
+    const int64_t img_off = (c / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
+                            G::swz(j, c % CPA) * 16;
+    for (int f = 0; f < p.F; ++f) {
+      const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+      float dS[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (stream_partials) {
+        const int s = f % S;
+        if (!warp_wait(full(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
+        if (active) {
+          const int2 cr = *reinterpret_cast<const int2*>(stage(s) + 2 * C::kSlotBytes);
+          const float4* x = reinterpret_cast<const float4*>(stage(s) + r * D * 4 + c * 32);
+          add8(dS, x[0], x[1]);
+          if (cr.y > cr.x) {
+            const float4* y = reinterpret_cast<const float4*>(stage(s) + C::kSlotBytes +
+                                                              r * D * 4 + c * 32);
+            add8(dS, y[0], y[1]);
+            for (int cc = cr.x + 2; cc <= cr.y; ++cc) {  // rare: unit split over > 2 CTAs
+              const float4* z = reinterpret_cast<const float4*>(gcol + (u + cc) * PF);
+              add8(dS, __ldg(z), __ldg(z + 1));
             }
           }
-          if (k + kAhead < nf) issue(k + kAhead, x[kk]);
-          const float g = __ldg(p.gate + u);
-          const float a = 1.0f / (1.0f + expf(-g));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(s));
+      }
+      if (active) {
+        const float g = __ldg(p.gate + u);
+        const float a = 1.0f / (1.0f + expf(-g));
 #pragma unroll
-          for (int e = 0; e < 8; ++e) S[e] = fmaf(a, S[e], dS[e]);
-          if (p.image != nullptr) {
-            uint4 w;
-            w.x = pack_bf16x2(S[0], S[1]);
-            w.y = pack_bf16x2(S[2], S[3]);
-            w.z = pack_bf16x2(S[4], S[5]);
-            w.w = pack_bf16x2(S[6], S[7]);
-            *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) = w;
-          }
+        for (int e = 0; e < 8; ++e) S8[e] = fmaf(a, S8[e], dS[e]);
+        if (p.image != nullptr) {
+          uint4 w;
+          w.x = pack_bf16x2(S8[0], S8[1]);
+          w.y = pack_bf16x2(S8[2], S8[3]);
+          w.z = pack_bf16x2(S8[4], S8[5]);
+          w.w = pack_bf16x2(S8[6], S8[7]);
+          *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) = w;
         }
       }
     }
   }
-  if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");
 
+  __syncwarp();
+  __syncthreads();  // every role is done with the stages and the tile
   if (p.state_out != nullptr) {
-    __syncthreads();  // every read of the tile (state_in) is done
     if (active) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) st[r][c * 8 + e] = S[e];
+      for (int e = 0; e < 8; ++e) st[r][c * 8 + e] = S8[e];
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kBlock) {
+    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kThreads) {
       const int jj = idx % C::kRows, i = idx / C::kRows;
       if (jj < nrows) p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jj] = st[jj][i];
     }
