@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     gla_forward_noalloc,
     gla_forward_timed,
     gla_noalloc_scratch_bytes,
+    gla_trim_workspace,
     gla_version,
     load_library,
 )

@@ -26,7 +26,7 @@ GLA_ERR_DEVICE = 7
 GLA_ERR_SCRATCH = 8
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
-            "gla_error_string", "gla_device_fault", "gla_version")
+            "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
 
 
 class GLAError(RuntimeError):
@@ -59,6 +59,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward_noalloc.restype = i32
     lib.gla_noalloc_scratch_bytes.argtypes = []
     lib.gla_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.gla_trim_workspace.argtypes = []
+    lib.gla_trim_workspace.restype = i32
     lib.gla_error_string.argtypes = [i32]
     lib.gla_error_string.restype = ctypes.c_char_p
     lib.gla_device_fault.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -153,6 +155,14 @@ def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, fr
 
 def gla_noalloc_scratch_bytes() -> int:
     return int(load_library().gla_noalloc_scratch_bytes())
+
+
+def gla_trim_workspace() -> None:
+    """Release the current device's unused workspace memory held by the
+    library's pool."""
+    st = load_library().gla_trim_workspace()
+    if st != GLA_OK:
+        raise GLAError(st, "gla_trim_workspace")
 
 
 def gla_error_string(status: int) -> str:

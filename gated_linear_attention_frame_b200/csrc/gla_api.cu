@@ -48,6 +48,33 @@ struct FixedScratch {
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
+// Per-device stream-ordered pool for gla_forward's workspace.  Its release
+// threshold is unbounded, so memory freed at the end of a call stays mapped
+// for the next call instead of going back to the driver at the caller's next
+// synchronisation (re-mapping hundreds of MB costs tens of milliseconds).
+// gla_trim_workspace() returns it.
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+cudaMemPool_t workspace_pool() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_pool[dev] == nullptr) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    uint64_t keep = ~uint64_t(0);
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = pool;
+  }
+  return g_pool[dev];
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 template <int D>
@@ -60,8 +87,11 @@ cudaError_t set_smem_attrs() {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::OutCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(gla::gla_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gla::ScanCfg<D>::kSmemBytes);
+  e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::ScanCfg<D, 1>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gla::ScanCfg<D, 3>::kSmemBytes);
 }
 
 // Per-device one-time set-up: SM count, architecture check, kernel attributes,
@@ -204,8 +234,10 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
     if (static_cast<size_t>(ws_bytes) > fixed->bytes) return GLA_ERR_SCRATCH;
     ws = ws_bytes > 0 ? fixed->ptr : nullptr;
   } else if (ws_bytes > 0) {
-    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), a.stream) !=
-        cudaSuccess) {
+    cudaMemPool_t pool = workspace_pool();
+    if (pool == nullptr ||
+        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
+                                a.stream) != cudaSuccess) {
       cudaGetLastError();
       return GLA_ERR_ALLOC;
     }
@@ -232,10 +264,14 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   record(1);
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
     gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, wp, a.H, a.F, tpu};
-    using SC = gla::ScanCfg<D>;
-    const unsigned grid = static_cast<unsigned>(SC::kGroups) * static_cast<unsigned>(a.B * a.H);
-    const cudaError_t e = launch_dependent(gla::gla_scan_kernel<D>, grid, SC::kThreads,
-                                           SC::kSmemBytes, a.stream, sp);
+    using SC1 = gla::ScanCfg<D, 1>;
+    using SC3 = gla::ScanCfg<D, 3>;
+    const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
+    const cudaError_t e =
+        a.F <= 1 ? launch_dependent(gla::gla_scan_kernel<D, 1>, grid, SC1::kThreads,
+                                    SC1::kSmemBytes, a.stream, sp)
+                 : launch_dependent(gla::gla_scan_kernel<D, 3>, grid, SC3::kThreads,
+                                    SC3::kSmemBytes, a.stream, sp);
     if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
   }
@@ -334,6 +370,18 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v, const float
 }
 
 size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int gla_trim_workspace(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GLA_ERR_DEVICE;
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    pool = g_pool[dev];
+  }
+  if (pool == nullptr) return GLA_OK;
+  return cudaMemPoolTrimTo(pool, 0) == cudaSuccess ? GLA_OK : GLA_ERR_LAUNCH;
+}
 
 const char* gla_error_string(int status) {
   switch (status) {

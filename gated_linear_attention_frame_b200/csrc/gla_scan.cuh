@@ -38,14 +38,14 @@ struct ScanParams {
   int H, F, tpu;
 };
 
-template <int D>
+template <int D, int kStagesT = 3>
 struct ScanCfg {
   static constexpr int kOcts = D / 8;                          // 8-float chunks per state row
   static constexpr int kConsumers = 256;                        // 8 consumer warps
   static constexpr int kThreads = kConsumers + 32;              // + 1 producer warp
   static constexpr int kRows = kConsumers / kOcts;              // state rows per block
   static constexpr int kGroups = (D + 1 + kRows - 1) / kRows;   // blocks per (b, h)
-  static constexpr int kStages = 3;
+  static constexpr int kStages = kStagesT;
   static constexpr int kSlotBytes = kRows * D * 4;              // one partial's rows: 8 KB
   static constexpr int kStageBytes = 2 * kSlotBytes + 16;       // two partials + header
   static constexpr int kTileBytes = kRows * (D + 1) * 4;        // state_in / state_out tile
@@ -60,11 +60,14 @@ __device__ __forceinline__ void add8(float (&acc)[8], const float4& a, const flo
 // Grid: kGroups blocks of 288 threads per (b, h), flattened; block g owns
 // state rows j in [g*kRows, (g+1)*kRows) (row d = normaliser).  Launched as a
 // programmatic dependent of the increment kernel: only caller inputs
-// (state_in) are read before griddepcontrol.wait.
-template <int D>
-__global__ void __launch_bounds__(288) gla_scan_kernel(const ScanParams p) {
+// (state_in) are read before griddepcontrol.wait.  kStagesT = 1 serves
+// single-frame calls (fewer registers and less shared memory: more blocks
+// per SM), 3 serves sequences of frames.
+template <int D, int kStagesT>
+__global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
+    gla_scan_kernel(const ScanParams p) {
   using G = Geo<D>;
-  using C = ScanCfg<D>;
+  using C = ScanCfg<D, kStagesT>;
   constexpr int PF = IncCfg<D>::kPartialFloats;
   constexpr int S = C::kStages;
   constexpr unsigned kCode = 4u;
@@ -103,21 +106,14 @@ __global__ void __launch_bounds__(288) gla_scan_kernel(const ScanParams p) {
     *abort = 0;
     fence_mbar_init();
   }
-  if (p.state_in != nullptr) {
-    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kThreads) {
-      const int jj = idx % C::kRows, i = idx / C::kRows;
-      if (jj < nrows) st[jj][i] = p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jj];
-    }
-  }
-  __syncthreads();
-  float S8[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) S8[e] = (active && p.state_in != nullptr) ? st[r][c * 8 + e] : 0.f;
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
+  __syncthreads();  // barriers initialised
 
   const bool stream_partials = p.tpu > 0 && p.F > 0;
+  float S8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
+    // Starts streaming partials while the consumers load state_in.
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
     if (lane == 0 && stream_partials) {
       const uint32_t bytes = static_cast<uint32_t>(nrows) * D * 4;
       int f = 0;
@@ -139,6 +135,18 @@ __global__ void __launch_bounds__(288) gla_scan_kernel(const ScanParams p) {
     }
   } else {
     // --------------------------------------------------------------- consumers
+    if (p.state_in != nullptr) {
+      for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kConsumers) {
+        const int jj = idx % C::kRows, i = idx / C::kRows;
+        if (jj < nrows) st[jj][i] = p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jj];
+      }
+      named_bar_sync(1, C::kConsumers);
+      if (active) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) S8[e] = st[r][c * 8 + e];
+      }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // partials read directly (rare)
     const float* gcol = p.partial + static_cast<int64_t>(j) * D + c * 8;
     constexpr int CPA = G::kAtomElems / 8;
     const int64_t img_off = (c / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
@@ -183,19 +191,20 @@ __global__ void __launch_bounds__(288) gla_scan_kernel(const ScanParams p) {
     }
   }
 
-  __syncwarp();
-  __syncthreads();  // every role is done with the stages and the tile
-  if (p.state_out != nullptr) {
+  if (consumer && p.state_out != nullptr) {
+    named_bar_sync(1, C::kConsumers);  // every consumer is done reading the tile
     if (active) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) st[r][c * 8 + e] = S8[e];
     }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kThreads) {
+    named_bar_sync(1, C::kConsumers);
+    for (int idx = threadIdx.x; idx < D * C::kRows; idx += C::kConsumers) {
       const int jj = idx % C::kRows, i = idx / C::kRows;
       if (jj < nrows) p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jj] = st[jj][i];
     }
   }
+  __syncwarp();
+  __syncthreads();  // the producer's copies have landed before the block exits
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 

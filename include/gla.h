@@ -79,9 +79,10 @@ typedef enum {
  *   stream       CUDA stream for all work (0 = legacy default stream).
  *
  * Memory: takes a workspace of about (B*H*frames*6 + #SMs*4) * (d+1)*d bytes
- * (per-frame fp32 state increments and bf16 prefix states) with
- * cudaMallocAsync on `stream` and frees it with cudaFreeAsync on the same
- * stream.
+ * (per-frame fp32 state increments and bf16 prefix states) from the
+ * library's stream-ordered memory pool on `stream` and frees it on the same
+ * stream.  The pool (one per device, created at the first call) keeps freed
+ * memory mapped for later calls; gla_trim_workspace() returns it.
  * Returns GLA_OK or a gla_status code; on error nothing was enqueued, except
  * GLA_ERR_LAUNCH, after which part of the work may have been enqueued.
  */
@@ -144,6 +145,13 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v,
 
 /* Size in bytes of gla_forward_noalloc's fixed scratch array.  Host only. */
 size_t gla_noalloc_scratch_bytes(void);
+
+/*
+ * gla_trim_workspace -- release the current device's unused workspace memory
+ * held by the library's pool (memory of calls still in flight is kept).
+ * Returns GLA_OK, GLA_ERR_DEVICE or GLA_ERR_LAUNCH.
+ */
+int gla_trim_workspace(void);
 
 /* Static string for a gla_status code (never NULL). Host only, no CUDA call. */
 const char* gla_error_string(int status);

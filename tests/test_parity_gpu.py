@@ -201,6 +201,15 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
 
 
+def test_trim_workspace_between_calls():
+    F, T, d = 4, 500, 128
+    w, q, k, v, g, s = small_case(2, 4, F, T, d, True, seed=31)
+    o1, s1 = run_gpu(q, k, v, g, s, F)
+    gla().gla_trim_workspace()
+    o2, s2 = run_gpu(q, k, v, g, s, F)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
 def test_guard_bands_untouched():
     """Writes stay inside out and state_out (TMA store clipping at ragged
     frame ends, scan bounds)."""
