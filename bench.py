@@ -41,22 +41,41 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "720p-5s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
-# DRAM traffic per launch of the dominant kernel from an ncu capture, valid
-# only while the kernel source is unchanged (hash of the .cuh files below).
-NCU_TRAFFIC = {}
-KERNEL_SOURCES = ["gla_increment.cuh", "gla_output.cuh", "gla_scan.cuh", "gla_common.cuh",
-                  "sm100_ptx.cuh", "gla_api.cu"]
+# DRAM bytes (read + write) per launch from one ncu capture of the full
+# workload (profiles/dram_traffic_720p5s.md), valid only while the kernel's
+# sources are unchanged: the hash of its files must match.
+KERNEL_DEPS = {
+    "output": ["gla_output.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "increment": ["gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "scan": ["gla_scan.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+}
+NCU_TRAFFIC = {
+    "720p-5s": {
+        "increment": (1899738368 + 65973760, "adfba699d59f78a6"),
+        "scan": (75846144 + 5643008, "4d675cb7e40bc9d1"),
+        "output": (985641728 + 897636864, "60851f75ff180302"),
+    },
+}
 
 
 # ----------------------------------------------------------------- helpers
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for n in KERNEL_SOURCES:
+    for n in KERNEL_DEPS[kernel]:
         with open(os.path.join(ROOT, "gated_linear_attention_frame_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch measured by ncu for this workload and kernel, or
+    None when there is no capture or the kernel changed since."""
+    entry = NCU_TRAFFIC.get(workload, {}).get(kernel)
+    if entry is None or entry[1] != kernel_source_hash(kernel):
+        return None
+    return entry[0]
 
 
 def load_peaks() -> dict:
@@ -322,12 +341,12 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     avg = per.mean(axis=0)
     dom = int(np.argmax(avg))
     achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
-    traffic = None
-    if NCU_TRAFFIC.get("kernel") == names[dom] and NCU_TRAFFIC.get("src") == kernel_source_hash():
-        traffic = NCU_TRAFFIC.get("bytes_per_launch")
+    traffic = ncu_traffic(w.name, names[dom])
     roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic, "peak_source": peaks["source"] + " (hbm_gbs)"}
+            "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read + write)",
+            "algorithmic_bytes_per_launch": work[names[dom]],
+            "peak_source": peaks["source"] + " (hbm_gbs)"}
     t_roof = max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
                  work["flops"] / (peaks["bf16_tflops"] * 1e12))
     layer = {"algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
