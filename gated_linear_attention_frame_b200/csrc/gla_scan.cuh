@@ -17,7 +17,8 @@
 // shared-memory stages with plain bulk copies (one copy per partial: the
 // block's rows of it are contiguous), so several frames are in flight without
 // holding them in registers; eight consumer warps take one stage per frame.
-// Which increment CTAs hold a unit's partials travels with the stage.
+// Which increment CTAs hold a unit's partials, and the frame's decay, travel
+// with the stage.
 // state_in and state_out, stored [d][d+1] by the caller, are moved through a
 // shared-memory tile so that global accesses run along rows.
 #pragma once
@@ -41,15 +42,23 @@ struct ScanParams {
 template <int D, int kStagesT = 3>
 struct ScanCfg {
   static constexpr int kOcts = D / 8;                          // 8-float chunks per state row
-  static constexpr int kConsumers = 256;                        // 8 consumer warps
+  static constexpr int kConsumerWarps = 8;
+  static constexpr int kConsumers = 32 * kConsumerWarps;
   static constexpr int kThreads = kConsumers + 32;              // + 1 producer warp
   static constexpr int kRows = kConsumers / kOcts;              // state rows per block
   static constexpr int kGroups = (D + 1 + kRows - 1) / kRows;   // blocks per (b, h)
   static constexpr int kStages = kStagesT;
   static constexpr int kSlotBytes = kRows * D * 4;              // one partial's rows: 8 KB
-  static constexpr int kStageBytes = 2 * kSlotBytes + 16;       // two partials + header
+  static constexpr int kStageBytes = 2 * kSlotBytes + 16;       // two partials + StageHeader
   static constexpr int kTileBytes = kRows * (D + 1) * 4;        // state_in / state_out tile
   static constexpr int kSmemBytes = 128 + kStages * kStageBytes + kTileBytes + 2 * kStages * 8 + 16;
+};
+
+// Header at the end of each stage, written by the producer with the copies.
+struct StageHeader {
+  int32_t c0, c1;  // the unit's partials are at slots u + c0 .. u + c1
+  float a;         // the frame's decay sigmoid(g)
+  int32_t pad;
 };
 
 __device__ __forceinline__ void add8(float (&acc)[8], const float4& a, const float4& b) {
@@ -91,7 +100,8 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
   const int r = threadIdx.x / C::kOcts;  // consumer: row within the block
   const int c = threadIdx.x % C::kOcts;  // consumer: key features 8c .. 8c+7
   const int j = j0 + r;                  // value column (j == D: normaliser)
-  const bool consumer = warp < 8;
+  constexpr int kCW = C::kConsumerWarps;
+  const bool consumer = warp < kCW;
   const bool active = consumer && r < nrows;
   const int b = bh / p.H;
   const int h = bh - b * p.H;
@@ -101,7 +111,7 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 8);
+      mbar_init(empty(s), kCW);
     }
     *abort = 0;
     fence_mbar_init();
@@ -110,28 +120,46 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
 
   const bool stream_partials = p.tpu > 0 && p.F > 0;
   float S8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (warp == 8) {
+  if (warp == kCW) {
     // ---------------------------------------------------------------- producer
     // Starts streaming partials while the consumers load state_in.
     asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
-    if (lane == 0 && stream_partials) {
+    if (stream_partials) {
+      // The whole warp loads the gate logits of 32 frames at a time (one lane
+      // per frame); lane 0 turns each into a = sigmoid(g) and hands it to the
+      // consumers in the stage header, so no consumer waits on a gate load.
       const uint32_t bytes = static_cast<uint32_t>(nrows) * D * 4;
+      float gl = 0.f;
       int f = 0;
       for (; f < p.F; ++f) {
-        const int s = f % S;
-        if (!mbar_wait(empty(s), static_cast<uint32_t>(((f / S) & 1) ^ 1), abort, kCode)) break;
-        const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
-        int32_t c0, c1;
-        p.wp.slot_range(u, c0, c1);
-        int2* hdr = reinterpret_cast<int2*>(stage(s) + 2 * C::kSlotBytes);
-        *hdr = make_int2(c0, c1);
-        const float* src = p.partial + (u + c0) * PF + static_cast<int64_t>(j0) * D;
-        mbar_arrive_expect_tx(full(s), (c1 > c0 ? 2u : 1u) * bytes);
-        bulk_load(smem_u32(stage(s)), src, bytes, full(s));
-        if (c1 > c0) bulk_load(smem_u32(stage(s)) + C::kSlotBytes, src + PF, bytes, full(s));
+        if ((f & 31) == 0) {
+          const int ff = f + lane;
+          gl = ff < p.F ? __ldg(p.gate + u0 + static_cast<int64_t>(ff) * p.H) : 0.f;
+        }
+        const float g = __shfl_sync(0xffffffffu, gl, f & 31);
+        int ok = 1;
+        if (lane == 0) {
+          const int s = f % S;
+          ok = mbar_wait(empty(s), static_cast<uint32_t>(((f / S) & 1) ^ 1), abort, kCode) ? 1 : 0;
+          if (ok) {
+            const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+            int32_t c0, c1;
+            p.wp.slot_range(u, c0, c1);
+            StageHeader* hdr = reinterpret_cast<StageHeader*>(stage(s) + 2 * C::kSlotBytes);
+            hdr->c0 = c0;
+            hdr->c1 = c1;
+            hdr->a = 1.0f / (1.0f + expf(-g));
+            const float* src = p.partial + (u + c0) * PF + static_cast<int64_t>(j0) * D;
+            mbar_arrive_expect_tx(full(s), (c1 > c0 ? 2u : 1u) * bytes);
+            bulk_load(smem_u32(stage(s)), src, bytes, full(s));
+            if (c1 > c0) bulk_load(smem_u32(stage(s)) + C::kSlotBytes, src + PF, bytes, full(s));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
-      for (int k = (f > S ? f - S : 0); k < f; ++k)
-        mbar_wait_drain(full(k % S), static_cast<uint32_t>((k / S) & 1));
+      if (lane == 0)
+        for (int k = (f > S ? f - S : 0); k < f; ++k)
+          mbar_wait_drain(full(k % S), static_cast<uint32_t>((k / S) & 1));
     }
   } else {
     // --------------------------------------------------------------- consumers
@@ -154,11 +182,14 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
     for (int f = 0; f < p.F; ++f) {
       const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
       float dS[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float a;
       if (stream_partials) {
         const int s = f % S;
         if (!warp_wait(full(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
+        const StageHeader hd = *reinterpret_cast<const StageHeader*>(stage(s) + 2 * C::kSlotBytes);
+        a = hd.a;
         if (active) {
-          const int2 cr = *reinterpret_cast<const int2*>(stage(s) + 2 * C::kSlotBytes);
+          const int2 cr = make_int2(hd.c0, hd.c1);
           const float4* x = reinterpret_cast<const float4*>(stage(s) + r * D * 4 + c * 32);
           add8(dS, x[0], x[1]);
           if (cr.y > cr.x) {
@@ -173,10 +204,10 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty(s));
+      } else {
+        a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));  // frames without tokens
       }
       if (active) {
-        const float g = __ldg(p.gate + u);
-        const float a = 1.0f / (1.0f + expf(-g));
 #pragma unroll
         for (int e = 0; e < 8; ++e) S8[e] = fmaf(a, S8[e], dS[e]);
         if (p.image != nullptr) {
