@@ -1,5 +1,8 @@
 """fp64 CPU oracle (test infrastructure only; see gla_oracle.py)."""
 
+from .gla_backward_oracle import (gla_backward, gla_backward_head, gla_backward_head_manual,
+                                  gla_forward_torch_head)
 from .gla_oracle import gla_bruteforce_head, gla_forward, gla_head, relu, sigmoid
 
-__all__ = ["gla_bruteforce_head", "gla_forward", "gla_head", "relu", "sigmoid"]
+__all__ = ["gla_bruteforce_head", "gla_forward", "gla_head", "relu", "sigmoid", "gla_backward",
+           "gla_backward_head", "gla_backward_head_manual", "gla_forward_torch_head"]
