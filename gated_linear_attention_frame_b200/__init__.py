@@ -13,7 +13,10 @@ from ._binding import (  # noqa: F401
     GLA_ERR_UNSUPPORTED_D,
     GLA_OK,
     GLAError,
+    backward,
     forward,
+    gla_backward,
+    gla_backward_timed,
     gla_device_fault,
     gla_error_string,
     gla_forward,

@@ -26,7 +26,8 @@ GLA_ERR_DEVICE = 7
 GLA_ERR_SCRATCH = 8
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
-            "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
+            "gla_backward", "gla_backward_timed", "gla_trim_workspace", "gla_error_string",
+            "gla_device_fault", "gla_version")
 
 
 class GLAError(RuntimeError):
@@ -57,6 +58,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward_timed.restype = i32
     lib.gla_forward_noalloc.argtypes = fwd
     lib.gla_forward_noalloc.restype = i32
+    bwd = [vp] * 12 + [i32, i32, i32, i32, i32, f32, vp]
+    lib.gla_backward.argtypes = bwd
+    lib.gla_backward.restype = i32
+    lib.gla_backward_timed.argtypes = bwd + [ctypes.POINTER(vp)]
+    lib.gla_backward_timed.restype = i32
     lib.gla_noalloc_scratch_bytes.argtypes = []
     lib.gla_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.gla_trim_workspace.argtypes = []
@@ -153,6 +159,54 @@ def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, fr
         raise GLAError(st, "gla_forward_noalloc")
 
 
+def _check_bwd_dtypes(dout, dstate_out, dq, dk, dv, dgate_logits, dstate_in):
+    for name, t, dt in (("dout", dout, torch.bfloat16), ("dq", dq, torch.bfloat16),
+                        ("dk", dk, torch.bfloat16), ("dv", dv, torch.bfloat16),
+                        ("dstate_out", dstate_out, torch.float32),
+                        ("dgate_logits", dgate_logits, torch.float32),
+                        ("dstate_in", dstate_in, torch.float32)):
+        if isinstance(t, torch.Tensor) and t.dtype != dt:
+            raise TypeError("gla: %s must be %s, got %s" % (name, dt, t.dtype))
+
+
+def _bwd_args(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+              dstate_in, B, H, frames, tokens_per_frame, d, eps, stream):
+    _check_dtypes(q, k, v, gate_logits, state_in, None, dq)
+    _check_bwd_dtypes(dout, dstate_out, dq, dk, dv, dgate_logits, dstate_in)
+    return (_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in), _ptr(dout),
+            _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate_logits), _ptr(dstate_in),
+            int(B), int(H), int(frames), int(tokens_per_frame), int(d), float(eps),
+            _stream(stream))
+
+
+def gla_backward(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+                 dstate_in, B, H, frames, tokens_per_frame, d, eps, stream=None) -> None:
+    """Enqueue the gradients of one layer call (see include/gla.h; d = 128).
+    Tensors or raw device addresses; raises GLAError on a nonzero status."""
+    args = _bwd_args(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+                     dstate_in, B, H, frames, tokens_per_frame, d, eps, stream)
+    st = load_library().gla_backward(*args)
+    if st != GLA_OK:
+        raise GLAError(st, "gla_backward")
+
+
+def gla_backward_timed(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv,
+                       dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream,
+                       events) -> None:
+    """gla_backward that records 7 CUDA events around its six kernels
+    (`events`: 7 torch.cuda.Event(enable_timing=True))."""
+    args = _bwd_args(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+                     dstate_in, B, H, frames, tokens_per_frame, d, eps, stream)
+    lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 7)(*[e.cuda_event for e in events])
+    st = lib.gla_backward_timed(*args, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_backward_timed")
+
+
 def gla_noalloc_scratch_bytes() -> int:
     return int(load_library().gla_noalloc_scratch_bytes())
 
@@ -201,3 +255,24 @@ def forward(q, k, v, gate_logits, state_in=None, eps: float = 1e-6, out=None, st
         state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
     gla_forward(q, k, v, gate_logits, state_in, state_out, out, B, H, frames, T, d, eps, stream)
     return out, state_out
+
+
+def backward(q, k, v, gate_logits, dout, state_in=None, dstate_out=None, eps: float = 1e-6,
+             stream=None, want_dstate_in: bool = True):
+    """Convenience wrapper of gla_backward: allocates the gradients and
+    returns (dq, dk, dv, dgate_logits, dstate_in or None)."""
+    B, N, H, d = q.shape
+    frames = gate_logits.shape[1]
+    if frames == 0:
+        T = 0
+    else:
+        if N % frames:
+            raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+        T = N // frames
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty_like(gate_logits)
+    ds_in = (torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
+             if want_dstate_in else None)
+    gla_backward(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dg, ds_in, B, H,
+                 frames, T, d, eps, stream)
+    return dq, dk, dv, dg, ds_in

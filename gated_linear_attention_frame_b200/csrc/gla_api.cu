@@ -6,6 +6,14 @@
 //   1. gla_increment_kernel  dS_f partials  (tcgen05, TMA, ReLU fused)
 //   2. gla_scan_kernel       S_f = a_f S_{f-1} + dS_f, state_out, bf16 S_f^T images
 //   3. gla_output_kernel     out = phi(q) S_f / (phi(q) S_f[:, d] + eps)   (tcgen05)
+// gla_backward (d = 128) recomputes the forward states and enqueues
+//   1. gla_increment_kernel  dS_f partials
+//   2. gla_scan_kernel       S_f (fp32, kept) and bf16 S_f^T images
+//   3. gla_bwd_q_kernel      dq and the local state gradients L_f   (tcgen05)
+//   4. gla_scan_bwd_kernel   G_f = L_f + a_{f+1} G_{f+1}, dstate_in, da_f partial sums,
+//                            bf16 G_f^T images
+//   5. gla_dgate_kernel      dg = a (1 - a) da
+//   6. gla_bwd_kv_kernel     dk, dv                                   (tcgen05)
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -15,10 +23,13 @@
 #include <mutex>
 
 #include "gla.h"
+#include "gla_bwd_kv.cuh"
+#include "gla_bwd_q.cuh"
 #include "gla_common.cuh"
 #include "gla_increment.cuh"
 #include "gla_output.cuh"
 #include "gla_scan.cuh"
+#include "gla_scan_bwd.cuh"
 #include "sm100_ptx.cuh"
 
 namespace {
@@ -90,8 +101,18 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::ScanCfg<D, 1>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gla::ScanCfg<D, 3>::kSmemBytes);
+  e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::ScanCfg<D, 3>::kSmemBytes);
+  if (e != cudaSuccess || D != 128) return e;
+  e = cudaFuncSetAttribute(gla::gla_bwd_q_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::BwdQCfg<128>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla::gla_bwd_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::BwdKVCfg<128>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gla::gla_scan_bwd_kernel<128>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gla::ScanBwdCfg<128>::kSmemBytes);
 }
 
 // Per-device one-time set-up: SM count, architecture check, kernel attributes,
@@ -263,7 +284,7 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   }
   record(1);
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
-    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, wp, a.H, a.F, tpu};
+    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu};
     using SC1 = gla::ScanCfg<D, 1>;
     using SC3 = gla::ScanCfg<D, 3>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
@@ -339,6 +360,170 @@ int forward_noalloc_impl(const Args& a) {
   }
 }
 
+struct BwdArgs {
+  const void *q, *k, *v;
+  const float* g;
+  const float* s_in;
+  const void* dout;
+  const float* ds_out;
+  void *dq, *dk, *dv;
+  float* dg;
+  float* ds_in;
+  int B, H, F, T, d;
+  float eps;
+  cudaStream_t stream;
+};
+
+// Host-only checks of gla_backward's arguments; no CUDA call.
+int validate_bwd(const BwdArgs& a) {
+  if (a.d != 128) return GLA_ERR_UNSUPPORTED_D;
+  Args f{a.q, a.k, a.v, a.g, a.s_in, nullptr, a.dq, a.B, a.H, a.F, a.T, a.d, a.eps, a.stream};
+  int st = validate(f);
+  if (st != GLA_OK) return st;
+  const int64_t elems = static_cast<int64_t>(a.B) * a.F * a.T * a.H * a.d;
+  const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
+  if (elems > 0 && (a.dout == nullptr || a.dk == nullptr || a.dv == nullptr)) return GLA_ERR_NULL;
+  if (units > 0 && a.dg == nullptr) return GLA_ERR_NULL;
+  if (elems > 0 && (!aligned(a.dout, 16) || !aligned(a.dk, 16) || !aligned(a.dv, 16)))
+    return GLA_ERR_ALIGN;
+  if ((a.dg && !aligned(a.dg, 4)) || (a.ds_out && !aligned(a.ds_out, 4)) ||
+      (a.ds_in && !aligned(a.ds_in, 4)))
+    return GLA_ERR_ALIGN;
+  return GLA_OK;
+}
+
+// The six kernels of the backward pass (d = 128).  The workspace holds the
+// partials (the recompute's increments, then the local state gradients L_f:
+// the forward scan has finished reading the first before the query kernel
+// writes the second), the bf16 images (S_f^T, then G_f^T, likewise), the fp32
+// forward states S_f and the per-warp partial sums of da_f.
+int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
+  constexpr int D = 128;
+  using G = Geo<D>;
+  constexpr int PF = gla::IncCfg<D>::kPartialFloats;
+  using RS = gla::ScanBwdCfg<D>;
+  const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
+  const int tpu = (a.T + gla::kTileTokens - 1) / gla::kTileTokens;
+  const int64_t W = units * tpu;
+  const int32_t G1 = static_cast<int32_t>(W < di.sms ? W : di.sms);
+  const gla::WorkPlan wp = W > 0 ? gla::WorkPlan::make(units, tpu, G1) : gla::WorkPlan{};
+
+  const int64_t partial_bytes = W > 0 ? align256((units + G1) * static_cast<int64_t>(PF) * 4) : 0;
+  const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
+  const int64_t states_bytes = align256(units * static_cast<int64_t>(PF) * 4);
+  const int64_t da_bytes = align256(units * static_cast<int64_t>(RS::kGroups) * 8 * 4);
+  const int64_t ws_bytes = partial_bytes + image_bytes + states_bytes + da_bytes;
+
+  CUtensorMap tm_q, tm_k, tm_v, tm_dq, tm_dk, tm_dv;
+  if (W > 0) {
+    int st;
+    if ((st = encode_map(&tm_q, a.q, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_k, a.k, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_v, a.v, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_dq, a.dq, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_dk, a.dk, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_dv, a.dv, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+  }
+
+  uint8_t* ws = nullptr;
+  if (ws_bytes > 0) {
+    cudaMemPool_t pool = workspace_pool();
+    if (pool == nullptr ||
+        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
+                                a.stream) != cudaSuccess) {
+      cudaGetLastError();
+      return GLA_ERR_ALLOC;
+    }
+  }
+  float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
+  uint8_t* image = W > 0 ? ws + partial_bytes : nullptr;
+  float* states = ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes) : nullptr;
+  float* da_part =
+      ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + states_bytes) : nullptr;
+
+  int status = GLA_OK;
+  auto check = [&]() {
+    if (cudaGetLastError() != cudaSuccess) status = GLA_ERR_LAUNCH;
+  };
+  auto record = [&](int i) {
+    if (ev != nullptr && status == GLA_OK && cudaEventRecord(ev[i], a.stream) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+  };
+
+  record(0);
+  if (W > 0 && status == GLA_OK) {
+    gla::IncParams ip{partial, wp, a.H, a.F};
+    gla::gla_increment_kernel<D>
+        <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    check();
+  }
+  record(1);
+  if (status == GLA_OK && a.F > 0) {
+    gla::ScanParams sp{partial, a.g, a.s_in, nullptr, image, states, wp, a.H, a.F, tpu};
+    using SC1 = gla::ScanCfg<D, 1>;
+    using SC3 = gla::ScanCfg<D, 3>;
+    const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
+    const cudaError_t e =
+        a.F <= 1 ? launch_dependent(gla::gla_scan_kernel<D, 1>, grid, SC1::kThreads,
+                                    SC1::kSmemBytes, a.stream, sp)
+                 : launch_dependent(gla::gla_scan_kernel<D, 3>, grid, SC3::kThreads,
+                                    SC3::kSmemBytes, a.stream, sp);
+    if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(2);
+  if (W > 0 && status == GLA_OK) {
+    gla::BwdQParams qp{image, static_cast<const uint16_t*>(a.dout), partial, a.eps, wp,
+                       a.H, a.F, a.T};
+    if (launch_dependent(gla::gla_bwd_q_kernel<D>, G1, gla::BwdQCfg<D>::kThreads,
+                         gla::BwdQCfg<D>::kSmemBytes, a.stream, tm_q, tm_dq, qp) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(3);
+  if (status == GLA_OK && (a.F > 0 || a.ds_in != nullptr)) {
+    gla::ScanBwdParams rp{partial, a.g, states, a.s_in, a.ds_out, a.ds_in, image, da_part, wp,
+                          a.H, a.F, tpu};
+    const unsigned grid = static_cast<unsigned>(RS::kGroups) * static_cast<unsigned>(a.B * a.H);
+    if (launch_dependent(gla::gla_scan_bwd_kernel<D>, grid, RS::kThreads, RS::kSmemBytes,
+                         a.stream, rp) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(4);
+  if (status == GLA_OK && units > 0) {
+    const unsigned grid = static_cast<unsigned>((units + 255) / 256);
+    if (launch_dependent(gla::gla_dgate_kernel<D>, grid, 256, 0, a.stream,
+                         static_cast<const float*>(da_part), a.g, a.dg, units) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(5);
+  if (W > 0 && status == GLA_OK) {
+    gla::BwdKVParams kp{image, wp, a.H, a.F, a.T};
+    if (launch_dependent(gla::gla_bwd_kv_kernel<D>, G1, gla::BwdKVCfg<D>::kThreads,
+                         gla::BwdKVCfg<D>::kSmemBytes, a.stream, tm_k, tm_v, tm_dk, tm_dv,
+                         kp) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(6);
+  if (ws != nullptr && cudaFreeAsync(ws, a.stream) != cudaSuccess) {
+    cudaGetLastError();
+    if (status == GLA_OK) status = GLA_ERR_LAUNCH;
+  }
+  return status;
+}
+
+int backward_impl(const BwdArgs& a, cudaEvent_t* ev) {
+  int st = validate_bwd(a);
+  if (st != GLA_OK) return st;
+  if (static_cast<int64_t>(a.B) * a.H == 0) return GLA_OK;
+  DeviceInfo di;
+  if ((st = device_setup(&di)) != GLA_OK) return st;
+  return run_backward(a, di, ev);
+}
+
 }  // namespace
 
 extern "C" {
@@ -371,6 +556,26 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v, const float
 
 size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
+int gla_backward(const void* q, const void* k, const void* v, const float* gate_logits,
+                 const float* state_in, const void* dout, const float* dstate_out, void* dq,
+                 void* dk, void* dv, float* dgate_logits, float* dstate_in, int B, int H,
+                 int frames, int tokens_per_frame, int d, float eps, cudaStream_t stream) {
+  BwdArgs a{q,  k,  v,  gate_logits, state_in, dout, dstate_out, dq, dk,     dv,
+            dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream};
+  return backward_impl(a, nullptr);
+}
+
+int gla_backward_timed(const void* q, const void* k, const void* v, const float* gate_logits,
+                       const float* state_in, const void* dout, const float* dstate_out, void* dq,
+                       void* dk, void* dv, float* dgate_logits, float* dstate_in, int B, int H,
+                       int frames, int tokens_per_frame, int d, float eps, cudaStream_t stream,
+                       cudaEvent_t* events) {
+  if (events == nullptr) return GLA_ERR_NULL;
+  BwdArgs a{q,  k,  v,  gate_logits, state_in, dout, dstate_out, dq, dk,     dv,
+            dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream};
+  return backward_impl(a, events);
+}
+
 int gla_trim_workspace(void) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GLA_ERR_DEVICE;
@@ -389,7 +594,8 @@ const char* gla_error_string(int status) {
     case GLA_ERR_NULL: return "a required pointer is NULL";
     case GLA_ERR_ALIGN: return "a pointer is not aligned (q, k, v, out: 16 bytes; others: 4)";
     case GLA_ERR_SHAPE: return "negative or too large size";
-    case GLA_ERR_UNSUPPORTED_D: return "head dim must be 32, 64 or 128";
+    case GLA_ERR_UNSUPPORTED_D:
+      return "head dim must be 32, 64 or 128 (gla_backward: 128)";
     case GLA_ERR_ALLOC: return "workspace allocation failed";
     case GLA_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
     case GLA_ERR_DEVICE: return "no CUDA device of compute capability 10.x";

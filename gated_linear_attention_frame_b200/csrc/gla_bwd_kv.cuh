@@ -1,0 +1,354 @@
+// gla_bwd_kv.cuh -- key/value side of the backward pass on tcgen05.
+//
+// With G_f the total gradient reaching the state S_f (from the reverse scan)
+// and S_f = a_f S_{f-1} + phi(K_f)^T [V_f | 1], for every token t of frame f:
+//   dk_t = 1[k_t > 0] * ([v_t | 1] G_f^T)      (d outputs)
+//   dv_t = phi(k_t) G_f[:, :d]                 (d outputs)
+// Per 128-token tile, two contractions into TMEM:
+//   dk~ : A = [v | 1]  [M = 128 tokens, K = d + 16]  K-major; the ones column
+//         is a constant 32-byte-swizzled region used by the last K step;
+//         B = G_f^T image read MN-major          [N = d key features]
+//   dv  : A = phi(k)   [M = 128 tokens, K = d]      K-major (ReLU in smem)
+//         B = G_f^T image read K-major           [N = d value columns]
+// One bf16 image of G_f^T (the scan's swizzled K-major layout, d + 1 rows
+// + 15 zero rows in shared memory) serves both.  The ReLU warps also keep a
+// per-row byte mask of phi(k) > 0 in a small ring for the dk epilogue.
+// Warp roles as the forward kernels: 0-3 epilogue, 4-7 ReLU/mask, 8 TMA, 9 MMA.
+#pragma once
+
+#include "gla_common.cuh"
+#include "gla_increment.cuh"  // warp_wait, unit_coords
+#include "sm100_ptx.cuh"
+
+namespace gla {
+
+template <int D>
+struct BwdKVCfg {
+  using G = Geo<D>;
+  static_assert(D == 128, "the backward kernels are built for d = 128");
+  static constexpr int kStages = 2;
+  static constexpr int kStageBytes = 2 * G::kTileBytes;                    // v tile + k tile
+  static constexpr int kGBufBytes = G::kAtoms * G::kNPad * G::kRowBytes;  // G^T image
+  static constexpr int kOnesBytes = kTileTokens * 32;                     // [1 | 0 x 15] rows
+  static constexpr int kMaskRing = 4;
+  static constexpr int kMaskBytes = kTileTokens * (D / 8);                // one byte per 8 features
+  static constexpr int kStageOutBytes = G::kAtomTileBytes;
+  static constexpr int kTmemCols = 512;                                   // 2 x (dk~ | dv)
+  static constexpr int kThreads = 320;
+  static constexpr int kBarCount = 3 * kStages + 2 + 4 + 2 * kMaskRing + 1;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kGBufBytes + kOnesBytes +
+                                    kMaskRing * kMaskBytes + 2 * kStageOutBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+struct BwdKVParams {
+  const uint8_t* gimage;  // [units][kImageBytes] bf16 G_f^T images
+  WorkPlan wp;
+  int H, F, T;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    gla_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_dk,
+                      const __grid_constant__ CUtensorMap tm_dv, const BwdKVParams p) {
+  using G = Geo<D>;
+  using C = BwdKVCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr int R = C::kMaskRing;
+  constexpr unsigned kCode = 16u;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto v_buf = [&](int s) { return sbase + s * C::kStageBytes; };
+  auto k_buf = [&](int s) { return sbase + s * C::kStageBytes + G::kTileBytes; };
+  const uint32_t g_buf = sbase + S * C::kStageBytes;
+  const uint32_t ones_buf = g_buf + C::kGBufBytes;
+  uint8_t* mask_ring = smem + S * C::kStageBytes + C::kGBufBytes + C::kOnesBytes;
+  const uint32_t o_base = ones_buf + C::kOnesBytes + R * C::kMaskBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kGBufBytes +
+                                               C::kOnesBytes + R * C::kMaskBytes +
+                                               2 * C::kStageOutBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  const uint32_t gfull = bar0 + 8u * (3 * S);
+  const uint32_t gempty = bar0 + 8u * (3 * S + 1);
+  auto accf = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };
+  auto acce = [&](int a) { return bar0 + 8u * (3 * S + 4 + a); };
+  auto maskfull = [&](int m) { return bar0 + 8u * (3 * S + 6 + m); };
+  auto maskfree = [&](int m) { return bar0 + 8u * (3 * S + 6 + R + m); };
+  const uint32_t done_bar = bar0 + 8u * (3 * S + 6 + 2 * R);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  TileCursor cur;
+  cur.init(p.wp, blockIdx.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(relu_done(s), 4);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(gfull, 1);
+    mbar_init(gempty, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf(a), 1);
+      mbar_init(acce(a), 4);
+    }
+    for (int m = 0; m < R; ++m) {
+      mbar_init(maskfull(m), 4);
+      mbar_init(maskfree(m), 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  {
+    // Zero rows d+1 .. d+15 of the G image buffer and build the ones region:
+    // row t holds bf16 1.0 in column 0 (32-byte swizzle: chunk c of row t sits
+    // at chunk slot c ^ ((t >> 2) & 1)), zeros elsewhere.
+    constexpr int kPadRows = G::kNPad - G::kStateRows;
+    constexpr int kPadChunks = G::kAtoms * kPadRows * (G::kRowBytes / 16);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int idx = threadIdx.x; idx < kPadChunks; idx += C::kThreads) {
+      const int ch = idx % (G::kRowBytes / 16);
+      const int rr = (idx / (G::kRowBytes / 16)) % kPadRows;
+      const int at = idx / ((G::kRowBytes / 16) * kPadRows);
+      st_shared_v4(g_buf + at * (G::kNPad * G::kRowBytes) + (G::kStateRows + rr) * G::kRowBytes +
+                       ch * 16,
+                   z);
+    }
+    for (int t = threadIdx.x; t < kTileTokens; t += C::kThreads) {
+      const uint32_t row = ones_buf + t * 32;
+      const int slot0 = (t >> 2) & 1;
+      st_shared_v4(row + slot0 * 16, make_uint4(0x3F80u, 0, 0, 0));
+      st_shared_v4(row + (slot0 ^ 1) * 16, z);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // G images of the reverse scan
+      int64_t issued = 0, seg = 0;
+      int b = 0, f = 0, h = 0;
+      for (; cur.valid(); cur.advance(), ++issued) {
+        if (cur.first) {
+          unit_coords(cur.u, p.H, p.F, b, f, h);
+          if (!mbar_wait(gempty, static_cast<uint32_t>((seg & 1) ^ 1), abort, kCode)) break;
+          mbar_arrive_expect_tx(gfull, G::kImageBytes);
+          const uint8_t* src = p.gimage + static_cast<int64_t>(cur.u) * G::kImageBytes;
+#pragma unroll
+          for (int a = 0; a < G::kAtoms; ++a)
+            bulk_load(g_buf + a * G::kNPad * G::kRowBytes, src + a * G::kImageAtomBytes,
+                      G::kImageAtomBytes, gfull);
+          ++seg;
+        }
+        const int s = static_cast<int>(issued % S);
+        if (!mbar_wait(empty(s), static_cast<uint32_t>(((issued / S) & 1) ^ 1), abort, kCode))
+          break;
+        const int t = cur.t;
+        mbar_arrive_expect_tx(full(s), 2u * G::kTileBytes);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a) {
+          tma_load_5d(v_buf(s) + a * G::kAtomTileBytes, &tm_v, full(s), a * G::kAtomElems, h,
+                      t * kTileTokens, f, b);
+          tma_load_5d(k_buf(s) + a * G::kAtomTileBytes, &tm_k, full(s), a * G::kAtomElems, h,
+                      t * kTileTokens, f, b);
+        }
+      }
+      for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
+      if (seg > 0) mbar_wait_drain(gfull, static_cast<uint32_t>((seg - 1) & 1));
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_dk = idesc_bf16_f32(128, D, false, true);   // B MN-major
+      constexpr uint32_t idesc_dv = idesc_bf16_f32(128, D, false, false);  // B K-major
+      constexpr int KPA = G::kAtomElems / 16;
+      constexpr uint32_t kGAtom = G::kNPad * G::kRowBytes;
+      int64_t i = 0, seg = 0;
+      for (; cur.valid(); cur.advance(), ++i) {
+        if (cur.first) {
+          if (!mbar_wait(gfull, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        }
+        const int ab = static_cast<int>(i & 1);
+        if (!mbar_wait(acce(ab), static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort, kCode)) break;
+        const int s = static_cast<int>(i % S);
+        if (!mbar_wait(relu_done(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+        tc_fence_after();
+        const uint32_t acc_dk = tmem + ab * 256;
+        const uint32_t acc_dv = acc_dk + 128;
+        // dk~ = [v | 1] . G^T : K over value columns j (d) plus the ones column
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc(v_buf(s) + (kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32,
+                                        16, G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(g_buf + kk * 2 * G::kGroupBytes, kGAtom, G::kGroupBytes,
+                                        G::kLayout);
+          mma_bf16(acc_dk, ad, bd, idesc_dk, kk > 0 ? 1u : 0u);
+        }
+        {
+          const uint64_t ad = smem_desc(ones_buf, 16, 256, kLayoutSW32);
+          const uint64_t bd = smem_desc(g_buf + (D / 16) * 2 * G::kGroupBytes, kGAtom,
+                                        G::kGroupBytes, G::kLayout);
+          mma_bf16(acc_dk, ad, bd, idesc_dk, 1u);
+        }
+        // dv = phi(k) . G[:, :d] : K over key features i
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int a = kk / KPA, w = kk % KPA;
+          const uint64_t ad = smem_desc(k_buf(s) + a * G::kAtomTileBytes + w * 32, 16,
+                                        G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(g_buf + a * kGAtom + w * 32, 16, G::kGroupBytes, G::kLayout);
+          mma_bf16(acc_dv, ad, bd, idesc_dv, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(empty(s));
+        mma_commit(accf(ab));
+        if (cur.last) {
+          mma_commit(gempty);
+          ++seg;
+        }
+      }
+      mma_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- ReLU on k + sign mask
+    constexpr int CPR = G::kChunksPerRow;
+    constexpr int RPP = kTileTokens / CPR;
+    constexpr int CPA = G::kAtomElems / 8;
+    const int rt = threadIdx.x - 128;
+    const int c = rt % CPR;
+    const int r0 = rt / CPR;
+    const uint32_t off0 =
+        (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes + G::swz(r0, c % CPA) * 16;
+    int64_t i = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
+      const int s = static_cast<int>(i % S);
+      const int m = static_cast<int>(i % R);
+      if (!warp_wait(full(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+      if (!warp_wait(maskfree(m), static_cast<uint32_t>(((i / R) & 1) ^ 1), abort, kCode)) break;
+      const uint32_t base = k_buf(s) + off0;
+      uint8_t* mrow = mask_ring + m * C::kMaskBytes;
+#pragma unroll
+      for (int mm = 0; mm < CPR; ++mm) {
+        const uint32_t addr = base + mm * RPP * G::kRowBytes;
+        uint4 w = ld_shared_v4(addr);
+        relu8(w);
+        st_shared_v4(addr, w);
+        // bit e set <=> feature 8c+e of this token is positive
+        uint32_t bits = 0;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bits |= ((ws[e] & 0x7FFFu) != 0u ? 1u : 0u) << (2 * e);
+          bits |= ((ws[e] & 0x7FFF0000u) != 0u ? 1u : 0u) << (2 * e + 1);
+        }
+        mrow[(r0 + mm * RPP) * (D / 8) + c] = static_cast<uint8_t>(bits);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(relu_done(s));
+        mbar_arrive(maskfull(m));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // token within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int64_t i = 0;
+    int b = 0, f = 0, h = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
+      const int ab = static_cast<int>(i & 1);
+      const int m = static_cast<int>(i % R);
+      if (!warp_wait(accf(ab), static_cast<uint32_t>((i >> 1) & 1), abort, kCode)) break;
+      if (!warp_wait(maskfull(m), static_cast<uint32_t>((i / R) & 1), abort, kCode)) break;
+      tc_fence_after();
+      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+      const int tok0 = cur.t * kTileTokens + q4 * 32;
+      // the row's sign mask
+      const uint4 mk = *reinterpret_cast<const uint4*>(mask_ring + m * C::kMaskBytes + row * (D / 8));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(maskfree(m));
+      const uint32_t mwords[4] = {mk.x, mk.y, mk.z, mk.w};
+#pragma unroll
+      for (int out = 0; out < 2; ++out) {  // 0: dk (masked), 1: dv
+        const uint32_t tb = tmem + lane_base + ab * 256 + out * 128;
+        const CUtensorMap* tm = out == 0 ? &tm_dk : &tm_dv;
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a) {
+          const int buf = static_cast<int>((i * 2 * G::kAtoms + out * G::kAtoms + a) & 1);
+          const uint32_t stg = o_base + buf * C::kStageOutBytes;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int cc = 0; cc < G::kAtomElems / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld_32cols(tb + a * G::kAtomElems + cc * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const int col8 = (a * G::kAtomElems + cc * 32) / 8 + ch;  // 8-feature chunk index
+              const uint32_t mb = (mwords[col8 >> 2] >> (8 * (col8 & 3))) & 0xFFu;
+              float x[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                x[e] = __uint_as_float(r[8 * ch + e]);
+                if (out == 0 && ((mb >> e) & 1u) == 0u) x[e] = 0.f;
+              }
+              uint4 w;
+              w.x = pack_bf16x2(x[0], x[1]);
+              w.y = pack_bf16x2(x[2], x[3]);
+              w.z = pack_bf16x2(x[4], x[5]);
+              w.w = pack_bf16x2(x[6], x[7]);
+              st_shared_v4(stg + row * G::kRowBytes + G::swz(row, cc * 4 + ch) * 16, w);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (tok0 < p.T)
+              tma_store_5d(tm, stg + q4 * 32 * G::kRowBytes, a * G::kAtomElems, h, tok0, f, b);
+            bulk_commit_group();
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce(ab));
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace gla

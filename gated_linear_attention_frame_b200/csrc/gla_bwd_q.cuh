@@ -1,0 +1,440 @@
+// gla_bwd_q.cuh -- query side of the backward pass on tcgen05.
+//
+// For the queries of frame f, with S_f the forward prefix state:
+//   num_t = phi(q_t) S_f[:, :d],  den_t = phi(q_t) S_f[:, d] + eps
+//   dnum_t = dout_t / den_t,      dden_t = -(dout_t . num_t) / den_t^2
+//   dq_t  = 1[q_t > 0] * ([dnum_t | dden_t] S_f^T)
+//   L_f   = sum_{t in f} phi(q_t)^T [dnum_t | dden_t]     (frame f's state gradient)
+// Per 128-token tile, three contractions into TMEM:
+//   MMA1  [num | den] = phi(Q) S_f     A = phi(Q) K-major, B = S_f^T image K-major (N = d+16)
+//   MMA2  dq~ = D S_f^T                A = D K-major (K = d+16), B = S_f^T image MN-major
+//   MMA3  L_f += phi(Q)^T D            A = phi(Q) MN-major, B = D MN-major
+// where D = [dnum | dden | 0 ...] is built in shared memory, in bf16, by the
+// epilogue from MMA1's result and dout (read by the epilogue threads directly
+// from global memory, one token row per thread).  D's first d columns sit in
+// two 128-byte-swizzled atoms; the dden column and 15 zero columns in a
+// 32-byte-swizzled region of 32-byte rows, so that every operand view of it
+// (MMA2's last K step, MMA3's N = 16 part) is a whole swizzle atom.  The same
+// swizzled bytes serve as MMA2's K-major A and MMA3's MN-major B; the same
+// S_f^T image serves MMA1 (K-major) and MMA2 (MN-major).  L_f is accumulated
+// over a unit's tiles and written as an fp32 partial in the forward
+// increment's slot layout (row d = sum_t phi(q_t) dden_t) for the reverse scan.
+// Warp roles: 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
+#pragma once
+
+#include "gla_common.cuh"
+#include "gla_increment.cuh"  // warp_wait, unit_coords, IncCfg
+#include "sm100_ptx.cuh"
+
+namespace gla {
+
+template <int D>
+struct BwdQCfg {
+  using G = Geo<D>;
+  static_assert(D == 128, "the backward kernels are built for d = 128");
+  static constexpr int kStages = 3;
+  static constexpr int kSBufBytes = G::kAtoms * G::kNPad * G::kRowBytes;  // S_f^T image
+  static constexpr int kDMainBytes = G::kAtoms * G::kAtomTileBytes;       // dnum, 128-byte swizzle
+  static constexpr int kDPadBytes = kTileTokens * 32;                     // [dden | 0 x 15], 32-byte swizzle
+  static constexpr int kDBytes = kDMainBytes + kDPadBytes;
+  static constexpr int kStageOutBytes = G::kAtomTileBytes;
+  static constexpr int kAcc1 = 0;    // [num | den]  : N = d + 16 columns
+  static constexpr int kAcc2 = 160;  // dq~          : N = d
+  static constexpr int kAcc3 = 288;  // L_f          : N = d + 16
+  static constexpr int kTmemCols = 512;
+  static constexpr int kThreads = 320;
+  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + kDBytes +
+                                    2 * kStageOutBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+struct BwdQParams {
+  const uint8_t* image;   // [units][kImageBytes] bf16 S_f^T images (forward recompute)
+  const uint16_t* dout;   // bf16 [B, F*T, H, d]
+  float* partial;         // L_f partials [(units + G) slots][d + 1][d]
+  float eps;
+  WorkPlan wp;
+  int H, F, T;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    gla_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_dq, const BwdQParams p) {
+  using G = Geo<D>;
+  using C = BwdQCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr unsigned kCode = 32u;
+  constexpr int PF = IncCfg<D>::kPartialFloats;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto q_buf = [&](int s) { return sbase + s * G::kTileBytes; };
+  const uint32_t s_buf = sbase + S * G::kTileBytes;
+  const uint32_t d_buf = s_buf + C::kSBufBytes;
+  const uint32_t d_pad = d_buf + C::kDMainBytes;
+  const uint32_t o_base = d_buf + C::kDBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::kTileBytes + C::kSBufBytes +
+                                               C::kDBytes + 2 * C::kStageOutBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto qfull = [&](int s) { return bar0 + 8u * s; };
+  auto qrelu = [&](int s) { return bar0 + 8u * (S + s); };
+  auto qempty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  const uint32_t sfull = bar0 + 8u * (3 * S + 0);
+  const uint32_t sempty = bar0 + 8u * (3 * S + 1);
+  const uint32_t acc1_full = bar0 + 8u * (3 * S + 2);
+  const uint32_t acc1_free = bar0 + 8u * (3 * S + 3);
+  const uint32_t dfull = bar0 + 8u * (3 * S + 4);
+  const uint32_t dfree = bar0 + 8u * (3 * S + 5);
+  const uint32_t acc2_full = bar0 + 8u * (3 * S + 6);
+  const uint32_t acc2_free = bar0 + 8u * (3 * S + 7);
+  const uint32_t acc3_full = bar0 + 8u * (3 * S + 8);
+  const uint32_t acc3_free = bar0 + 8u * (3 * S + 9);
+  const uint32_t done_bar = bar0 + 8u * (3 * S + 10);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  TileCursor cur;
+  cur.init(p.wp, blockIdx.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(qfull(s), 1);
+      mbar_init(qrelu(s), 4);
+      mbar_init(qempty(s), 4);
+    }
+    mbar_init(sfull, 1);
+    mbar_init(sempty, 1);
+    mbar_init(acc1_full, 1);
+    mbar_init(acc1_free, 4);
+    mbar_init(dfull, 4);
+    mbar_init(dfree, 1);
+    mbar_init(acc2_full, 1);
+    mbar_init(acc2_free, 4);
+    mbar_init(acc3_full, 1);
+    mbar_init(acc3_free, 4);
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  {
+    // zero: the S image's padding rows, and D's pad region (only the chunk
+    // holding column 0, dden, is rewritten per tile)
+    constexpr int kPadRows = G::kNPad - G::kStateRows;
+    constexpr int kPadChunks = G::kAtoms * kPadRows * (G::kRowBytes / 16);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int idx = threadIdx.x; idx < kPadChunks; idx += C::kThreads) {
+      const int ch = idx % (G::kRowBytes / 16);
+      const int rr = (idx / (G::kRowBytes / 16)) % kPadRows;
+      const int at = idx / ((G::kRowBytes / 16) * kPadRows);
+      st_shared_v4(s_buf + at * (G::kNPad * G::kRowBytes) + (G::kStateRows + rr) * G::kRowBytes +
+                       ch * 16,
+                   z);
+    }
+    for (int o = threadIdx.x * 16; o < C::kDPadBytes; o += C::kThreads * 16)
+      st_shared_v4(d_pad + o, z);
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // S images of the forward recompute
+      int64_t issued = 0, seg = 0;
+      int b = 0, f = 0, h = 0;
+      for (; cur.valid(); cur.advance(), ++issued) {
+        if (cur.first) {
+          unit_coords(cur.u, p.H, p.F, b, f, h);
+          if (!mbar_wait(sempty, static_cast<uint32_t>((seg & 1) ^ 1), abort, kCode)) break;
+          mbar_arrive_expect_tx(sfull, G::kImageBytes);
+          const uint8_t* src = p.image + static_cast<int64_t>(cur.u) * G::kImageBytes;
+#pragma unroll
+          for (int a = 0; a < G::kAtoms; ++a)
+            bulk_load(s_buf + a * G::kNPad * G::kRowBytes, src + a * G::kImageAtomBytes,
+                      G::kImageAtomBytes, sfull);
+          ++seg;
+        }
+        const int s = static_cast<int>(issued % S);
+        if (!mbar_wait(qempty(s), static_cast<uint32_t>(((issued / S) & 1) ^ 1), abort, kCode))
+          break;
+        mbar_arrive_expect_tx(qfull(s), G::kTileBytes);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a)
+          tma_load_5d(q_buf(s) + a * G::kAtomTileBytes, &tm_q, qfull(s), a * G::kAtomElems, h,
+                      cur.t * kTileTokens, f, b);
+      }
+      for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait_drain(qfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
+      if (seg > 0) mbar_wait_drain(sfull, static_cast<uint32_t>((seg - 1) & 1));
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc1 = idesc_bf16_f32(128, G::kNPad, false, false);
+      constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc3 = idesc_bf16_f32(128, D, true, true);
+      constexpr uint32_t idesc3z = idesc_bf16_f32(128, 16, true, true);
+      constexpr int KPA = G::kAtomElems / 16;
+      constexpr uint32_t kSAtom = G::kNPad * G::kRowBytes;
+      int64_t i = 0, seg = 0;
+      for (; cur.valid(); cur.advance(), ++i) {
+        const uint32_t ph = static_cast<uint32_t>(i & 1);
+        if (cur.first) {
+          if (!mbar_wait(sfull, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        }
+        const int s = static_cast<int>(i % S);
+        if (!mbar_wait(qrelu(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+        if (!mbar_wait(acc1_free, ph ^ 1u, abort, kCode)) break;
+        tc_fence_after();
+        // MMA1: [num | den] = phi(Q) . S_f
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int a = kk / KPA, w = kk % KPA;
+          const uint64_t ad = smem_desc(q_buf(s) + a * G::kAtomTileBytes + w * 32, 16,
+                                        G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(s_buf + a * kSAtom + w * 32, 16, G::kGroupBytes, G::kLayout);
+          mma_bf16(tmem + C::kAcc1, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(acc1_full);
+        // wait for D of this tile, the free dq~ accumulator and (unit start) L_f's
+        if (!mbar_wait(dfull, ph, abort, kCode)) break;
+        if (!mbar_wait(acc2_free, ph ^ 1u, abort, kCode)) break;
+        if (cur.first &&
+            !mbar_wait(acc3_free, static_cast<uint32_t>((seg & 1) ^ 1), abort, kCode))
+          break;
+        tc_fence_after();
+        // MMA2: dq~ = D . S_f^T  (K over the d value columns, then the pad
+        // region: the normaliser column and 15 zeros)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int a = kk / KPA, w = kk % KPA;
+          const uint64_t ad = smem_desc(d_buf + a * G::kAtomTileBytes + w * 32, 16,
+                                        G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(s_buf + kk * 2 * G::kGroupBytes, kSAtom, G::kGroupBytes,
+                                        G::kLayout);
+          mma_bf16(tmem + C::kAcc2, ad, bd, idesc2, kk > 0 ? 1u : 0u);
+        }
+        {
+          const uint64_t ad = smem_desc(d_pad, 16, 256, kLayoutSW32);
+          const uint64_t bd = smem_desc(s_buf + (D / 16) * 2 * G::kGroupBytes, kSAtom,
+                                        G::kGroupBytes, G::kLayout);
+          mma_bf16(tmem + C::kAcc2, ad, bd, idesc2, 1u);
+        }
+        // MMA3: L_f += phi(Q)^T . D  (K over the tile's tokens; N = d value
+        // columns from the main atoms, N = 16 from the pad region)
+#pragma unroll
+        for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+          const uint32_t acc = (cur.first && kk == 0) ? 0u : 1u;
+          const uint64_t ad = smem_desc(q_buf(s) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                        G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(d_buf + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                        G::kGroupBytes, G::kLayout);
+          mma_bf16(tmem + C::kAcc3, ad, bd, idesc3, acc);
+          const uint64_t bz = smem_desc(d_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
+          mma_bf16(tmem + C::kAcc3 + D, ad, bz, idesc3z, acc);
+        }
+        mma_commit(dfree);
+        mma_commit(acc2_full);
+        if (cur.last) {
+          mma_commit(acc3_full);
+          mma_commit(sempty);
+          ++seg;
+        }
+      }
+      mma_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ ReLU
+    constexpr int CPR = G::kChunksPerRow;
+    constexpr int RPP = kTileTokens / CPR;
+    constexpr int CPA = G::kAtomElems / 8;
+    const int rt = threadIdx.x - 128;
+    const int c = rt % CPR;
+    const int r0 = rt / CPR;
+    const uint32_t off0 =
+        (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes + G::swz(r0, c % CPA) * 16;
+    int64_t i = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
+      const int s = static_cast<int>(i % S);
+      if (!warp_wait(qfull(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+      const uint32_t base = q_buf(s) + off0;
+#pragma unroll
+      for (int m = 0; m < CPR; ++m) {
+        const uint32_t addr = base + m * RPP * G::kRowBytes;
+        uint4 w = ld_shared_v4(addr);
+        relu8(w);
+        st_shared_v4(addr, w);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qrelu(s));
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // token within the tile (= key feature for L_f)
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int64_t i = 0, seg = 0;
+    int b = 0, f = 0, h = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
+      const uint32_t ph = static_cast<uint32_t>(i & 1);
+      const int s = static_cast<int>(i % S);
+      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+      const int tok = cur.t * kTileTokens + row;
+      const bool valid_tok = tok < p.T;
+      // dout row of this token (zero past the frame's end)
+      uint4 dv4[D / 8];
+      {
+        const uint16_t* src =
+            p.dout + ((static_cast<int64_t>(b) * p.F + f) * p.T + (valid_tok ? tok : 0)) *
+                         static_cast<int64_t>(p.H) * D +
+                     static_cast<int64_t>(h) * D;
+#pragma unroll
+        for (int x = 0; x < D / 8; ++x)
+          dv4[x] = valid_tok ? __ldg(reinterpret_cast<const uint4*>(src) + x) : make_uint4(0, 0, 0, 0);
+      }
+      // ---- Epi1: D = [dout / den | -(dout . num) / den^2]
+      if (!warp_wait(acc1_full, ph, abort, kCode)) break;
+      if (!warp_wait(dfree, ph ^ 1u, abort, kCode)) break;  // previous tile's MMA2/MMA3 done
+      tc_fence_after();
+      const uint32_t t1 = tmem + lane_base + C::kAcc1;
+      uint32_t dr;
+      tmem_ld_1col(t1 + D, dr);
+      tmem_wait_ld();
+      const float rden = 1.0f / (__uint_as_float(dr) + p.eps);
+      float dot = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld_32cols(t1 + cc * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
+          uint32_t w[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint32_t wpair = (&dv4[0].x)[cc * 16 + ch * 4 + e2];
+            const float d0 = bf16lo_to_f32(wpair), d1 = bf16hi_to_f32(wpair);
+            dot = fmaf(d0, __uint_as_float(r[8 * ch + 2 * e2]), dot);
+            dot = fmaf(d1, __uint_as_float(r[8 * ch + 2 * e2 + 1]), dot);
+            w[e2] = pack_bf16x2(d0 * rden, d1 * rden);
+          }
+          const int chunk = cc * 4 + ch;
+          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
+          st_shared_v4(d_buf + a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16,
+                       make_uint4(w[0], w[1], w[2], w[3]));
+        }
+      }
+      tc_fence_before();
+      const float dden = valid_tok ? -dot * rden * rden : 0.f;
+      // pad region row: chunk 0 (columns 0..7) sits at chunk slot (row >> 2) & 1
+      st_shared_v4(d_pad + row * 32 + ((row >> 2) & 1) * 16,
+                   make_uint4(pack_bf16x2(dden, 0.f), 0u, 0u, 0u));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(acc1_free);
+        mbar_arrive(dfull);
+      }
+      // ---- Epi2: dq = 1[q > 0] * dq~
+      if (!warp_wait(acc2_full, ph, abort, kCode)) break;
+      tc_fence_after();
+      const uint32_t t2 = tmem + lane_base + C::kAcc2;
+      const int tok0 = cur.t * kTileTokens + q4 * 32;
+#pragma unroll
+      for (int a = 0; a < G::kAtoms; ++a) {
+        const int buf = static_cast<int>((i * G::kAtoms + a) & 1);
+        const uint32_t stg = o_base + buf * C::kStageOutBytes;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < G::kAtomElems / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(t2 + a * G::kAtomElems + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int cin = cc * 4 + ch;
+            const uint4 qv = ld_shared_v4(q_buf(s) + a * G::kAtomTileBytes + row * G::kRowBytes +
+                                          G::swz(row, cin) * 16);
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t bits = (e & 1) ? (qw[e >> 1] >> 16) : (qw[e >> 1] & 0xFFFFu);
+              x[e] = (bits & 0x7FFFu) != 0u ? __uint_as_float(r[8 * ch + e]) : 0.f;
+            }
+            uint4 w;
+            w.x = pack_bf16x2(x[0], x[1]);
+            w.y = pack_bf16x2(x[2], x[3]);
+            w.z = pack_bf16x2(x[4], x[5]);
+            w.w = pack_bf16x2(x[6], x[7]);
+            st_shared_v4(stg + row * G::kRowBytes + G::swz(row, cin) * 16, w);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (tok0 < p.T)
+            tma_store_5d(&tm_dq, stg + q4 * 32 * G::kRowBytes, a * G::kAtomElems, h, tok0, f, b);
+          bulk_commit_group();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(acc2_free);
+        mbar_arrive(qempty(s));  // phi(Q) of this stage no longer read (mask, MMA3 done)
+      }
+      // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
+      if (cur.last) {
+        if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        tc_fence_after();
+        float* dst = p.partial + cur.slot() * static_cast<int64_t>(PF) + row;
+        const uint32_t t3 = tmem + lane_base + C::kAcc3;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(t3 + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+        }
+        uint32_t zr;
+        tmem_ld_1col(t3 + D, zr);
+        tmem_wait_ld();
+        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc3_free);
+        ++seg;
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace gla

@@ -147,6 +147,59 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v,
 size_t gla_noalloc_scratch_bytes(void);
 
 /*
+ * gla_backward -- gradients of one gla_forward call (head dim d = 128 only).
+ *
+ * The pages train the video model end to end but give no gradient formulas;
+ * these are the exact derivatives of the forward definition above.  With
+ * L = sum(dout * out) + sum(dstate_out * state_out), per (b, h) and frame f:
+ *   dnum_t = dout_t / den_t,  dden_t = -(dout_t . out_t) / den_t
+ *   dq_t   = 1[q_t > 0] * ([dnum_t | dden_t] S_f^T)
+ *   G_f    = sum_{t in f} phi(q_t)^T [dnum_t | dden_t] + a_{f+1} G_{f+1},
+ *            G_{frames-1} adds dstate_out       (G_f = dL/dS_f, d x (d+1))
+ *   dk_t   = 1[k_t > 0] * ([v_t | 1] G_f^T),   dv_t = phi(k_t) G_f[:, :d]
+ *   dgate_logits[b, f, h] = a_f (1 - a_f) <G_f, S_{f-1}>,  dstate_in = a_0 G_0
+ * The forward states are recomputed (nothing is saved between the calls).
+ *
+ * Arguments (device pointers):
+ *   q, k, v, gate_logits, state_in, B, H, frames, tokens_per_frame, eps
+ *                 exactly as given to gla_forward (state_in may be NULL).
+ *   dout          bf16 [B, frames * tokens_per_frame, H, d], 16-byte aligned.
+ *   dstate_out    fp32 [B, H, d, d + 1] or NULL (zero).
+ *   dq, dk, dv    bf16 outputs, same shape and alignment as q; must not
+ *                 overlap any input.
+ *   dgate_logits  fp32 [B, frames, H] output; must not be NULL when
+ *                 B * H * frames > 0.
+ *   dstate_in     fp32 [B, H, d, d + 1] output or NULL (not written).  Written
+ *                 even when state_in is NULL (the gradient at the zero state).
+ *   d             must be 128 (GLA_ERR_UNSUPPORTED_D otherwise).
+ * Memory: a workspace of about (B*H*frames*10 + #SMs*4) * (d+1)*d bytes from
+ * the same pool as gla_forward, freed on `stream`.  Return codes and error
+ * behaviour as gla_forward.
+ */
+int gla_backward(const void* q, const void* k, const void* v,
+                 const float* gate_logits, const float* state_in,
+                 const void* dout, const float* dstate_out,
+                 void* dq, void* dk, void* dv,
+                 float* dgate_logits, float* dstate_in,
+                 int B, int H, int frames, int tokens_per_frame, int d,
+                 float eps, cudaStream_t stream);
+
+/*
+ * gla_backward_timed -- gla_backward that records seven caller-created CUDA
+ * events on `stream`: events[0] before the first kernel and events[i] after
+ * the i-th of the six kernels (state increments, forward scan, query-side
+ * gradients, reverse scan, gate gradients, key/value gradients).  `events`
+ * is a host array of 7 cudaEvent_t.
+ */
+int gla_backward_timed(const void* q, const void* k, const void* v,
+                       const float* gate_logits, const float* state_in,
+                       const void* dout, const float* dstate_out,
+                       void* dq, void* dk, void* dv,
+                       float* dgate_logits, float* dstate_in,
+                       int B, int H, int frames, int tokens_per_frame, int d,
+                       float eps, cudaStream_t stream, cudaEvent_t* events);
+
+/*
  * gla_trim_workspace -- release the current device's unused workspace memory
  * held by the library's pool (memory of calls still in flight is kept).
  * Returns GLA_OK, GLA_ERR_DEVICE or GLA_ERR_LAUNCH.
@@ -161,7 +214,9 @@ const char* gla_error_string(int status);
  * library's device-side fault word of the current device.  Nonzero means a
  * kernel gave up a bounded wait (about one second) and returned early; its
  * output is then invalid.  Bit 0: state-increment kernel, bit 1: output
- * kernel.  `code` is a host pointer.  Returns GLA_OK or GLA_ERR_LAUNCH.
+ * kernel, bit 2: forward scan, bit 3: reverse scan, bit 4: key/value
+ * gradient kernel, bit 5: query gradient kernel.  `code` is a host pointer.
+ * Returns GLA_OK or GLA_ERR_LAUNCH.
  */
 int gla_device_fault(cudaStream_t stream, unsigned int* code);
 

@@ -83,6 +83,35 @@ def test_validation_before_any_cuda_call(lib):
     assert _call(lib, H=0) == gl.GLA_OK
 
 
+def _bcall(lib, d=128, B=1, H=1, F=1, T=16, **kw):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, s_in=None, dout=FAKE, ds_out=None, dq=FAKE,
+             dk=FAKE, dv=FAKE, dg=FAKE, ds_in=None)
+    p.update(kw)
+    return lib.gla_backward(p["q"], p["k"], p["v"], p["g"], p["s_in"], p["dout"], p["ds_out"],
+                            p["dq"], p["dk"], p["dv"], p["dg"], p["ds_in"], B, H, F, T, d, 1e-6,
+                            None)
+
+
+def test_backward_validation_before_any_cuda_call(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    assert _bcall(lib, d=64) == gl.GLA_ERR_UNSUPPORTED_D   # backward is built for d = 128
+    assert _bcall(lib, d=32) == gl.GLA_ERR_UNSUPPORTED_D
+    assert _bcall(lib, B=-1) == gl.GLA_ERR_SHAPE
+    for name in ("q", "k", "v", "dout", "dq", "dk", "dv", "dg", "g"):
+        assert _bcall(lib, **{name: None}) == gl.GLA_ERR_NULL, name
+    for name in ("q", "dout", "dq", "dk", "dv"):
+        assert _bcall(lib, **{name: FAKE + 8}) == gl.GLA_ERR_ALIGN, name
+    for name in ("dg", "ds_in", "ds_out", "s_in"):
+        assert _bcall(lib, **{name: FAKE + 2}) == gl.GLA_ERR_ALIGN, name
+    # no tokens: dq/dk/dv/dout may be NULL; no frames: dgate_logits may be NULL
+    assert _bcall(lib, B=0) == gl.GLA_OK
+    assert _bcall(lib, H=0, dg=None, dq=None) == gl.GLA_OK
+    st = lib.gla_backward_timed(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                                None, 1, 1, 1, 16, 128, 1e-6, None, None)
+    assert st == gl.GLA_ERR_NULL
+
+
 def test_timed_variant_requires_events(lib):
     import gated_linear_attention_frame_b200 as gl
 

@@ -26,7 +26,7 @@ from dataclasses import dataclass, replace
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "seed_for"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "seed_for"]
 
 BASE_SEED = 20261202
 
@@ -120,3 +120,19 @@ def make_state(w: Workload, device="cpu", seed: int | None = None):
     gen = torch.Generator(device=dev)
     gen.manual_seed((seed_for(w) if seed is None else seed) + 7)
     return _normal((w.B, w.H, w.d, w.d + 1), gen, dev)
+
+
+def make_grads(w: Workload, device="cpu", seed: int | None = None, dstate_out: bool = False,
+               dstate_scale: float = 1e-3):
+    """Upstream gradients for the backward pass: dout bf16 [B, tokens, H, d]
+    ~ N(0, 1) rounded to nearest even, and (if `dstate_out`) an fp32
+    [B, H, d, d+1] state gradient ~ N(0, dstate_scale^2), else None.  Drawn in
+    that order from a generator seeded with seed_for(w) + 11 (or `seed`)."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed((seed_for(w) if seed is None else seed) + 11)
+    dout = _normal((w.B, w.tokens, w.H, w.d), gen, dev).to(torch.bfloat16)
+    ds = None
+    if dstate_out:
+        ds = _normal((w.B, w.H, w.d, w.d + 1), gen, dev).mul_(dstate_scale)
+    return dout, ds
