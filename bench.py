@@ -1,9 +1,11 @@
 """Benchmark of the gated linear attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+                    [--mode forward|backward]
 
 One step = one gla_forward call (increment -> gated scan -> output kernels)
-over one batch of the workload, inputs resident in HBM.  With N > 1 (torchrun,
+over one batch of the workload, inputs resident in HBM; with --mode backward,
+one gla_backward call (d = 128) instead.  With N > 1 (torchrun,
 one process per GPU) every rank runs its own independent copy of the workload
 (heads and sequences are independent: weak scaling, no data-path
 collective); the timed region is bracketed by a barrier and a device
@@ -34,9 +36,10 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, make_inputs, make_state  # noqa: E402
+from workloads import WORKLOADS, make_grads, make_inputs, make_state  # noqa: E402
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
+METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "720p-5s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
@@ -106,6 +109,34 @@ def algorithmic_work(w, state_in: bool, state_out: bool = True) -> dict:
     flops = th * (4 * d * (d + 1) + d) + units * 2 * d * (d + 1)
     return {"increment": k1_bytes, "scan": k2_bytes, "output": k3_bytes,
             "bytes": k1_bytes + k2_bytes + k3_bytes, "flops": flops}
+
+
+def algorithmic_work_backward(w, state_in: bool, dstate_out: bool, dstate_in: bool) -> dict:
+    """Bytes and flops of the backward pass (no workspace traffic).
+    Per token-head, each kernel's own operands in bf16: the recompute's
+    increment reads k, v (4d bytes); the query kernel reads q, dout and writes
+    dq (6d); the key/value kernel reads k, v and writes dk, dv (8d).  The
+    layer's minimum reads q, k, v, dout once and writes dq, dk, dv once (14d).
+    Flops per token-head: increment 2d(d+1); [num | den], dq~ and L_f 2d(d+1)
+    each; dk~ 2d(d+1), dv 2d^2.  Per (b, f, h): gates and dgate (8 bytes) and
+    the scans' 2d(d+1) each way; per (b, h): the fp32 states read / written."""
+    d = w.d
+    th = w.B * w.tokens * w.H
+    bh = w.B * w.H
+    units = w.B * w.frames * w.H
+    sbytes = bh * d * (d + 1) * 4
+    work = {
+        "increment": th * 4 * d,
+        "scan": units * 4 + sbytes * int(state_in),
+        "bwd_q": th * 6 * d,
+        "scan_bwd": units * 4 + sbytes * (int(state_in) + int(dstate_out) + int(dstate_in)),
+        "dgate": units * 8,
+        "bwd_kv": th * 8 * d,
+    }
+    work["bytes"] = th * 14 * d + units * 8 + sbytes * (int(state_in) + int(dstate_out) +
+                                                         int(dstate_in))
+    work["flops"] = th * (10 * d * (d + 1) + 2 * d * d) + units * 4 * d * (d + 1)
+    return work
 
 
 class ClockSampler:
@@ -269,6 +300,68 @@ def time_oracle(w, budget_s: float, max_heads: int | None = None, device="cpu") 
 # ---------------------------------------------------------------- GPU arm
 
 
+def e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call, E, tokens):
+    """End-to-end metric through the public API with host buffers.  Each of E
+    steps copies `host_in` (pinned; None entries pass through as None) to
+    device buffers, runs `call(inputs, outputs)` on `stream` and copies the
+    outputs back to pinned host buffers, all inside the timed region.  Steps
+    are pipelined over three streams (H2D, compute, D2H) with double-buffered
+    device buffers, so step i+1's upload overlaps step i's compute and
+    download."""
+    host_out = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in dev_out]
+                for _ in range(2)]
+    dbuf = [[None if x is None else torch.empty(x.shape, dtype=x.dtype, device=dev)
+             for x in host_in] for _ in range(2)]
+    dout = [dev_out, [torch.empty_like(o) for o in dev_out]]
+    h2d = sum(x.numel() * x.element_size() for x in host_in if x is not None)
+    d2h = sum(o.numel() * o.element_size() for o in dev_out)
+    s_h2d = torch.cuda.Stream(dev)
+    s_d2h = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # call on buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # results of buffer b downloaded
+
+    def step(i):
+        bb = i % 2
+        with torch.cuda.stream(s_h2d):
+            if i >= 2:
+                s_h2d.wait_event(ev_done[bb])  # buffer bb's previous call has read it
+            for d_, h_ in zip(dbuf[bb], host_in):
+                if h_ is not None:
+                    d_.copy_(h_, non_blocking=True)
+            ev_in[bb].record(s_h2d)
+        stream.wait_event(ev_in[bb])
+        if i >= 2:
+            stream.wait_event(ev_out[bb])  # buffer bb's previous results downloaded
+        call(dbuf[bb], dout[bb])
+        ev_done[bb].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev_done[bb])
+            for h_, d_ in zip(host_out[bb], dout[bb]):
+                h_.copy_(d_, non_blocking=True)
+            ev_out[bb].record(s_d2h)
+
+    for i in range(2):  # warm the path
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_h2d.wait_event(e0)
+    for i in range(E):
+        step(i)
+    stream.wait_event(ev_out[(E - 1) % 2])
+    stream.wait_event(ev_out[E % 2])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / E
+    return {"value": round(world * tokens / (e_ms * 1e-3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E,
+            "ms_per_step": round(e_ms, 3),
+            "note": "pinned host buffers; H2D, call and D2H pipelined over 3 streams"}
+
+
 def run_gpu(args, w, dist, rank, local_rank, world):
     import gated_linear_attention_frame_b200 as gla
 
@@ -358,72 +451,20 @@ def run_gpu(args, w, dist, rank, local_rank, world):
 
     # End to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory, runs the call and copies out and
-    # state_out back, all inside the timed region.  Steps are pipelined over
-    # three streams (H2D, compute, D2H) with double-buffered device buffers,
-    # so step i+1's upload overlaps step i's compute and download.
+    # state_out back, all inside the timed region.
     e2e = None
     if not args.no_e2e:
-        E = max(2, min(K, args.e2e_steps))
-        host = [x.cpu().pin_memory() for x in sets[0]]
-        host_state = state_buf.cpu().pin_memory() if state_buf is not None else None
-        host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-        host_so = [torch.empty(so.shape, dtype=so.dtype).pin_memory() for _ in range(2)]
-        dbuf = [[torch.empty_like(x) for x in sets[0]] for _ in range(2)]
-        dstate = [torch.empty_like(state_buf) if state_buf is not None else None for _ in range(2)]
-        douts = [out, torch.empty_like(out)]
-        dsos = [so, torch.empty_like(so)]
-        h2d = sum(x.numel() * x.element_size() for x in host)
-        if host_state is not None:
-            h2d += host_state.numel() * 4
-        d2h = host_out[0].numel() * host_out[0].element_size() + host_so[0].numel() * 4
-        s_h2d = torch.cuda.Stream(dev)
-        s_d2h = torch.cuda.Stream(dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
-        ev_done = [torch.cuda.Event() for _ in range(2)]  # call on buffer b finished
-        ev_out = [torch.cuda.Event() for _ in range(2)]   # results of buffer b downloaded
+        host_in = [x.cpu().pin_memory() for x in sets[0]]
+        host_in.append(state_buf.cpu().pin_memory() if state_buf is not None else None)
+        dev_out = [out, so]
 
-        def e2e_step(i):
-            bb = i % 2
-            with torch.cuda.stream(s_h2d):
-                if i >= 2:
-                    s_h2d.wait_event(ev_done[bb])  # buffer bb's previous call has read it
-                for d_, h_ in zip(dbuf[bb], host):
-                    d_.copy_(h_, non_blocking=True)
-                if host_state is not None:
-                    dstate[bb].copy_(host_state, non_blocking=True)
-                ev_in[bb].record(s_h2d)
-            stream.wait_event(ev_in[bb])
-            if i >= 2:
-                stream.wait_event(ev_out[bb])  # buffer bb's previous results downloaded
-            q_, k_, v_, g_ = dbuf[bb]
-            gla.gla_forward(q_, k_, v_, g_, dstate[bb], dsos[bb], douts[bb], w.B, w.H, w.frames,
+        def call(bi, bo):
+            q_, k_, v_, g_, s_ = bi
+            gla.gla_forward(q_, k_, v_, g_, s_, bo[1], bo[0], w.B, w.H, w.frames,
                             w.tokens_per_frame, w.d, w.eps, stream)
-            ev_done[bb].record(stream)
-            with torch.cuda.stream(s_d2h):
-                s_d2h.wait_event(ev_done[bb])
-                host_out[bb].copy_(douts[bb], non_blocking=True)
-                host_so[bb].copy_(dsos[bb], non_blocking=True)
-                ev_out[bb].record(s_d2h)
 
-        for i in range(2):  # warm the path
-            e2e_step(i)
-        torch.cuda.synchronize(dev)
-        barrier(dist, dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        s_h2d.wait_event(e0)
-        for i in range(E):
-            e2e_step(i)
-        stream.wait_event(ev_out[(E - 1) % 2])
-        stream.wait_event(ev_out[E % 2])
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / E
-        e2e = {"value": round(world * w.total_tokens / (e_ms * 1e-3), 1), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E,
-               "ms_per_step": round(e_ms, 3),
-               "note": "pinned host buffers; H2D, call and D2H pipelined over 3 streams"}
+        e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
+                            max(2, min(K, args.e2e_steps)), w.total_tokens)
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -440,6 +481,146 @@ def run_gpu(args, w, dist, rank, local_rank, world):
         "gpu": torch.cuda.get_device_name(dev),
     }
     return res
+
+
+def run_gpu_backward(args, w, dist, rank, local_rank, world):
+    """One step = one gla_backward call over one batch of the workload
+    (recompute of the forward states, then the five gradient kernels)."""
+    import gated_linear_attention_frame_b200 as gla
+
+    if w.d != 128:
+        raise SystemExit("the backward pass is built for d = 128")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    q, k, v, g = make_inputs(w, device=dev)
+    s_in = make_state(w, device=dev)
+    dout, ds_out = make_grads(w, device=dev, dstate_out=s_in is not None)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty_like(g)
+    ds_in = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev) if s_in is not None else None
+    work = algorithmic_work_backward(w, s_in is not None, ds_out is not None, ds_in is not None)
+
+    def step(events=None):
+        a = (q, k, v, g, s_in, dout, ds_out, dq, dk, dv, dg, ds_in, w.B, w.H, w.frames,
+             w.tokens_per_frame, w.d, w.eps, stream)
+        if events is None:
+            gla.gla_backward(*a)
+        else:
+            gla.gla_backward_timed(*a, events)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_device_fault(stream) == 0
+
+    K = args.steps
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with clocks:
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_step = reduce_max(t0.elapsed_time(t1), dist, dev) / K
+    value = world * w.total_tokens / (ms_step * 1e-3)
+
+    names = ["increment", "scan", "bwd_q", "scan_bwd", "dgate", "bwd_kv"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    for e7 in evs:
+        for e in e7:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    for i in range(K):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    fault = gla.gla_device_fault(stream)
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs])
+    avg = per.mean(axis=0)
+    dom = int(np.argmax(avg))
+    achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": None, "traffic_unit": "bytes per launch (ncu dram read + write)",
+            "algorithmic_bytes_per_launch": work[names[dom]],
+            "peak_source": peaks["source"] + " (hbm_gbs)"}
+    t_roof = max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                 work["flops"] / (peaks["bf16_tflops"] * 1e12))
+    layer = {"algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
+             "roofline_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_step, 4),
+             "achieved_GBps": round(work["bytes"] / (ms_step * 1e-3) / 1e9, 1),
+             "kernel_ms": {n: round(float(a), 4) for n, a in zip(names, avg)},
+             "kernel_ms_note": "per-kernel means from a second pass of K calls with events "
+                               "between the kernels"}
+
+    e2e = None
+    if not args.no_e2e:
+        host_in = [x.cpu().pin_memory() for x in (q, k, v, g, dout)]
+        host_in += [None if x is None else x.cpu().pin_memory() for x in (s_in, ds_out)]
+        dev_out = [dq, dk, dv, dg] + ([ds_in] if ds_in is not None else [])
+
+        def call(bi, bo):
+            q_, k_, v_, g_, do_, s_, dso_ = bi
+            gla.gla_backward(q_, k_, v_, g_, s_, do_, dso_, bo[0], bo[1], bo[2], bo[3],
+                             bo[4] if len(bo) > 4 else None, w.B, w.H, w.frames,
+                             w.tokens_per_frame, w.d, w.eps, stream)
+
+        e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
+                            max(2, min(K, args.e2e_steps)), w.total_tokens)
+
+    return {
+        "metric": METRIC_BWD, "mode": "backward", "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": warm, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.frames,
+                   "tokens_per_frame": w.tokens_per_frame, "tokens_per_step_per_gpu": w.total_tokens,
+                   "state_in": "fp32 with dstate_out" if s_in is not None else "zero",
+                   "l2": "inputs larger than L2 (%.2f GB read+written per step); no flush"
+                         % (work["bytes"] / 1e9),
+                   "parallelism": "dp%d (independent sequences per GPU)" % world},
+        "roofline": roof, "layer_roofline": layer, "gpu_launches": 6 * K, "e2e": e2e,
+        "clocks": clocks.summary(), "device_fault": fault,
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+
+
+def time_oracle_backward(w, budget_s: float) -> dict:
+    """Time the fp64 gradient oracle on (b, h) slices until `budget_s` of CPU
+    work; tokens/s counts full-layer tokens (all heads)."""
+    import oracle
+
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)][:4]
+    slices = oracle_head_slices(w, pairs)
+    dout, _ = make_grads(w)
+    douts = [dout[b, :, h].clone() for (b, h) in pairs]
+    del dout
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        i = done % len(pairs)
+        q, k, v, g = slices[i]
+        oracle.gla_backward_head_manual(q, k, v, g, w.tokens_per_frame, douts[i], None, None,
+                                        w.eps)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": done * w.tokens / w.H / el, "unit": UNIT, "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": "%d (batch, head) slices of %s (%d frames x %d tokens each), fp64 numpy "
+                      "gradient oracle, %.1f s wall" % (done, w.name, w.frames,
+                                                        w.tokens_per_frame, el),
+            "seconds": round(el, 3)}
 
 
 def run_reference(args, w):
@@ -485,6 +666,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
+                    help="time gla_forward (the layer metric) or gla_backward")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=0,
                     help="override the workload's frame count (small profiling cases)")
@@ -507,9 +690,13 @@ def main(argv=None):
         print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
     dist = dist_init(world, "nccl")
     try:
-        res = run_gpu(args, w, dist, rank, local_rank, world)
+        if args.mode == "backward":
+            res = run_gpu_backward(args, w, dist, rank, local_rank, world)
+        else:
+            res = run_gpu(args, w, dist, rank, local_rank, world)
         if rank == 0 and world == 1 and args.cpu_budget > 0:
-            res["cpu_baseline"] = time_oracle(w, args.cpu_budget)
+            res["cpu_baseline"] = (time_oracle_backward(w, args.cpu_budget)
+                                   if args.mode == "backward" else time_oracle(w, args.cpu_budget))
         elif rank == 0:
             res["cpu_baseline"] = None
         if rank == 0:
