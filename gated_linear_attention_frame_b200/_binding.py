@@ -24,10 +24,25 @@ GLA_ERR_ALLOC = 5
 GLA_ERR_LAUNCH = 6
 GLA_ERR_DEVICE = 7
 GLA_ERR_SCRATCH = 8
+GLA_ERR_ROPE = 9
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
-            "gla_backward", "gla_backward_timed", "gla_trim_workspace", "gla_error_string",
-            "gla_device_fault", "gla_version")
+            "gla_forward_rope", "gla_forward_rope_timed", "gla_backward", "gla_backward_timed",
+            "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
+
+
+class RopeConfig(ctypes.Structure):
+    """gla_rope_config of include/gla.h (3D rotary position embedding)."""
+
+    _fields_ = [("grid_w", ctypes.c_int), ("frame_offset", ctypes.c_int),
+                ("dim_t", ctypes.c_int), ("dim_y", ctypes.c_int), ("dim_x", ctypes.c_int),
+                ("theta", ctypes.c_float)]
+
+
+def rope_config(grid_w: int, dims=(32, 48, 48), frame_offset: int = 0,
+                theta: float = 10000.0) -> RopeConfig:
+    return RopeConfig(int(grid_w), int(frame_offset), int(dims[0]), int(dims[1]), int(dims[2]),
+                      float(theta))
 
 
 class GLAError(RuntimeError):
@@ -58,6 +73,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward_timed.restype = i32
     lib.gla_forward_noalloc.argtypes = fwd
     lib.gla_forward_noalloc.restype = i32
+    rope_p = ctypes.POINTER(RopeConfig)
+    lib.gla_forward_rope.argtypes = fwd[:13] + [rope_p, vp]
+    lib.gla_forward_rope.restype = i32
+    lib.gla_forward_rope_timed.argtypes = fwd[:13] + [rope_p, vp, ctypes.POINTER(vp)]
+    lib.gla_forward_rope_timed.restype = i32
     bwd = [vp] * 12 + [i32, i32, i32, i32, i32, f32, vp]
     lib.gla_backward.argtypes = bwd
     lib.gla_backward.restype = i32
@@ -159,6 +179,37 @@ def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, fr
         raise GLAError(st, "gla_forward_noalloc")
 
 
+def gla_forward_rope(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
+                     tokens_per_frame, d, eps, rope: RopeConfig, stream=None) -> None:
+    """gla_forward with the 3D rotary position embedding (see include/gla.h)."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    st = lib.gla_forward_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in),
+                              _ptr(state_out), _ptr(out), int(B), int(H), int(frames),
+                              int(tokens_per_frame), int(d), float(eps),
+                              None if rope is None else ctypes.byref(rope), _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_rope")
+
+
+def gla_forward_rope_timed(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
+                           tokens_per_frame, d, eps, rope: RopeConfig, stream, events) -> None:
+    """gla_forward_rope that records 4 CUDA events around the kernels."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+    st = lib.gla_forward_rope_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
+                                    _ptr(state_in), _ptr(state_out), _ptr(out), int(B), int(H),
+                                    int(frames), int(tokens_per_frame), int(d), float(eps),
+                                    ctypes.byref(rope), _stream(stream),
+                                    ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_rope_timed")
+
+
 def _check_bwd_dtypes(dout, dstate_out, dq, dk, dv, dgate_logits, dstate_in):
     for name, t, dt in (("dout", dout, torch.bfloat16), ("dq", dq, torch.bfloat16),
                         ("dk", dk, torch.bfloat16), ("dv", dv, torch.bfloat16),
@@ -254,6 +305,23 @@ def forward(q, k, v, gate_logits, state_in=None, eps: float = 1e-6, out=None, st
     if state_out is None:
         state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
     gla_forward(q, k, v, gate_logits, state_in, state_out, out, B, H, frames, T, d, eps, stream)
+    return out, state_out
+
+
+def forward_rope(q, k, v, gate_logits, rope: RopeConfig, state_in=None, eps: float = 1e-6,
+                 out=None, state_out=None, stream=None):
+    """Convenience wrapper of gla_forward_rope; returns (out, state_out)."""
+    B, N, H, d = q.shape
+    frames = gate_logits.shape[1]
+    T = N // frames if frames else 0
+    if frames and N % frames:
+        raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None:
+        state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
+    gla_forward_rope(q, k, v, gate_logits, state_in, state_out, out, B, H, frames, T, d, eps,
+                     rope, stream)
     return out, state_out
 
 

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -28,6 +29,7 @@
 #include "gla_common.cuh"
 #include "gla_increment.cuh"
 #include "gla_output.cuh"
+#include "gla_rope.cuh"
 #include "gla_scan.cuh"
 #include "gla_scan_bwd.cuh"
 #include "sm100_ptx.cuh"
@@ -103,6 +105,13 @@ cudaError_t set_smem_attrs() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::ScanCfg<D, 3>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, gla::IncCfg<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla::gla_output_kernel<D, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::OutCfg<D, true>::kSmemBytes);
   if (e != cudaSuccess || D != 128) return e;
   e = cudaFuncSetAttribute(gla::gla_bwd_q_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::BwdQCfg<128>::kSmemBytes);
@@ -178,7 +187,20 @@ struct Args {
   int B, H, F, T, d;
   float eps;
   cudaStream_t stream;
+  const gla_rope_config* rope = nullptr;  // rotary variant when set
 };
+
+// Host-only checks of a rotary configuration; no CUDA call.
+int validate_rope(const gla_rope_config* r, int d) {
+  if (r == nullptr) return GLA_ERR_NULL;
+  const int dims[3] = {r->dim_t, r->dim_y, r->dim_x};
+  for (int n : dims)
+    if (n < 0 || n % 8 != 0) return GLA_ERR_ROPE;
+  if (dims[0] + dims[1] + dims[2] != d) return GLA_ERR_ROPE;
+  if (r->grid_w < 1 || r->frame_offset < 0 || r->frame_offset > (1 << 24)) return GLA_ERR_ROPE;
+  if (!(r->theta > 0.0f) || r->theta > 3.0e38f) return GLA_ERR_ROPE;  // rejects NaN and inf
+  return GLA_OK;
+}
 
 // Host-only checks; no CUDA call.
 int validate(const Args& a) {
@@ -225,7 +247,7 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned b
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int D>
+template <int D, bool kRope = false>
 int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
         const FixedScratch* fixed = nullptr) {
   using G = Geo<D>;
@@ -239,7 +261,25 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   const int64_t partial_bytes =
       W > 0 ? align256((units + G1) * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4) : 0;
   const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
-  const int64_t ws_bytes = partial_bytes + image_bytes;
+  // rotary variant: the (cos, sin) table and the fp32 normaliser column per unit
+  gla::RopeGeo rg{};
+  int64_t table_pairs = 0;
+  if (kRope && W > 0) {
+    rg.dt = a.rope->dim_t;
+    rg.dy = a.rope->dim_y;
+    rg.dx = a.rope->dim_x;
+    rg.grid_w = a.rope->grid_w;
+    rg.rows = (a.T + rg.grid_w - 1) / rg.grid_w;
+    rg.cols = a.T < rg.grid_w ? a.T : rg.grid_w;
+    rg.frames = a.F;
+    rg.frame_offset = a.rope->frame_offset;
+    rg.sec_y = static_cast<int64_t>(a.F) * (rg.dt / 2);
+    rg.sec_x = rg.sec_y + static_cast<int64_t>(rg.rows) * (rg.dy / 2);
+    table_pairs = rg.sec_x + static_cast<int64_t>(rg.cols) * (rg.dx / 2);
+  }
+  const int64_t table_bytes = align256(table_pairs * 8);
+  const int64_t zvec_bytes = (kRope && W > 0) ? align256(units * static_cast<int64_t>(D) * 4) : 0;
+  const int64_t ws_bytes = partial_bytes + image_bytes + table_bytes + zvec_bytes;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_out;
   if (W > 0) {
@@ -265,6 +305,12 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   }
   float* partial = reinterpret_cast<float*>(ws);
   uint8_t* image = ws ? ws + partial_bytes : nullptr;
+  float2* table = table_pairs > 0 ? reinterpret_cast<float2*>(ws + partial_bytes + image_bytes)
+                                  : nullptr;
+  float* zvec = zvec_bytes > 0
+                    ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + table_bytes)
+                    : nullptr;
+  rg.table = reinterpret_cast<const float4*>(table);
 
   int status = GLA_OK;
   auto check = [&]() {
@@ -276,15 +322,22 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   };
 
   record(0);
+  if (table_pairs > 0 && status == GLA_OK) {
+    const int64_t blocks = (table_pairs + 255) / 256;
+    gla::gla_rope_table_kernel<<<static_cast<unsigned>(blocks < 4 * di.sms ? blocks : 4 * di.sms),
+                                 256, 0, a.stream>>>(table, rg,
+                                                     std::log2(static_cast<double>(a.rope->theta)));
+    check();
+  }
   if (W > 0 && status == GLA_OK) {
-    gla::IncParams ip{partial, wp, a.H, a.F};
-    gla::gla_increment_kernel<D>
+    gla::IncParams ip{partial, wp, a.H, a.F, a.T, rg};
+    gla::gla_increment_kernel<D, kRope>
         <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
     check();
   }
   record(1);
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
-    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu};
+    gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu, zvec};
     using SC1 = gla::ScanCfg<D, 1>;
     using SC3 = gla::ScanCfg<D, 3>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
@@ -298,9 +351,10 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   }
   record(2);
   if (W > 0 && status == GLA_OK) {
-    gla::OutParams op{image, a.eps, wp, a.H, a.F, a.T};
-    if (launch_dependent(gla::gla_output_kernel<D>, G3, gla::OutCfg<D>::kThreads,
-                         gla::OutCfg<D>::kSmemBytes, a.stream, tm_q, tm_out, op) != cudaSuccess)
+    gla::OutParams op{image, a.eps, wp, a.H, a.F, a.T, zvec, rg};
+    if (launch_dependent(gla::gla_output_kernel<D, kRope>, G3, gla::OutCfg<D, kRope>::kThreads,
+                         gla::OutCfg<D, kRope>::kSmemBytes, a.stream, tm_q, tm_out,
+                         op) != cudaSuccess)
       status = GLA_ERR_LAUNCH;
     check();
   }
@@ -315,9 +369,17 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
 int forward_impl(const Args& a, cudaEvent_t* ev) {
   int st = validate(a);
   if (st != GLA_OK) return st;
+  if (a.rope != nullptr && (st = validate_rope(a.rope, a.d)) != GLA_OK) return st;
   if (static_cast<int64_t>(a.B) * a.H == 0) return GLA_OK;  // nothing to compute or write
   DeviceInfo di;
   if ((st = device_setup(&di)) != GLA_OK) return st;
+  if (a.rope != nullptr) {
+    switch (a.d) {
+      case 32: return run<32, true>(a, di, ev);
+      case 64: return run<64, true>(a, di, ev);
+      default: return run<128, true>(a, di, ev);
+    }
+  }
   switch (a.d) {
     case 32: return run<32>(a, di, ev);
     case 64: return run<64>(a, di, ev);
@@ -556,6 +618,26 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v, const float
 
 size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
+int gla_forward_rope(const void* q, const void* k, const void* v, const float* gate_logits,
+                     const float* state_in, float* state_out, void* out, int B, int H, int frames,
+                     int tokens_per_frame, int d, float eps, const gla_rope_config* rope,
+                     cudaStream_t stream) {
+  if (rope == nullptr) return GLA_ERR_NULL;
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream, rope};
+  return forward_impl(a, nullptr);
+}
+
+int gla_forward_rope_timed(const void* q, const void* k, const void* v, const float* gate_logits,
+                           const float* state_in, float* state_out, void* out, int B, int H,
+                           int frames, int tokens_per_frame, int d, float eps,
+                           const gla_rope_config* rope, cudaStream_t stream, cudaEvent_t* events) {
+  if (rope == nullptr || events == nullptr) return GLA_ERR_NULL;
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream, rope};
+  return forward_impl(a, events);
+}
+
 int gla_backward(const void* q, const void* k, const void* v, const float* gate_logits,
                  const float* state_in, const void* dout, const float* dstate_out, void* dq,
                  void* dk, void* dv, float* dgate_logits, float* dstate_in, int B, int H,
@@ -601,6 +683,9 @@ const char* gla_error_string(int status) {
     case GLA_ERR_DEVICE: return "no CUDA device of compute capability 10.x";
     case GLA_ERR_SCRATCH:
       return "problem needs more scratch than gla_forward_noalloc's fixed 32 MiB buffer";
+    case GLA_ERR_ROPE:
+      return "invalid rotary configuration (blocks: multiples of 8 summing to d; grid_w >= 1; "
+             "0 <= frame_offset <= 2^24; theta > 0 and finite)";
     default: return "unknown status";
   }
 }

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "gla_common.cuh"
+#include "gla_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace gla {
@@ -49,6 +50,8 @@ struct IncParams {
   float* partial;   // [(units + gridDim.x) slots][d + 1][d] fp32
   WorkPlan wp;      // tile assignment (gridDim.x == wp.G)
   int H, F;         // heads, frames
+  int T;            // tokens per frame (rotary variant)
+  RopeGeo rope;     // rotary variant only
 };
 
 // (b, f, h) of unit u = (b * F + f) * H + h.
@@ -69,7 +72,10 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return ok != 0;
 }
 
-template <int D>
+// kRope: the rotary variant (gla_rope.cuh): phi(K) is rotated in shared
+// memory after its normaliser sums are taken, so the contraction forms
+// (R phi(K))^T V while row d keeps sum phi(k).
+template <int D, bool kRope = false>
 __global__ void __launch_bounds__(320, 1)
     gla_increment_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const IncParams p) {
@@ -209,16 +215,33 @@ __global__ void __launch_bounds__(320, 1)
     for (int e = 0; e < 8; ++e) z[e] = 0.f;
     int64_t i = 0;
     uint32_t zround = 0;
+    RopeChunk rc{};
+    int frame = 0;
+    if constexpr (kRope) rc = rope_chunk(p.rope, c);
     for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
       if (!warp_wait(full(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
       const uint32_t base = a_buf(s) + off0;
+      RopeRowPos rp{};
+      if constexpr (kRope) {
+        if (cur.first) frame = static_cast<int>((cur.u / p.H) % p.F);
+        rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
+      }
 #pragma unroll
       for (int m = 0; m < CPR; ++m) {
         const uint32_t addr = base + m * RPP * G::kRowBytes;
         uint4 w = ld_shared_v4(addr);
         relu8(w);
-        st_shared_v4(addr, w);
+        if constexpr (kRope) {
+          uint4 wr = w;
+          float4 cs01, cs23;
+          rope_coeffs(p.rope, rc, frame, rp, p.T, cs01, cs23);
+          rotate8(wr, cs01, cs23);
+          st_shared_v4(addr, wr);
+          rp.next(RPP, p.rope.grid_w);
+        } else {
+          st_shared_v4(addr, w);
+        }
         z[0] += bf16lo_to_f32(w.x);
         z[1] += bf16hi_to_f32(w.x);
         z[2] += bf16lo_to_f32(w.y);

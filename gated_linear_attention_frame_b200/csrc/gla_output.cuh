@@ -21,11 +21,12 @@
 
 #include "gla_common.cuh"
 #include "gla_increment.cuh"  // warp_wait
+#include "gla_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace gla {
 
-template <int D>
+template <int D, bool kRope = false>
 struct OutCfg {
   using G = Geo<D>;
   static constexpr int kStages = (D == 128) ? 3 : 4;
@@ -33,9 +34,12 @@ struct OutCfg {
   static constexpr int kStageOutBytes = G::kAtomTileBytes;               // one staging buffer
   static constexpr int kTmemCols = (2 * G::kNPad <= 128) ? 128 : (2 * G::kNPad <= 256) ? 256 : 512;
   static constexpr int kThreads = 320;
-  static constexpr int kBarBytes = (3 * kStages + 9) * 8;
-  static constexpr int kSmemBytes =
-      1024 + kStages * G::kTileBytes + 2 * kSBufBytes + 2 * kStageOutBytes + kBarBytes + 16;
+  static constexpr int kDenRing = kRope ? 8 : 0;                          // per-tile normalisers
+  static constexpr int kDenBytes = kDenRing * kTileTokens * 4;
+  static constexpr int kBarCount = 3 * kStages + 9 + 2 * kDenRing;
+  static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + 2 * kSBufBytes +
+                                    2 * kStageOutBytes + kDenBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 struct OutParams {
@@ -43,14 +47,22 @@ struct OutParams {
   float eps;
   WorkPlan wp;           // tile assignment (gridDim.x == wp.G)
   int H, F, T;
+  const float* zvec;     // rotary variant: fp32 S_f[:, d] per unit, [units][d]
+  RopeGeo rope;          // rotary variant only
 };
 
-template <int D>
+// kRope: the rotary variant (gla_rope.cuh).  The ReLU warps rotate phi(Q) in
+// shared memory for the contraction (only its d value columns are used) and
+// form the un-rotated normaliser phi(q_t) . S_f[:, d] themselves, from the
+// scan's fp32 copy of S_f[:, d]; they pass it to the epilogue through a ring
+// of per-tile arrays in shared memory.
+template <int D, bool kRope = false>
 __global__ void __launch_bounds__(320, 1)
     gla_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_out, const OutParams p) {
   using G = Geo<D>;
-  using C = OutCfg<D>;
+  using C = OutCfg<D, kRope>;
+  constexpr int R = C::kDenRing;
   constexpr int S = C::kStages;
   constexpr unsigned kCode = 2u;
 
@@ -61,8 +73,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t q_base = sbase;
   const uint32_t s_base = q_base + S * G::kTileBytes;
   const uint32_t o_base = s_base + 2 * C::kSBufBytes;
+  float* den_ring = reinterpret_cast<float*>(smem + S * G::kTileBytes + 2 * C::kSBufBytes +
+                                             2 * C::kStageOutBytes);  // [R][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::kTileBytes + 2 * C::kSBufBytes +
-                                               2 * C::kStageOutBytes);
+                                               2 * C::kStageOutBytes + C::kDenBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto qfull = [&](int s) { return bar0 + 8u * s; };
   auto qrelu = [&](int s) { return bar0 + 8u * (S + s); };
@@ -72,7 +86,9 @@ __global__ void __launch_bounds__(320, 1)
   auto accf = [&](int a) { return bar0 + 8u * (3 * S + 4 + a); };
   auto acce = [&](int a) { return bar0 + 8u * (3 * S + 6 + a); };
   const uint32_t done_bar = bar0 + 8u * (3 * S + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 9);
+  auto denfull = [&](int m) { return bar0 + 8u * (3 * S + 9 + m); };
+  auto denfree = [&](int m) { return bar0 + 8u * (3 * S + 9 + R + m); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto q_buf = [&](int s) { return q_base + s * G::kTileBytes; };
   auto s_buf = [&](int b) { return s_base + b * C::kSBufBytes; };
@@ -95,6 +111,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(acce(b), 4);
     }
     mbar_init(done_bar, 1);
+    for (int m = 0; m < R; ++m) {
+      mbar_init(denfull(m), 4);
+      mbar_init(denfree(m), 4);
+    }
     *abort = 0;
     fence_mbar_init();
   }
@@ -213,17 +233,68 @@ __global__ void __launch_bounds__(320, 1)
     const int r0 = rt / CPR;
     const uint32_t off0 =
         (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes + G::swz(r0, c % CPA) * 16;
+    RopeChunk rc{};
+    int frame = 0;
+    float zc[8];  // rotary: S_f[8c .. 8c+7, d] of the current unit
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zc[e] = 0.f;
+    if constexpr (kRope) {
+      rc = rope_chunk(p.rope, c);
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // zvec comes from the scan kernel
+    }
     int64_t i = 0;
     for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
       if (!warp_wait(qfull(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
       const uint32_t base = q_buf(s) + off0;
+      if constexpr (!kRope) {
 #pragma unroll
-      for (int m = 0; m < CPR; ++m) {
-        const uint32_t addr = base + m * RPP * G::kRowBytes;
-        uint4 w = ld_shared_v4(addr);
-        relu8(w);
-        st_shared_v4(addr, w);
+        for (int m = 0; m < CPR; ++m) {
+          const uint32_t addr = base + m * RPP * G::kRowBytes;
+          uint4 w = ld_shared_v4(addr);
+          relu8(w);
+          st_shared_v4(addr, w);
+        }
+      } else {
+        const int mr = static_cast<int>(i % R);
+        if (!warp_wait(denfree(mr), static_cast<uint32_t>(((i / R) & 1) ^ 1), abort, kCode)) break;
+        if (cur.first) {
+          frame = static_cast<int>((cur.u / p.H) % p.F);
+          const float4* zp = reinterpret_cast<const float4*>(p.zvec + cur.u * D + c * 8);
+          const float4 z0 = __ldg(zp), z1 = __ldg(zp + 1);
+          zc[0] = z0.x; zc[1] = z0.y; zc[2] = z0.z; zc[3] = z0.w;
+          zc[4] = z1.x; zc[5] = z1.y; zc[6] = z1.z; zc[7] = z1.w;
+        }
+        RopeRowPos rp;
+        rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
+        float* den = den_ring + mr * kTileTokens;
+#pragma unroll
+        for (int m = 0; m < CPR; ++m) {
+          const uint32_t addr = base + m * RPP * G::kRowBytes;
+          uint4 w = ld_shared_v4(addr);
+          relu8(w);
+          // normaliser on the un-rotated features; the CPR lanes of a row
+          // hold its CPR chunks
+          float part = 0.f;
+          part = fmaf(bf16lo_to_f32(w.x), zc[0], part);
+          part = fmaf(bf16hi_to_f32(w.x), zc[1], part);
+          part = fmaf(bf16lo_to_f32(w.y), zc[2], part);
+          part = fmaf(bf16hi_to_f32(w.y), zc[3], part);
+          part = fmaf(bf16lo_to_f32(w.z), zc[4], part);
+          part = fmaf(bf16hi_to_f32(w.z), zc[5], part);
+          part = fmaf(bf16lo_to_f32(w.w), zc[6], part);
+          part = fmaf(bf16hi_to_f32(w.w), zc[7], part);
+#pragma unroll
+          for (int o = CPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          if (c == 0) den[r0 + m * RPP] = part;
+          float4 cs01, cs23;
+          rope_coeffs(p.rope, rc, frame, rp, p.T, cs01, cs23);
+          rotate8(w, cs01, cs23);
+          st_shared_v4(addr, w);
+          rp.next(RPP, p.rope.grid_w);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(denfull(mr));
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -241,12 +312,22 @@ __global__ void __launch_bounds__(320, 1)
       if (!warp_wait(accf(ab), static_cast<uint32_t>((i >> 1) & 1), abort, kCode)) break;
       tc_fence_after();
       const uint32_t tb = tmem + lane_base + ab * G::kNPad;
-      uint32_t dr;
-      tmem_ld_1col(tb + D, dr);
-      tmem_wait_ld();
-      const float rinv = 1.0f / (__uint_as_float(dr) + p.eps);
+      float den;
+      if constexpr (kRope) {
+        const int mr = static_cast<int>(i % R);
+        if (!warp_wait(denfull(mr), static_cast<uint32_t>((i / R) & 1), abort, kCode)) break;
+        den = den_ring[mr * kTileTokens + row];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(denfree(mr));
+      } else {
+        uint32_t dr;
+        tmem_ld_1col(tb + D, dr);
+        tmem_wait_ld();
+        den = __uint_as_float(dr);
+      }
+      const float rinv = 1.0f / (den + p.eps);
       if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
-      const int tok0 = cur.t * kTileTokens + q4 * 32;  // first token of this warp's rows  // first token of this warp's rows
+      const int tok0 = cur.t * kTileTokens + q4 * 32;  // first token of this warp's rows
 #pragma unroll
       for (int a = 0; a < G::kAtoms; ++a) {
         const int buf = static_cast<int>((i * G::kAtoms + a) & 1);

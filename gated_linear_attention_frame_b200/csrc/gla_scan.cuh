@@ -38,6 +38,7 @@ struct ScanParams {
   float* states;           // [units][d+1][d] fp32 S_f^T per frame, or nullptr (backward only)
   WorkPlan wp;             // increment kernel's tile assignment (valid if tpu > 0)
   int H, F, tpu;
+  float* zvec;             // [units][d] fp32 S_f[:, d] per frame, or nullptr (rotary variant)
 };
 
 template <int D, int kStagesT = 3>
@@ -218,6 +219,11 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
           w.z = pack_bf16x2(S8[4], S8[5]);
           w.w = pack_bf16x2(S8[6], S8[7]);
           *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) = w;
+        }
+        if (p.zvec != nullptr && j == D) {
+          float4* dst = reinterpret_cast<float4*>(p.zvec + u * D + c * 8);
+          dst[0] = make_float4(S8[0], S8[1], S8[2], S8[3]);
+          dst[1] = make_float4(S8[4], S8[5], S8[6], S8[7]);
         }
         if (p.states != nullptr) {
           float4* dst = reinterpret_cast<float4*>(p.states + u * PF + static_cast<int64_t>(j) * D +

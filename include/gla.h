@@ -53,7 +53,8 @@ typedef enum {
   GLA_ERR_ALLOC = 5,           /* stream-ordered workspace allocation failed */
   GLA_ERR_LAUNCH = 6,          /* a CUDA runtime call or kernel launch failed */
   GLA_ERR_DEVICE = 7,          /* no CUDA device, or not compute capability 10.x */
-  GLA_ERR_SCRATCH = 8          /* gla_forward_noalloc: problem exceeds the fixed scratch */
+  GLA_ERR_SCRATCH = 8,         /* gla_forward_noalloc: problem exceeds the fixed scratch */
+  GLA_ERR_ROPE = 9             /* gla_forward_rope: invalid rotary configuration */
 } gla_status;
 
 /*
@@ -145,6 +146,57 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v,
 
 /* Size in bytes of gla_forward_noalloc's fixed scratch array.  Host only. */
 size_t gla_noalloc_scratch_bytes(void);
+
+/*
+ * Rotary position embedding of gla_forward_rope.  The SANA-Video ICLR 2026
+ * talk (temporal modelling segment) adds a 3D RoPE to the linear attention
+ * without a formula; this library reads it in the RoFormer form for linear
+ * attention.  Token t of frame f sits at
+ *     (p_t, p_y, p_x) = (frame_offset + f, t / grid_w, t % grid_w);
+ * the head dim is split into feature blocks [dim_t | dim_y | dim_x], and pair
+ * j (features 2j, 2j+1 of a block of n features) turns by the angle
+ * p_axis * theta^(-2j/n).  With R_t the rotation of token t:
+ *     S_f[:, :d] = a_f S_{f-1}[:, :d] + (R phi(K_f))^T V_f
+ *     S_f[:, d]  = a_f S_{f-1}[:, d]  + phi(K_f)^T 1          (not rotated)
+ *     out_t = (R_t phi(q_t)) S_f[:, :d] / (phi(q_t) S_f[:, d] + eps)
+ * The state keeps the rotated keys: a stream of calls passes state_out on as
+ * state_in and advances frame_offset by the frames already processed.
+ */
+typedef struct {
+  int grid_w;        /* tokens per latent row, >= 1 (80 for a 46 x 80 grid) */
+  int frame_offset;  /* temporal position of the call's first frame, 0 .. 2^24 */
+  int dim_t;         /* feature blocks: multiples of 8 (0 allowed), */
+  int dim_y;         /*   dim_t + dim_y + dim_x == d              */
+  int dim_x;
+  float theta;       /* frequency base, > 0 and finite (e.g. 10000) */
+} gla_rope_config;
+
+/*
+ * gla_forward_rope -- gla_forward with the rotary position embedding above
+ * fused into the loads of the two tensor-core kernels.  Arguments as
+ * gla_forward, plus `rope` (host pointer, read during the call only).
+ * Returns GLA_ERR_NULL if rope is NULL and GLA_ERR_ROPE for an invalid
+ * configuration (nothing enqueued); otherwise as gla_forward.  The workspace
+ * adds a (cos, sin) table of 8 * (frames*dim_t/2 + rows*dim_y/2 +
+ * min(T, grid_w)*dim_x/2) bytes (rows = ceil(T / grid_w)) and 4*d bytes per
+ * (batch, frame, head).
+ */
+int gla_forward_rope(const void* q, const void* k, const void* v,
+                     const float* gate_logits,
+                     const float* state_in, float* state_out,
+                     void* out,
+                     int B, int H, int frames, int tokens_per_frame, int d,
+                     float eps, const gla_rope_config* rope, cudaStream_t stream);
+
+/* gla_forward_rope with four events recorded as in gla_forward_timed (the
+ * table kernel counts with the state-increment kernel). */
+int gla_forward_rope_timed(const void* q, const void* k, const void* v,
+                           const float* gate_logits,
+                           const float* state_in, float* state_out,
+                           void* out,
+                           int B, int H, int frames, int tokens_per_frame, int d,
+                           float eps, const gla_rope_config* rope, cudaStream_t stream,
+                           cudaEvent_t* events);
 
 /*
  * gla_backward -- gradients of one gla_forward call (head dim d = 128 only).

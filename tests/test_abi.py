@@ -46,11 +46,11 @@ def test_error_strings(lib):
     import gated_linear_attention_frame_b200 as g
 
     seen = set()
-    for st in range(0, 9):
+    for st in range(0, 10):
         s = g.gla_error_string(st)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 9
+    assert len(seen) == 10
     assert g.gla_error_string(99) == "unknown status"
     assert g.gla_version() >= 100
 
@@ -110,6 +110,36 @@ def test_backward_validation_before_any_cuda_call(lib):
     st = lib.gla_backward_timed(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE,
                                 None, 1, 1, 1, 16, 128, 1e-6, None, None)
     assert st == gl.GLA_ERR_NULL
+
+
+def test_rope_validation_before_any_cuda_call(lib):
+    import ctypes
+
+    import gated_linear_attention_frame_b200 as gl
+
+    def call(rope, d=128, **kw):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, out=FAKE)
+        p.update(kw)
+        return lib.gla_forward_rope(p["q"], p["k"], p["v"], p["g"], None, None, p["out"], 1, 1,
+                                    1, 16, d, 1e-6,
+                                    None if rope is None else ctypes.byref(rope), None)
+
+    assert call(None) == gl.GLA_ERR_NULL
+    bad = [gl.rope_config(80, (32, 48, 40)),         # blocks do not sum to d
+           gl.rope_config(80, (36, 44, 48)),         # not multiples of 8
+           gl.rope_config(80, (-8, 88, 48)),
+           gl.rope_config(0, (32, 48, 48)),          # grid_w < 1
+           gl.rope_config(80, (32, 48, 48), frame_offset=-1),
+           gl.rope_config(80, (32, 48, 48), theta=0.0),
+           gl.rope_config(80, (32, 48, 48), theta=float("inf")),
+           gl.rope_config(80, (32, 48, 48), theta=float("nan"))]
+    for r in bad:
+        assert call(r) == gl.GLA_ERR_ROPE, (r.grid_w, r.dim_t, r.dim_y, r.dim_x, r.theta)
+    assert call(gl.rope_config(8, (8, 8, 16)), d=32, q=None) == gl.GLA_ERR_NULL
+    assert call(gl.rope_config(8, (32, 48, 48)), d=48) == gl.GLA_ERR_UNSUPPORTED_D
+    # valid configuration, empty batch: nothing to do
+    assert lib.gla_forward_rope(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 0, 1, 1, 16, 128, 1e-6,
+                                ctypes.byref(gl.rope_config(80)), None) == gl.GLA_OK
 
 
 def test_timed_variant_requires_events(lib):
