@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, make_grads, make_inputs, make_state  # noqa: E402
+from workloads import WORKLOADS, make_grads, make_inputs, make_state, rope_dims  # noqa: E402
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
@@ -378,17 +378,25 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     out = torch.empty_like(sets[0][0])
     so = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev, dtype=torch.float32)
     work = algorithmic_work(w, state_in=state is not None)
+    rope = args.variant == "rope"
 
     def step(i, events=None):
         q, k, v, g = sets[i % nsets]
         s_in = state_buf  # streaming: the state carries from call to call
         s_out = state_buf if state_buf is not None else so
-        a = (q, k, v, g, s_in, s_out, out, w.B, w.H, w.frames, w.tokens_per_frame, w.d, w.eps,
-             stream)
-        if events is None:
-            gla.gla_forward(*a)
+        a = (q, k, v, g, s_in, s_out, out, w.B, w.H, w.frames, w.tokens_per_frame, w.d, w.eps)
+        if rope:
+            # a carried state advances the temporal position call by call
+            off = (i * w.frames) % (1 << 20) if state_buf is not None else 0
+            cfg = gla.rope_config(w.grid_w, rope_dims(w.d), off)
+            if events is None:
+                gla.gla_forward_rope(*a, cfg, stream)
+            else:
+                gla.gla_forward_rope_timed(*a, cfg, stream, events)
+        elif events is None:
+            gla.gla_forward(*a, stream)
         else:
-            gla.gla_forward_timed(*a, events)
+            gla.gla_forward_timed(*a, stream, events)
 
     warm = max(3, args.warmup)
     for i in range(warm):
@@ -460,14 +468,21 @@ def run_gpu(args, w, dist, rank, local_rank, world):
 
         def call(bi, bo):
             q_, k_, v_, g_, s_ = bi
-            gla.gla_forward(q_, k_, v_, g_, s_, bo[1], bo[0], w.B, w.H, w.frames,
-                            w.tokens_per_frame, w.d, w.eps, stream)
+            a = (q_, k_, v_, g_, s_, bo[1], bo[0], w.B, w.H, w.frames, w.tokens_per_frame, w.d,
+                 w.eps)
+            if rope:
+                gla.gla_forward_rope(*a, gla.rope_config(w.grid_w, rope_dims(w.d)), stream)
+            else:
+                gla.gla_forward(*a, stream)
 
         e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
                             max(2, min(K, args.e2e_steps)), w.total_tokens)
 
+    if rope:
+        roof["traffic"] = None  # the counters were taken on the plain kernels
     res = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": METRIC if not rope else METRIC.replace("attention", "attention + 3D RoPE", 1),
+        "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": warm, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.frames,
@@ -475,8 +490,11 @@ def run_gpu(args, w, dist, rank, local_rank, world):
                    "state_in": "carried fp32" if state is not None else "zero",
                    "l2": "inputs larger than L2 (%.2f GB read+written per step); no flush"
                          % (work["bytes"] / 1e9),
-                   "parallelism": "dp%d (independent sequences per GPU)" % world},
-        "roofline": roof, "layer_roofline": layer, "gpu_launches": 3 * K, "e2e": e2e,
+                   "parallelism": "dp%d (independent sequences per GPU)" % world,
+                   **({"rope": {"grid_w": w.grid_w, "dims": list(rope_dims(w.d)),
+                                "theta": 10000.0}} if rope else {})},
+        "roofline": roof, "layer_roofline": layer, "gpu_launches": (4 if rope else 3) * K,
+        "e2e": e2e,
         "clocks": clocks.summary(), "device_fault": fault,
         "gpu": torch.cuda.get_device_name(dev),
     }
@@ -668,6 +686,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
                     help="time gla_forward (the layer metric) or gla_backward")
+    ap.add_argument("--variant", choices=["plain", "rope"], default="plain",
+                    help="forward only: the plain layer or gla_forward_rope (3D RoPE)")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=0,
                     help="override the workload's frame count (small profiling cases)")

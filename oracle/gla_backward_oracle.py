@@ -84,7 +84,8 @@ def gla_backward_head(q, k, v, g, T, dout, state_in=None, dstate_out=None, eps=1
     return dq, dk, dv, dg, ds_in
 
 
-def gla_backward_head_manual(q, k, v, g, T, dout, state_in=None, dstate_out=None, eps=1e-6):
+def gla_backward_head_manual(q, k, v, g, T, dout, state_in=None, dstate_out=None, eps=1e-6,
+                             return_g=False):
     """The same gradients by the chain rule written out (numpy float64):
       dnum_t = dout_t / den_t,  dden_t = -(dout_t . out_t) / den_t
       dq_t   = 1[q_t > 0] * ([dnum_t | dden_t] S_f^T)
@@ -92,6 +93,7 @@ def gla_backward_head_manual(q, k, v, g, T, dout, state_in=None, dstate_out=None
       G_f    = dS_f + a_{f+1} G_{f+1},   G_F = dstate_out
       da_f   = <G_f, S_{f-1}>,  dg_f = da_f a_f (1 - a_f),  dstate_in = a_0 G_0
       dk_t   = 1[k_t > 0] * ([v_t | 1] G_f^T),  dv_t = k~_t G_f[:, :d]
+    With return_g, also returns the list of G_f (frame order) as a sixth item.
     """
     q, k, v, g, dout = (_t64(x).numpy() for x in (q, k, v, g, dout))
     g = g.reshape(-1)
@@ -112,6 +114,7 @@ def gla_backward_head_manual(q, k, v, g, T, dout, state_in=None, dstate_out=None
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     dg = np.zeros(F)
+    Gs = [None] * F
     G_next = np.zeros((d, d + 1)) if dstate_out is None else _t64(dstate_out).numpy().copy()
     a_next = 1.0
     for f in range(F - 1, -1, -1):
@@ -133,11 +136,14 @@ def gla_backward_head_manual(q, k, v, g, T, dout, state_in=None, dstate_out=None
         V1 = np.hstack([v[rows], np.ones((T, 1))])
         dk[rows] = (k[rows] > 0) * (V1 @ G.T)
         dv[rows] = Kf @ G[:, :d]
+        Gs[f] = G
         G_next = G
         a_next = a[f]
     ds_in = None
     if state_in is not None:
         ds_in = a[0] * G_next if F > 0 else G_next
+    if return_g:
+        return dq, dk, dv, dg, ds_in, Gs
     return dq, dk, dv, dg, ds_in
 
 

@@ -26,7 +26,8 @@ from dataclasses import dataclass, replace
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "seed_for"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "rope_dims",
+           "seed_for"]
 
 BASE_SEED = 20261202
 
@@ -46,6 +47,7 @@ class Workload:
     random_state_in: bool
     calls: int = 1      # consecutive streaming calls (state carried)
     eps: float = 1e-6
+    grid_w: int = 1     # latent grid width (token t of a frame sits at row t // grid_w)
 
     @property
     def tokens(self) -> int:
@@ -65,18 +67,25 @@ WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
         Workload("tiny", 0, B=1, H=2, d=32, frames=4, tokens_per_frame=16,
-                 g_mu=2.0, g_sigma=1.0, k_scaled=False, random_state_in=False),
+                 g_mu=2.0, g_sigma=1.0, k_scaled=False, random_state_in=False, grid_w=4),
         Workload("480p-5s", 1, B=2, H=20, d=128, frames=21, tokens_per_frame=1560,
-                 g_mu=3.0, g_sigma=1.0, k_scaled=True, random_state_in=False),
+                 g_mu=3.0, g_sigma=1.0, k_scaled=True, random_state_in=False, grid_w=52),
         Workload("720p-5s", 2, B=2, H=24, d=128, frames=21, tokens_per_frame=3680,
-                 g_mu=3.0, g_sigma=1.0, k_scaled=True, random_state_in=False),
+                 g_mu=3.0, g_sigma=1.0, k_scaled=True, random_state_in=False, grid_w=80),
         Workload("720p-60s", 3, B=1, H=24, d=128, frames=241, tokens_per_frame=3680,
-                 g_mu=4.0, g_sigma=0.5, k_scaled=True, random_state_in=False),
+                 g_mu=4.0, g_sigma=0.5, k_scaled=True, random_state_in=False, grid_w=80),
         Workload("stream", 4, B=8, H=24, d=128, frames=1, tokens_per_frame=3680,
                  g_mu=3.0, g_sigma=1.0, k_scaled=False, random_state_in=True,
-                 calls=64),
+                 calls=64, grid_w=80),
     ]
 }
+
+
+def rope_dims(d: int) -> tuple[int, int, int]:
+    """Feature blocks [temporal | height | width] of the rotary variant: a
+    quarter of the head dim for time, the rest split between the two spatial
+    axes (multiples of 8)."""
+    return {32: (8, 8, 16), 64: (16, 24, 24), 128: (32, 48, 48)}[d]
 
 
 def seed_for(w: Workload, call: int = 0) -> int:
