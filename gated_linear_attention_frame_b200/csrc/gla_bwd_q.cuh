@@ -19,6 +19,12 @@
 // S_f^T image serves MMA1 (K-major) and MMA2 (MN-major).  L_f is accumulated
 // over a unit's tiles and written as an fp32 partial in the forward
 // increment's slot layout (row d = sum_t phi(q_t) dden_t) for the reverse scan.
+// D enters MMA3 as a hi/lo pair of bf16 copies (D = D_hi + D_lo, D_lo the
+// bf16 rounding of the remainder): the gate gradient <G_f, S_{f-1}> and dk
+// sum thousands of products of L_f with random signs, and one bf16 rounding
+// of D would put their error near the tolerance; dq uses D_hi alone.
+// The ReLU warps keep a byte mask of q > 0 for the dq epilogue, so a q stage
+// is released as soon as MMA3 has read it.
 // Warp roles: 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
 #pragma once
 
@@ -32,20 +38,23 @@ template <int D>
 struct BwdQCfg {
   using G = Geo<D>;
   static_assert(D == 128, "the backward kernels are built for d = 128");
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 2;
   static constexpr int kSBufBytes = G::kAtoms * G::kNPad * G::kRowBytes;  // S_f^T image
   static constexpr int kDMainBytes = G::kAtoms * G::kAtomTileBytes;       // dnum, 128-byte swizzle
   static constexpr int kDPadBytes = kTileTokens * 32;                     // [dden | 0 x 15], 32-byte swizzle
-  static constexpr int kDBytes = kDMainBytes + kDPadBytes;
+  static constexpr int kDBytes = kDMainBytes + kDPadBytes;                // one copy (hi or lo)
   static constexpr int kStageOutBytes = G::kAtomTileBytes;
+  static constexpr int kMaskRing = 4;
+  static constexpr int kMaskBytes = kTileTokens * (D / 8);                // one bit per feature
   static constexpr int kAcc1 = 0;    // [num | den]  : N = d + 16 columns
   static constexpr int kAcc2 = 160;  // dq~          : N = d
   static constexpr int kAcc3 = 288;  // L_f          : N = d + 16
   static constexpr int kTmemCols = 512;
   static constexpr int kThreads = 320;
-  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
-  static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + kDBytes +
-                                    2 * kStageOutBytes + kBarCount * 8 + 16;
+  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing;
+  static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + 2 * kDBytes +
+                                    2 * kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 +
+                                    16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -74,11 +83,14 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t sbase = smem_u32(smem);
   auto q_buf = [&](int s) { return sbase + s * G::kTileBytes; };
   const uint32_t s_buf = sbase + S * G::kTileBytes;
-  const uint32_t d_buf = s_buf + C::kSBufBytes;
+  const uint32_t d_buf = s_buf + C::kSBufBytes;          // D_hi
   const uint32_t d_pad = d_buf + C::kDMainBytes;
-  const uint32_t o_base = d_buf + C::kDBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::kTileBytes + C::kSBufBytes +
-                                               C::kDBytes + 2 * C::kStageOutBytes);
+  const uint32_t l_buf = d_buf + C::kDBytes;             // D_lo
+  const uint32_t l_pad = l_buf + C::kDMainBytes;
+  const uint32_t o_base = l_buf + C::kDBytes;
+  uint8_t* mask_ring = smem + S * G::kTileBytes + C::kSBufBytes + 2 * C::kDBytes +
+                       2 * C::kStageOutBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + C::kMaskRing * C::kMaskBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto qfull = [&](int s) { return bar0 + 8u * s; };
   auto qrelu = [&](int s) { return bar0 + 8u * (S + s); };
@@ -94,6 +106,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t acc3_full = bar0 + 8u * (3 * S + 8);
   const uint32_t acc3_free = bar0 + 8u * (3 * S + 9);
   const uint32_t done_bar = bar0 + 8u * (3 * S + 10);
+  constexpr int R = C::kMaskRing;
+  auto maskfull = [&](int m) { return bar0 + 8u * (3 * S + 11 + m); };
+  auto maskfree = [&](int m) { return bar0 + 8u * (3 * S + 11 + R + m); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -106,7 +121,11 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(qfull(s), 1);
       mbar_init(qrelu(s), 4);
-      mbar_init(qempty(s), 4);
+      mbar_init(qempty(s), 1);
+    }
+    for (int m = 0; m < R; ++m) {
+      mbar_init(maskfull(m), 4);
+      mbar_init(maskfree(m), 4);
     }
     mbar_init(sfull, 1);
     mbar_init(sempty, 1);
@@ -136,8 +155,10 @@ __global__ void __launch_bounds__(320, 1)
                        ch * 16,
                    z);
     }
-    for (int o = threadIdx.x * 16; o < C::kDPadBytes; o += C::kThreads * 16)
+    for (int o = threadIdx.x * 16; o < C::kDPadBytes; o += C::kThreads * 16) {
       st_shared_v4(d_pad + o, z);
+      st_shared_v4(l_pad + o, z);
+    }
     fence_proxy_async_smem();
   }
   if (warp == 0) {
@@ -246,7 +267,13 @@ __global__ void __launch_bounds__(320, 1)
           mma_bf16(tmem + C::kAcc3, ad, bd, idesc3, acc);
           const uint64_t bz = smem_desc(d_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
           mma_bf16(tmem + C::kAcc3 + D, ad, bz, idesc3z, acc);
+          const uint64_t bl = smem_desc(l_buf + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                        G::kGroupBytes, G::kLayout);
+          mma_bf16(tmem + C::kAcc3, ad, bl, idesc3, 1u);
+          const uint64_t blz = smem_desc(l_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
+          mma_bf16(tmem + C::kAcc3 + D, ad, blz, idesc3z, 1u);
         }
+        mma_commit(qempty(s));
         mma_commit(dfree);
         mma_commit(acc2_full);
         if (cur.last) {
@@ -271,18 +298,33 @@ __global__ void __launch_bounds__(320, 1)
     int64_t i = 0;
     for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
+      const int mr = static_cast<int>(i % R);
       if (!warp_wait(qfull(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
+      if (!warp_wait(maskfree(mr), static_cast<uint32_t>(((i / R) & 1) ^ 1), abort, kCode)) break;
       const uint32_t base = q_buf(s) + off0;
+      uint8_t* mrow = mask_ring + mr * C::kMaskBytes;
 #pragma unroll
       for (int m = 0; m < CPR; ++m) {
         const uint32_t addr = base + m * RPP * G::kRowBytes;
         uint4 w = ld_shared_v4(addr);
         relu8(w);
         st_shared_v4(addr, w);
+        // bit e set <=> feature 8c + e of this token is positive
+        uint32_t bits = 0;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bits |= ((ws[e] & 0x7FFFu) != 0u ? 1u : 0u) << (2 * e);
+          bits |= ((ws[e] & 0x7FFF0000u) != 0u ? 1u : 0u) << (2 * e + 1);
+        }
+        mrow[(r0 + m * RPP) * (D / 8) + c] = static_cast<uint8_t>(bits);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(qrelu(s));
+      if (lane == 0) {
+        mbar_arrive(qrelu(s));
+        mbar_arrive(maskfull(mr));
+      }
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -293,7 +335,6 @@ __global__ void __launch_bounds__(320, 1)
     int b = 0, f = 0, h = 0;
     for (; cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
-      const int s = static_cast<int>(i % S);
       if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       const int tok = cur.t * kTileTokens + row;
       const bool valid_tok = tok < p.T;
@@ -325,26 +366,32 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
-          uint32_t w[4];
+          uint32_t w[4], wl[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const uint32_t wpair = (&dv4[0].x)[cc * 16 + ch * 4 + e2];
             const float d0 = bf16lo_to_f32(wpair), d1 = bf16hi_to_f32(wpair);
             dot = fmaf(d0, __uint_as_float(r[8 * ch + 2 * e2]), dot);
             dot = fmaf(d1, __uint_as_float(r[8 * ch + 2 * e2 + 1]), dot);
-            w[e2] = pack_bf16x2(d0 * rden, d1 * rden);
+            const float x0 = d0 * rden, x1 = d1 * rden;
+            w[e2] = pack_bf16x2(x0, x1);
+            wl[e2] = pack_bf16x2(x0 - bf16lo_to_f32(w[e2]), x1 - bf16hi_to_f32(w[e2]));
           }
           const int chunk = cc * 4 + ch;
           const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
-          st_shared_v4(d_buf + a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16,
-                       make_uint4(w[0], w[1], w[2], w[3]));
+          const uint32_t off = a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16;
+          st_shared_v4(d_buf + off, make_uint4(w[0], w[1], w[2], w[3]));
+          st_shared_v4(l_buf + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
         }
       }
       tc_fence_before();
       const float dden = valid_tok ? -dot * rden * rden : 0.f;
+      const uint32_t dden_hi = pack_bf16x2(dden, 0.f);
+      const float dden_lo = dden - bf16lo_to_f32(dden_hi);
       // pad region row: chunk 0 (columns 0..7) sits at chunk slot (row >> 2) & 1
-      st_shared_v4(d_pad + row * 32 + ((row >> 2) & 1) * 16,
-                   make_uint4(pack_bf16x2(dden, 0.f), 0u, 0u, 0u));
+      const uint32_t poff = row * 32 + ((row >> 2) & 1) * 16;
+      st_shared_v4(d_pad + poff, make_uint4(dden_hi, 0u, 0u, 0u));
+      st_shared_v4(l_pad + poff, make_uint4(pack_bf16x2(dden_lo, 0.f), 0u, 0u, 0u));
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -353,7 +400,14 @@ __global__ void __launch_bounds__(320, 1)
       }
       // ---- Epi2: dq = 1[q > 0] * dq~
       if (!warp_wait(acc2_full, ph, abort, kCode)) break;
+      const int mr = static_cast<int>(i % R);
+      if (!warp_wait(maskfull(mr), static_cast<uint32_t>((i / R) & 1), abort, kCode)) break;
       tc_fence_after();
+      const uint4 mk =
+          *reinterpret_cast<const uint4*>(mask_ring + mr * C::kMaskBytes + row * (D / 8));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(maskfree(mr));
+      const uint32_t mwords[4] = {mk.x, mk.y, mk.z, mk.w};
       const uint32_t t2 = tmem + lane_base + C::kAcc2;
       const int tok0 = cur.t * kTileTokens + q4 * 32;
 #pragma unroll
@@ -370,15 +424,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int cin = cc * 4 + ch;
-            const uint4 qv = ld_shared_v4(q_buf(s) + a * G::kAtomTileBytes + row * G::kRowBytes +
-                                          G::swz(row, cin) * 16);
-            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            const int col8 = (a * G::kAtomElems + cc * 32) / 8 + ch;  // 8-feature chunk index
+            const uint32_t mb = (mwords[col8 >> 2] >> (8 * (col8 & 3))) & 0xFFu;
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t bits = (e & 1) ? (qw[e >> 1] >> 16) : (qw[e >> 1] & 0xFFFFu);
-              x[e] = (bits & 0x7FFFu) != 0u ? __uint_as_float(r[8 * ch + e]) : 0.f;
-            }
+            for (int e = 0; e < 8; ++e)
+              x[e] = ((mb >> e) & 1u) != 0u ? __uint_as_float(r[8 * ch + e]) : 0.f;
             uint4 w;
             w.x = pack_bf16x2(x[0], x[1]);
             w.y = pack_bf16x2(x[2], x[3]);
@@ -397,10 +448,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(acc2_free);
-        mbar_arrive(qempty(s));  // phi(Q) of this stage no longer read (mask, MMA3 done)
-      }
+      if (lane == 0) mbar_arrive(acc2_free);
       // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
       if (cur.last) {
         if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
