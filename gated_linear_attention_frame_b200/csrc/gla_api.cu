@@ -107,7 +107,8 @@ cudaError_t set_smem_attrs() {
                            gla::ScanCfg<D, 3>::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, gla::IncCfg<D>::kSmemBytes);
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::IncCfg<D, true>::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_output_kernel<D, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -332,7 +333,8 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   if (W > 0 && status == GLA_OK) {
     gla::IncParams ip{partial, wp, a.H, a.F, a.T, rg};
     gla::gla_increment_kernel<D, kRope>
-        <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+        <<<G1, gla::IncCfg<D, kRope>::kThreads, gla::IncCfg<D, kRope>::kSmemBytes, a.stream>>>(
+            tm_k, tm_v, ip);
     check();
   }
   record(1);

@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(320, 1)
                                         G::kGroupBytes, G::kLayout);
           mma_bf16(tmem + C::kAcc2, ad, bd, idesc2, 1u);
         }
+        mma_commit(acc2_full);  // the dq epilogue need not wait for MMA3
         // MMA3: L_f += phi(Q)^T . D  (K over the tile's tokens; N = d value
         // columns from the main atoms, N = 16 from the pad region)
 #pragma unroll
@@ -275,7 +276,6 @@ __global__ void __launch_bounds__(320, 1)
         }
         mma_commit(qempty(s));
         mma_commit(dfree);
-        mma_commit(acc2_full);
         if (cur.last) {
           mma_commit(acc3_full);
           mma_commit(sempty);
@@ -333,22 +333,28 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     int64_t i = 0, seg = 0;
     int b = 0, f = 0, h = 0;
+    // dout row of this thread's token in a tile (zero past the frame's end);
+    // the next tile's row is loaded while the current tile's dq is written
+    auto load_dout = [&](const TileCursor& tc, uint4 (&dst)[D / 8]) {
+      int bb, ff, hh;
+      unit_coords(tc.u, p.H, p.F, bb, ff, hh);
+      const int tk = tc.t * kTileTokens + row;
+      const bool ok = tk < p.T;
+      const uint16_t* src =
+          p.dout + ((static_cast<int64_t>(bb) * p.F + ff) * p.T + (ok ? tk : 0)) *
+                       static_cast<int64_t>(p.H) * D +
+                   static_cast<int64_t>(hh) * D;
+#pragma unroll
+      for (int x = 0; x < D / 8; ++x)
+        dst[x] = ok ? __ldg(reinterpret_cast<const uint4*>(src) + x) : make_uint4(0, 0, 0, 0);
+    };
+    uint4 dv4[D / 8];
+    if (cur.valid()) load_dout(cur, dv4);
     for (; cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       const int tok = cur.t * kTileTokens + row;
       const bool valid_tok = tok < p.T;
-      // dout row of this token (zero past the frame's end)
-      uint4 dv4[D / 8];
-      {
-        const uint16_t* src =
-            p.dout + ((static_cast<int64_t>(b) * p.F + f) * p.T + (valid_tok ? tok : 0)) *
-                         static_cast<int64_t>(p.H) * D +
-                     static_cast<int64_t>(h) * D;
-#pragma unroll
-        for (int x = 0; x < D / 8; ++x)
-          dv4[x] = valid_tok ? __ldg(reinterpret_cast<const uint4*>(src) + x) : make_uint4(0, 0, 0, 0);
-      }
       // ---- Epi1: D = [dout / den | -(dout . num) / den^2]
       if (!warp_wait(acc1_full, ph, abort, kCode)) break;
       if (!warp_wait(dfree, ph ^ 1u, abort, kCode)) break;  // previous tile's MMA2/MMA3 done
@@ -397,6 +403,11 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) {
         mbar_arrive(acc1_free);
         mbar_arrive(dfull);
+      }
+      {
+        TileCursor nxt = cur;
+        nxt.advance();
+        if (nxt.valid()) load_dout(nxt, dv4);
       }
       // ---- Epi2: dq = 1[q > 0] * dq~
       if (!warp_wait(acc2_full, ph, abort, kCode)) break;

@@ -19,8 +19,9 @@
 // normaliser column, the four ReLU warps' sums added in a fixed order) to the
 // plan's slot.  The scan kernel sums a unit's partials.
 //
-// Warp roles (320 threads): warps 0-3 drain TMEM (epilogue), warps 4-7 apply
-// ReLU, warp 8 issues TMA, warp 9 issues MMAs.
+// Warp roles: warps 0-3 drain TMEM (epilogue), the next kReluWarps (4; 8 in
+// the rotary variant, which has more to do per element) apply ReLU, then one
+// warp issues TMA and one issues MMAs.
 #pragma once
 
 #include "gla_common.cuh"
@@ -29,7 +30,7 @@
 
 namespace gla {
 
-template <int D>
+template <int D, bool kRope = false>
 struct IncCfg {
   using G = Geo<D>;
   static constexpr int kStages = (D == 128) ? 3 : 4;
@@ -40,9 +41,10 @@ struct IncCfg {
   static constexpr int kTmemCols = 2 * D;                       // two fp32 accumulators of N = D
   static constexpr int kPartialRows = D + 1;
   static constexpr int kPartialFloats = kPartialRows * D;
-  static constexpr int kThreads = 320;
+  static constexpr int kReluWarps = kRope ? 8 : 4;
+  static constexpr int kThreads = (kReluWarps + 6) * 32;        // + epilogue, TMA, MMA warps
   static constexpr int kBarBytes = (3 * kStages + 7) * 8;
-  static constexpr int kZBytes = 4 * D * 4;  // per-ReLU-warp normaliser sums
+  static constexpr int kZBytes = kReluWarps * D * 4;  // per-ReLU-warp normaliser sums
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kZBytes + kBarBytes + 16;
 };
 
@@ -76,11 +78,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // memory after its normaliser sums are taken, so the contraction forms
 // (R phi(K))^T V while row d keeps sum phi(k).
 template <int D, bool kRope = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(IncCfg<D, kRope>::kThreads, 1)
     gla_increment_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const IncParams p) {
   using G = Geo<D>;
-  using C = IncCfg<D>;
+  using C = IncCfg<D, kRope>;
+  constexpr int RW = C::kReluWarps;
+  constexpr int kTmaWarp = 4 + RW, kMmaWarp = 5 + RW;
   constexpr int S = C::kStages;
   constexpr unsigned kCode = 1u;
 
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* zpart = reinterpret_cast<float*>(smem + S * C::kStageBytes);  // [4][D]
+  float* zpart = reinterpret_cast<float*>(smem + S * C::kStageBytes);  // [RW][D]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kZBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(320, 1)
   auto accf = [&](int a) { return bar0 + 8u * (3 * S + a); };
   auto acce = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (3 * S + 4);
-  const uint32_t zfull = bar0 + 8u * (3 * S + 5);  // 4 ReLU warps wrote zpart
+  const uint32_t zfull = bar0 + 8u * (3 * S + 5);  // the ReLU warps wrote zpart
   const uint32_t zfree = bar0 + 8u * (3 * S + 6);  // warp 4 consumed zpart
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 7);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(relu_done(s), 4);
+      mbar_init(relu_done(s), RW);
       mbar_init(empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -120,7 +124,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(acce(a), 4);
     }
     mbar_init(done_bar, 1);
-    mbar_init(zfull, 4);
+    mbar_init(zfull, RW);
     mbar_init(zfree, 1);
     *abort = 0;
     fence_mbar_init();
@@ -143,7 +147,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_k);
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
         mbar_wait_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
@@ -203,7 +207,8 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------- ReLU + normaliser sums
     constexpr int CPR = G::kChunksPerRow;     // 16-byte chunks per token row
-    constexpr int RPP = kTileTokens / CPR;    // rows covered per pass of 128 threads
+    constexpr int RPP = RW * 32 / CPR;        // rows covered per pass of the ReLU warps
+    constexpr int kPasses = kTileTokens / RPP;
     constexpr int CPA = G::kAtomElems / 8;    // chunks per swizzle row
     const int rt = threadIdx.x - 128;
     const int c = rt % CPR;
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(320, 1)
         rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
       }
 #pragma unroll
-      for (int m = 0; m < CPR; ++m) {
+      for (int m = 0; m < kPasses; ++m) {
         const uint32_t addr = base + m * RPP * G::kRowBytes;
         uint4 w = ld_shared_v4(addr);
         relu8(w);
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(320, 1)
       if (cur.last) {
         // Unit range ends: the column sums of phi(K) become row d of the
         // partial.  Each warp reduces its lanes, parks its sums in zpart[warp];
-        // warp 4 adds the four in a fixed order and writes the row.
+        // warp 4 adds the RW of them in a fixed order and writes the row.
 #pragma unroll
         for (int o = CPR; o < 32; o <<= 1)
 #pragma unroll
@@ -274,8 +279,12 @@ __global__ void __launch_bounds__(320, 1)
           if (!warp_wait(zfull, zround & 1u, abort, kCode)) break;
           float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) +
                        static_cast<int64_t>(D) * D;
-          for (int col = lane; col < D; col += 32)
-            dst[col] = ((zpart[col] + zpart[D + col]) + zpart[2 * D + col]) + zpart[3 * D + col];
+          for (int col = lane; col < D; col += 32) {
+            float zs = zpart[col];
+#pragma unroll
+            for (int w = 1; w < RW; ++w) zs += zpart[w * D + col];
+            dst[col] = zs;
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(zfree);
         }

@@ -16,7 +16,8 @@
 // tensor stores (one 32-row box per epilogue warp; rows past the frame's end
 // are clipped by the tensor bounds).
 //
-// Warp roles (320 threads): warps 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
+// Warp roles: warps 0-3 epilogue, the next kReluWarps ReLU (4; 8 in the
+// rotary variant), then one TMA and one MMA warp.
 #pragma once
 
 #include "gla_common.cuh"
@@ -33,7 +34,8 @@ struct OutCfg {
   static constexpr int kSBufBytes = G::kAtoms * G::kNPad * G::kRowBytes;  // padded S image
   static constexpr int kStageOutBytes = G::kAtomTileBytes;               // one staging buffer
   static constexpr int kTmemCols = (2 * G::kNPad <= 128) ? 128 : (2 * G::kNPad <= 256) ? 256 : 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kReluWarps = kRope ? 8 : 4;
+  static constexpr int kThreads = (kReluWarps + 6) * 32;
   static constexpr int kDenRing = kRope ? 8 : 0;                          // per-tile normalisers
   static constexpr int kDenBytes = kDenRing * kTileTokens * 4;
   static constexpr int kBarCount = 3 * kStages + 9 + 2 * kDenRing;
@@ -57,12 +59,14 @@ struct OutParams {
 // scan's fp32 copy of S_f[:, d]; they pass it to the epilogue through a ring
 // of per-tile arrays in shared memory.
 template <int D, bool kRope = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
     gla_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_out, const OutParams p) {
   using G = Geo<D>;
   using C = OutCfg<D, kRope>;
   constexpr int R = C::kDenRing;
+  constexpr int RW = C::kReluWarps;
+  constexpr int kTmaWarp = 4 + RW, kMmaWarp = 5 + RW;
   constexpr int S = C::kStages;
   constexpr unsigned kCode = 2u;
 
@@ -101,7 +105,7 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(qfull(s), 1);
-      mbar_init(qrelu(s), 4);
+      mbar_init(qrelu(s), RW);
       mbar_init(qempty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(done_bar, 1);
     for (int m = 0; m < R; ++m) {
-      mbar_init(denfull(m), 4);
+      mbar_init(denfull(m), RW);
       mbar_init(denfree(m), 4);
     }
     *abort = 0;
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -185,7 +189,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int64_t sg = (seg > 2 ? seg - 2 : 0); sg < seg; ++sg)
         mbar_wait_drain(sfull(static_cast<int>(sg & 1)), static_cast<uint32_t>((sg >> 1) & 1));
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, G::kNPad, false, false);
@@ -226,7 +230,8 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ ReLU
     constexpr int CPR = G::kChunksPerRow;
-    constexpr int RPP = kTileTokens / CPR;
+    constexpr int RPP = RW * 32 / CPR;  // rows per pass of the ReLU warps
+    constexpr int kPasses = kTileTokens / RPP;
     constexpr int CPA = G::kAtomElems / 8;
     const int rt = threadIdx.x - 128;
     const int c = rt % CPR;
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t base = q_buf(s) + off0;
       if constexpr (!kRope) {
 #pragma unroll
-        for (int m = 0; m < CPR; ++m) {
+        for (int m = 0; m < kPasses; ++m) {
           const uint32_t addr = base + m * RPP * G::kRowBytes;
           uint4 w = ld_shared_v4(addr);
           relu8(w);
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(320, 1)
         rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
         float* den = den_ring + mr * kTileTokens;
 #pragma unroll
-        for (int m = 0; m < CPR; ++m) {
+        for (int m = 0; m < kPasses; ++m) {
           const uint32_t addr = base + m * RPP * G::kRowBytes;
           uint4 w = ld_shared_v4(addr);
           relu8(w);
