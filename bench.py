@@ -36,7 +36,8 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, make_grads, make_inputs, make_state, rope_dims  # noqa: E402
+from workloads import (WORKLOADS, gdn_workload, make_beta, make_grads, make_inputs,  # noqa: E402
+                       make_state, rope_dims)
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
@@ -370,6 +371,11 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     stream = torch.cuda.current_stream(dev)
     peaks = load_peaks()
 
+    rope = args.variant == "rope"
+    gdn = args.variant == "gdn"
+    if gdn:
+        w = gdn_workload(w)  # keys scaled by 1/sqrt(d T): the delta recurrence contracts
+        beta_l = make_beta(w, device=dev)
     # inputs: a ring of input sets (fresh frames for the streaming workload)
     nsets = 4 if w.name == "stream" else 1
     sets = [make_inputs(w, call=c, device=dev) for c in range(nsets)]
@@ -378,7 +384,6 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     out = torch.empty_like(sets[0][0])
     so = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev, dtype=torch.float32)
     work = algorithmic_work(w, state_in=state is not None)
-    rope = args.variant == "rope"
 
     def step(i, events=None):
         q, k, v, g = sets[i % nsets]
@@ -393,6 +398,12 @@ def run_gpu(args, w, dist, rank, local_rank, world):
                 gla.gla_forward_rope(*a, cfg, stream)
             else:
                 gla.gla_forward_rope_timed(*a, cfg, stream, events)
+        elif gdn:
+            ag = a[:4] + (beta_l,) + a[4:]
+            if events is None:
+                gla.gla_forward_gdn(*ag, stream)
+            else:
+                gla.gla_forward_gdn_timed(*ag, stream, events)
         elif events is None:
             gla.gla_forward(*a, stream)
         else:
@@ -464,24 +475,32 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     if not args.no_e2e:
         host_in = [x.cpu().pin_memory() for x in sets[0]]
         host_in.append(state_buf.cpu().pin_memory() if state_buf is not None else None)
+        host_in.append(beta_l.cpu().pin_memory() if gdn else None)
         dev_out = [out, so]
 
         def call(bi, bo):
-            q_, k_, v_, g_, s_ = bi
+            q_, k_, v_, g_, s_, b_ = bi
             a = (q_, k_, v_, g_, s_, bo[1], bo[0], w.B, w.H, w.frames, w.tokens_per_frame, w.d,
                  w.eps)
             if rope:
                 gla.gla_forward_rope(*a, gla.rope_config(w.grid_w, rope_dims(w.d)), stream)
+            elif gdn:
+                gla.gla_forward_gdn(*(a[:4] + (b_,) + a[4:]), stream)
             else:
                 gla.gla_forward(*a, stream)
 
         e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
                             max(2, min(K, args.e2e_steps)), w.total_tokens)
 
-    if rope:
+    if rope or gdn:
         roof["traffic"] = None  # the counters were taken on the plain kernels
+    metric = METRIC
+    if rope:
+        metric = METRIC.replace("attention", "attention + 3D RoPE", 1)
+    elif gdn:
+        metric = METRIC.replace("gated linear attention", "frame-wise gated delta rule", 1)
     res = {
-        "metric": METRIC if not rope else METRIC.replace("attention", "attention + 3D RoPE", 1),
+        "metric": metric,
         "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": warm, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -492,7 +511,8 @@ def run_gpu(args, w, dist, rank, local_rank, world):
                          % (work["bytes"] / 1e9),
                    "parallelism": "dp%d (independent sequences per GPU)" % world,
                    **({"rope": {"grid_w": w.grid_w, "dims": list(rope_dims(w.d)),
-                                "theta": 10000.0}} if rope else {})},
+                                "theta": 10000.0}} if rope else {}),
+                   **({"keys": "N(0,1)/sqrt(d T)", "beta_logits": "N(0,1)"} if gdn else {})},
         "roofline": roof, "layer_roofline": layer, "gpu_launches": (4 if rope else 3) * K,
         "e2e": e2e,
         "clocks": clocks.summary(), "device_fault": fault,
@@ -686,8 +706,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
                     help="time gla_forward (the layer metric) or gla_backward")
-    ap.add_argument("--variant", choices=["plain", "rope"], default="plain",
-                    help="forward only: the plain layer or gla_forward_rope (3D RoPE)")
+    ap.add_argument("--variant", choices=["plain", "rope", "gdn"], default="plain",
+                    help="forward only: the plain layer, gla_forward_rope (3D RoPE) or "
+                         "gla_forward_gdn (frame-wise gated delta rule)")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=0,
                     help="override the workload's frame count (small profiling cases)")

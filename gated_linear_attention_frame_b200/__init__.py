@@ -17,12 +17,15 @@ from ._binding import (  # noqa: F401
     RopeConfig,
     backward,
     forward,
+    forward_gdn,
     forward_rope,
     gla_backward,
     gla_backward_timed,
     gla_device_fault,
     gla_error_string,
     gla_forward,
+    gla_forward_gdn,
+    gla_forward_gdn_timed,
     gla_forward_noalloc,
     gla_forward_rope,
     gla_forward_rope_timed,

@@ -27,7 +27,8 @@ GLA_ERR_SCRATCH = 8
 GLA_ERR_ROPE = 9
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
-            "gla_forward_rope", "gla_forward_rope_timed", "gla_backward", "gla_backward_timed",
+            "gla_forward_rope", "gla_forward_rope_timed", "gla_forward_gdn", "gla_forward_gdn_timed",
+            "gla_backward", "gla_backward_timed",
             "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
 
 
@@ -73,6 +74,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward_timed.restype = i32
     lib.gla_forward_noalloc.argtypes = fwd
     lib.gla_forward_noalloc.restype = i32
+    gdn = fwd[:4] + [vp] + fwd[4:]
+    lib.gla_forward_gdn.argtypes = gdn
+    lib.gla_forward_gdn.restype = i32
+    lib.gla_forward_gdn_timed.argtypes = gdn + [ctypes.POINTER(vp)]
+    lib.gla_forward_gdn_timed.restype = i32
     rope_p = ctypes.POINTER(RopeConfig)
     lib.gla_forward_rope.argtypes = fwd[:13] + [rope_p, vp]
     lib.gla_forward_rope.restype = i32
@@ -177,6 +183,38 @@ def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, fr
                                  int(tokens_per_frame), int(d), float(eps), _stream(stream))
     if st != GLA_OK:
         raise GLAError(st, "gla_forward_noalloc")
+
+
+def gla_forward_gdn(q, k, v, gate_logits, beta_logits, state_in, state_out, out, B, H, frames,
+                    tokens_per_frame, d, eps, stream=None) -> None:
+    """The frame-wise gated delta-rule variant (see include/gla.h)."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    _check_dtypes(None, None, None, beta_logits, None, None, None)
+    lib = load_library()
+    st = lib.gla_forward_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(beta_logits),
+                             _ptr(state_in), _ptr(state_out), _ptr(out), int(B), int(H),
+                             int(frames), int(tokens_per_frame), int(d), float(eps),
+                             _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_gdn")
+
+
+def gla_forward_gdn_timed(q, k, v, gate_logits, beta_logits, state_in, state_out, out, B, H,
+                          frames, tokens_per_frame, d, eps, stream, events) -> None:
+    """gla_forward_gdn that records 4 CUDA events around the kernels."""
+    _check_dtypes(q, k, v, gate_logits, state_in, state_out, out)
+    lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+    st = lib.gla_forward_gdn_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
+                                   _ptr(beta_logits), _ptr(state_in), _ptr(state_out), _ptr(out),
+                                   int(B), int(H), int(frames), int(tokens_per_frame), int(d),
+                                   float(eps), _stream(stream),
+                                   ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_gdn_timed")
 
 
 def gla_forward_rope(q, k, v, gate_logits, state_in, state_out, out, B, H, frames,
@@ -305,6 +343,23 @@ def forward(q, k, v, gate_logits, state_in=None, eps: float = 1e-6, out=None, st
     if state_out is None:
         state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
     gla_forward(q, k, v, gate_logits, state_in, state_out, out, B, H, frames, T, d, eps, stream)
+    return out, state_out
+
+
+def forward_gdn(q, k, v, gate_logits, beta_logits, state_in=None, eps: float = 1e-6, out=None,
+                state_out=None, stream=None):
+    """Convenience wrapper of gla_forward_gdn; returns (out, state_out)."""
+    B, N, H, d = q.shape
+    frames = gate_logits.shape[1]
+    T = N // frames if frames else 0
+    if frames and N % frames:
+        raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None:
+        state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
+    gla_forward_gdn(q, k, v, gate_logits, beta_logits, state_in, state_out, out, B, H, frames, T,
+                    d, eps, stream)
     return out, state_out
 
 

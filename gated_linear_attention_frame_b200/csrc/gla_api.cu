@@ -14,6 +14,10 @@
 //                            bf16 G_f^T images
 //   5. gla_dgate_kernel      dg = a (1 - a) da
 //   6. gla_bwd_kv_kernel     dk, dv                                   (tcgen05)
+// gla_forward_gdn (the frame-wise delta-rule variant) enqueues
+//   1. gla_increment_kernel  dS_f and M_f = phi(K_f)^T phi(K_f) partials (tcgen05)
+//   2. gla_gdn_scan_kernel   S_f = a_f (S_{f-1} - beta_f M_f S_{f-1}) + beta_f dS_f
+//   3. gla_output_kernel     as gla_forward
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -27,6 +31,7 @@
 #include "gla_bwd_kv.cuh"
 #include "gla_bwd_q.cuh"
 #include "gla_common.cuh"
+#include "gla_gdn_scan.cuh"
 #include "gla_increment.cuh"
 #include "gla_output.cuh"
 #include "gla_rope.cuh"
@@ -105,6 +110,13 @@ cudaError_t set_smem_attrs() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::ScanCfg<D, 3>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, false, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::IncCfg<D, false, true>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla::gla_gdn_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::GdnScanCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -189,6 +201,7 @@ struct Args {
   float eps;
   cudaStream_t stream;
   const gla_rope_config* rope = nullptr;  // rotary variant when set
+  const float* beta = nullptr;            // delta-rule variant: [B, F, H] write-strength logits
 };
 
 // Host-only checks of a rotary configuration; no CUDA call.
@@ -368,13 +381,114 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   return status;
 }
 
+// The frame-wise delta-rule variant: increment + Gram partials, the delta
+// scan, the output kernel.
+template <int D>
+int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
+  using G = Geo<D>;
+  using GC = gla::GdnScanCfg<D>;
+  const int64_t units = static_cast<int64_t>(a.B) * a.F * a.H;
+  const int tpu = (a.T + gla::kTileTokens - 1) / gla::kTileTokens;
+  const int64_t W = units * tpu;
+  const int32_t G1 = static_cast<int32_t>(W < di.sms ? W : di.sms);
+  const gla::WorkPlan wp = W > 0 ? gla::WorkPlan::make(units, tpu, G1) : gla::WorkPlan{};
+  const int64_t slots = units + G1;
+  const int64_t partial_bytes =
+      W > 0 ? align256(slots * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4) : 0;
+  const int64_t mpartial_bytes = W > 0 ? align256(slots * static_cast<int64_t>(D) * D * 4) : 0;
+  const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
+  const int64_t ws_bytes = partial_bytes + mpartial_bytes + image_bytes;
+
+  // state columns per scan block: as many blocks per (b, h) as fill the SMs
+  // once, at least ceil((D + 1) / kMaxCols) and at most one per 8 columns
+  const int64_t bh = static_cast<int64_t>(a.B) * a.H;
+  const int min_groups = (D + 1 + GC::kMaxCols - 1) / GC::kMaxCols;
+  const int max_groups = (D + 1 + 7) / 8;
+  int64_t want = bh > 0 ? di.sms / bh : 1;
+  const int groups0 = static_cast<int>(want < min_groups ? min_groups
+                                                         : (want > max_groups ? max_groups : want));
+  const int cols = (D + 1 + groups0 - 1) / groups0;
+  const int groups = (D + 1 + cols - 1) / cols;
+
+  CUtensorMap tm_q, tm_k, tm_v, tm_out;
+  if (W > 0) {
+    int st;
+    if ((st = encode_map(&tm_q, a.q, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_k, a.k, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_v, a.v, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_out, a.out, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+  }
+  uint8_t* ws = nullptr;
+  if (ws_bytes > 0) {
+    cudaMemPool_t pool = workspace_pool();
+    if (pool == nullptr ||
+        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
+                                a.stream) != cudaSuccess) {
+      cudaGetLastError();
+      return GLA_ERR_ALLOC;
+    }
+  }
+  float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
+  float* mpartial = W > 0 ? reinterpret_cast<float*>(ws + partial_bytes) : nullptr;
+  uint8_t* image = W > 0 ? ws + partial_bytes + mpartial_bytes : nullptr;
+
+  int status = GLA_OK;
+  auto check = [&]() {
+    if (cudaGetLastError() != cudaSuccess) status = GLA_ERR_LAUNCH;
+  };
+  auto record = [&](int i) {
+    if (ev != nullptr && status == GLA_OK && cudaEventRecord(ev[i], a.stream) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+  };
+  record(0);
+  if (W > 0 && status == GLA_OK) {
+    gla::IncParams ip{partial, wp, a.H, a.F, a.T, gla::RopeGeo{}, mpartial};
+    using IC = gla::IncCfg<D, false, true>;
+    gla::gla_increment_kernel<D, false, true>
+        <<<G1, IC::kThreads, IC::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    check();
+  }
+  record(1);
+  if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
+    gla::GdnScanParams sp{partial, mpartial, a.g, a.beta, a.s_in, a.s_out, image, wp,
+                          a.H, a.F, tpu, groups, cols};
+    if (launch_dependent(gla::gla_gdn_scan_kernel<D>,
+                         static_cast<unsigned>(groups) * static_cast<unsigned>(bh), GC::kThreads,
+                         GC::kSmemBytes, a.stream, sp) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(2);
+  if (W > 0 && status == GLA_OK) {
+    gla::OutParams op{image, a.eps, wp, a.H, a.F, a.T};
+    if (launch_dependent(gla::gla_output_kernel<D>, G1, gla::OutCfg<D>::kThreads,
+                         gla::OutCfg<D>::kSmemBytes, a.stream, tm_q, tm_out, op) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
+    check();
+  }
+  record(3);
+  if (ws != nullptr && cudaFreeAsync(ws, a.stream) != cudaSuccess) {
+    cudaGetLastError();
+    if (status == GLA_OK) status = GLA_ERR_LAUNCH;
+  }
+  return status;
+}
+
 int forward_impl(const Args& a, cudaEvent_t* ev) {
   int st = validate(a);
   if (st != GLA_OK) return st;
   if (a.rope != nullptr && (st = validate_rope(a.rope, a.d)) != GLA_OK) return st;
+  if (a.beta != nullptr && !aligned(a.beta, 4)) return GLA_ERR_ALIGN;
   if (static_cast<int64_t>(a.B) * a.H == 0) return GLA_OK;  // nothing to compute or write
   DeviceInfo di;
   if ((st = device_setup(&di)) != GLA_OK) return st;
+  if (a.beta != nullptr) {
+    switch (a.d) {
+      case 32: return run_gdn<32>(a, di, ev);
+      case 64: return run_gdn<64>(a, di, ev);
+      default: return run_gdn<128>(a, di, ev);
+    }
+  }
   if (a.rope != nullptr) {
     switch (a.d) {
       case 32: return run<32, true>(a, di, ev);
@@ -478,9 +592,11 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   const int64_t da_bytes = align256(units * static_cast<int64_t>(RS::kGroups) * 8 * 4);
   const int64_t ws_bytes = partial_bytes + image_bytes + states_bytes + da_bytes;
 
-  CUtensorMap tm_q, tm_k, tm_v, tm_dq, tm_dk, tm_dv;
+  CUtensorMap tm_q, tm_k, tm_v, tm_dout, tm_dq, tm_dk, tm_dv;
   if (W > 0) {
     int st;
+    if ((st = encode_map(&tm_dout, a.dout, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK)
+      return st;
     if ((st = encode_map(&tm_q, a.q, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
     if ((st = encode_map(&tm_k, a.k, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
     if ((st = encode_map(&tm_v, a.v, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
@@ -537,10 +653,10 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(2);
   if (W > 0 && status == GLA_OK) {
-    gla::BwdQParams qp{image, static_cast<const uint16_t*>(a.dout), partial, a.eps, wp,
-                       a.H, a.F, a.T};
+    gla::BwdQParams qp{image, partial, a.eps, wp, a.H, a.F, a.T};
     if (launch_dependent(gla::gla_bwd_q_kernel<D>, G1, gla::BwdQCfg<D>::kThreads,
-                         gla::BwdQCfg<D>::kSmemBytes, a.stream, tm_q, tm_dq, qp) != cudaSuccess)
+                         gla::BwdQCfg<D>::kSmemBytes, a.stream, tm_q, tm_dout, tm_dq,
+                         qp) != cudaSuccess)
       status = GLA_ERR_LAUNCH;
     check();
   }
@@ -619,6 +735,31 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v, const float
 }
 
 size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int gla_forward_gdn(const void* q, const void* k, const void* v, const float* gate_logits,
+                    const float* beta_logits, const float* state_in, float* state_out, void* out,
+                    int B, int H, int frames, int tokens_per_frame, int d, float eps,
+                    cudaStream_t stream) {
+  if (static_cast<int64_t>(B) * frames * H > 0 && beta_logits == nullptr) return GLA_ERR_NULL;
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream, nullptr, beta_logits};
+  static const float kNone = 0.f;  // marks the variant when there are no units
+  if (a.beta == nullptr) a.beta = &kNone;
+  return forward_impl(a, nullptr);
+}
+
+int gla_forward_gdn_timed(const void* q, const void* k, const void* v, const float* gate_logits,
+                          const float* beta_logits, const float* state_in, float* state_out,
+                          void* out, int B, int H, int frames, int tokens_per_frame, int d,
+                          float eps, cudaStream_t stream, cudaEvent_t* events) {
+  if (events == nullptr) return GLA_ERR_NULL;
+  if (static_cast<int64_t>(B) * frames * H > 0 && beta_logits == nullptr) return GLA_ERR_NULL;
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream, nullptr, beta_logits};
+  static const float kNone = 0.f;
+  if (a.beta == nullptr) a.beta = &kNone;
+  return forward_impl(a, events);
+}
 
 int gla_forward_rope(const void* q, const void* k, const void* v, const float* gate_logits,
                      const float* state_in, float* state_out, void* out, int B, int H, int frames,

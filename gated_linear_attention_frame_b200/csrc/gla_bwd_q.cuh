@@ -10,8 +10,9 @@
 //   MMA2  dq~ = D S_f^T                A = D K-major (K = d+16), B = S_f^T image MN-major
 //   MMA3  L_f += phi(Q)^T D            A = phi(Q) MN-major, B = D MN-major
 // where D = [dnum | dden | 0 ...] is built in shared memory, in bf16, by the
-// epilogue from MMA1's result and dout (read by the epilogue threads directly
-// from global memory, one token row per thread).  D's first d columns sit in
+// epilogue from MMA1's result and dout: the producer loads the dout tile by
+// TMA into the D_hi buffer itself (same swizzled 128 x d layout), and each
+// epilogue thread overwrites its token row of dout with dnum in place.  D's first d columns sit in
 // two 128-byte-swizzled atoms; the dden column and 15 zero columns in a
 // 32-byte-swizzled region of 32-byte rows, so that every operand view of it
 // (MMA2's last K step, MMA3's N = 16 part) is a whole swizzle atom.  The same
@@ -51,7 +52,7 @@ struct BwdQCfg {
   static constexpr int kAcc3 = 288;  // L_f          : N = d + 16
   static constexpr int kTmemCols = 512;
   static constexpr int kThreads = 320;
-  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing;
+  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing + 1;
   static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + 2 * kDBytes +
                                     2 * kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 +
                                     16;
@@ -60,7 +61,6 @@ struct BwdQCfg {
 
 struct BwdQParams {
   const uint8_t* image;   // [units][kImageBytes] bf16 S_f^T images (forward recompute)
-  const uint16_t* dout;   // bf16 [B, F*T, H, d]
   float* partial;         // L_f partials [(units + G) slots][d + 1][d]
   float eps;
   WorkPlan wp;
@@ -70,6 +70,7 @@ struct BwdQParams {
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     gla_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_dout,
                      const __grid_constant__ CUtensorMap tm_dq, const BwdQParams p) {
   using G = Geo<D>;
   using C = BwdQCfg<D>;
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int R = C::kMaskRing;
   auto maskfull = [&](int m) { return bar0 + 8u * (3 * S + 11 + m); };
   auto maskfree = [&](int m) { return bar0 + 8u * (3 * S + 11 + R + m); };
+  const uint32_t doutfull = bar0 + 8u * (3 * S + 11 + 2 * R);  // dout tile landed in D_hi
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -133,6 +135,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(acc1_free, 4);
     mbar_init(dfull, 4);
     mbar_init(dfree, 1);
+    mbar_init(doutfull, 1);
     mbar_init(acc2_full, 1);
     mbar_init(acc2_free, 4);
     mbar_init(acc3_full, 1);
@@ -174,6 +177,7 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_dout);
       asm volatile("griddepcontrol.wait;" ::: "memory");  // S images of the forward recompute
       int64_t issued = 0, seg = 0;
       int b = 0, f = 0, h = 0;
@@ -197,9 +201,17 @@ __global__ void __launch_bounds__(320, 1)
         for (int a = 0; a < G::kAtoms; ++a)
           tma_load_5d(q_buf(s) + a * G::kAtomTileBytes, &tm_q, qfull(s), a * G::kAtomElems, h,
                       cur.t * kTileTokens, f, b);
+        // dout of this tile into D_hi once the previous tile's MMA2/MMA3 read it
+        if (!mbar_wait(dfree, static_cast<uint32_t>((issued & 1) ^ 1), abort, kCode)) break;
+        mbar_arrive_expect_tx(doutfull, G::kTileBytes);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a)
+          tma_load_5d(d_buf + a * G::kAtomTileBytes, &tm_dout, doutfull, a * G::kAtomElems, h,
+                      cur.t * kTileTokens, f, b);
       }
       for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
         mbar_wait_drain(qfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
+      if (issued > 0) mbar_wait_drain(doutfull, static_cast<uint32_t>((issued - 1) & 1));
       if (seg > 0) mbar_wait_drain(sfull, static_cast<uint32_t>((seg - 1) & 1));
     }
   } else if (warp == 9) {
@@ -333,23 +345,6 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     int64_t i = 0, seg = 0;
     int b = 0, f = 0, h = 0;
-    // dout row of this thread's token in a tile (zero past the frame's end);
-    // the next tile's row is loaded while the current tile's dq is written
-    auto load_dout = [&](const TileCursor& tc, uint4 (&dst)[D / 8]) {
-      int bb, ff, hh;
-      unit_coords(tc.u, p.H, p.F, bb, ff, hh);
-      const int tk = tc.t * kTileTokens + row;
-      const bool ok = tk < p.T;
-      const uint16_t* src =
-          p.dout + ((static_cast<int64_t>(bb) * p.F + ff) * p.T + (ok ? tk : 0)) *
-                       static_cast<int64_t>(p.H) * D +
-                   static_cast<int64_t>(hh) * D;
-#pragma unroll
-      for (int x = 0; x < D / 8; ++x)
-        dst[x] = ok ? __ldg(reinterpret_cast<const uint4*>(src) + x) : make_uint4(0, 0, 0, 0);
-    };
-    uint4 dv4[D / 8];
-    if (cur.valid()) load_dout(cur, dv4);
     for (; cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
@@ -357,7 +352,7 @@ __global__ void __launch_bounds__(320, 1)
       const bool valid_tok = tok < p.T;
       // ---- Epi1: D = [dout / den | -(dout . num) / den^2]
       if (!warp_wait(acc1_full, ph, abort, kCode)) break;
-      if (!warp_wait(dfree, ph ^ 1u, abort, kCode)) break;  // previous tile's MMA2/MMA3 done
+      if (!warp_wait(doutfull, ph, abort, kCode)) break;  // dout in D_hi (previous D read)
       tc_fence_after();
       const uint32_t t1 = tmem + lane_base + C::kAcc1;
       uint32_t dr;
@@ -372,10 +367,15 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
+          const int chunk = cc * 4 + ch;
+          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
+          const uint32_t off = a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16;
+          const uint4 dq4 = ld_shared_v4(d_buf + off);  // dout (zero past the frame's end)
+          const uint32_t dw[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
           uint32_t w[4], wl[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
-            const uint32_t wpair = (&dv4[0].x)[cc * 16 + ch * 4 + e2];
+            const uint32_t wpair = dw[e2];
             const float d0 = bf16lo_to_f32(wpair), d1 = bf16hi_to_f32(wpair);
             dot = fmaf(d0, __uint_as_float(r[8 * ch + 2 * e2]), dot);
             dot = fmaf(d1, __uint_as_float(r[8 * ch + 2 * e2 + 1]), dot);
@@ -383,9 +383,6 @@ __global__ void __launch_bounds__(320, 1)
             w[e2] = pack_bf16x2(x0, x1);
             wl[e2] = pack_bf16x2(x0 - bf16lo_to_f32(w[e2]), x1 - bf16hi_to_f32(w[e2]));
           }
-          const int chunk = cc * 4 + ch;
-          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
-          const uint32_t off = a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16;
           st_shared_v4(d_buf + off, make_uint4(w[0], w[1], w[2], w[3]));
           st_shared_v4(l_buf + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
         }
@@ -404,11 +401,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(acc1_free);
         mbar_arrive(dfull);
       }
-      {
-        TileCursor nxt = cur;
-        nxt.advance();
-        if (nxt.valid()) load_dout(nxt, dv4);
-      }
+
       // ---- Epi2: dq = 1[q > 0] * dq~
       if (!warp_wait(acc2_full, ph, abort, kCode)) break;
       const int mr = static_cast<int>(i % R);

@@ -1,0 +1,304 @@
+// gla_gdn_scan.cuh -- the frame-wise gated delta-rule scan.
+//
+// The SANA-WM pages describe frame-wise Gated DeltaNet: the recurrent state of
+// the linear attention gets decay gates and delta-rule corrections.  This
+// library reads it as (per (b, h), frames in order, a_f = sigmoid(g),
+// beta_f = sigmoid(beta logit), K~ = relu(K_f), M_f = K~^T K~, dS_f = K~^T [V_f | 1]):
+//   S_f = a_f S_{f-1} + beta_f K~^T ([V_f | 1] - a_f K~ S_{f-1})
+//       = a_f (S_{f-1} - beta_f M_f S_{f-1}) + beta_f dS_f
+// The frame's keys read what the decayed state holds for them and write back
+// only the difference.  Unlike the plain gated scan, the update couples the
+// d rows of S through M_f, but every state column j is still independent:
+//   S_f[:, j] = a_f (S_{f-1}[:, j] - beta_f M_f S_{f-1}[:, j]) + beta_f dS_f[:, j].
+// One block owns a group of columns of one (b, h) and loops over the frames:
+// a producer warp bulk-copies M_f (fp32, d x d, the increment kernel's Gram
+// partial) into a two-stage shared-memory ring; eight consumer warps each own
+// d/8 rows of S and every lane one or two of the group's columns, so a warp
+// reads each row k of M_f once (a broadcast) for all its columns and forms
+// M_f S_{f-1}[:, j] in fp32 from the previous state held in shared memory
+// (row-major [i][j], columns contiguous).  Each lane then adds the frame's
+// dS_f rows (read from global memory before the contraction, so the loads
+// overlap it), writes the next state to the other buffer and the bf16 S_f^T
+// image that the output kernel reads.  Further partials of a unit that the
+// tile schedule split over several increment CTAs are added from global
+// memory.  The warps pass a frame to each other through an mbarrier, so every
+// wait is bounded.
+#pragma once
+
+#include <type_traits>
+
+#include "gla_common.cuh"
+#include "gla_increment.cuh"
+#include "gla_scan.cuh"  // add8
+#include "sm100_ptx.cuh"
+
+namespace gla {
+
+struct GdnScanParams {
+  const float* partial;   // dS_f partials [slots][d + 1][d] (transposed, row d = normaliser)
+  const float* mpartial;  // M_f partials [slots][d][d]
+  const float* gate;      // [B, F, H] decay logits
+  const float* beta;      // [B, F, H] write-strength logits
+  const float* state_in;  // [B, H, d, d + 1] or nullptr
+  float* state_out;       // [B, H, d, d + 1] or nullptr
+  uint8_t* image;         // [units][kImageBytes] or nullptr
+  WorkPlan wp;
+  int H, F, tpu;
+  int groups;             // blocks per (b, h)
+  int cols;               // state columns per block (the last block may have fewer)
+};
+
+template <int D>
+struct GdnScanCfg {
+  static constexpr int kConsumerWarps = (D / 8 < 8) ? D / 8 : 8;  // each warp >= 8 rows
+  static constexpr int kConsumers = 32 * kConsumerWarps;
+  static constexpr int kThreads = kConsumers + 32;
+  static constexpr int kRowsPerWarp = D / kConsumerWarps;  // 16 at d = 128, else 8
+  static constexpr int kMaxCols = 44;                      // >= ceil((D + 1) / 3); <= 64
+  static_assert(3 * kMaxCols >= D + 1 && kMaxCols <= 64, "columns per block");
+  static constexpr int kColStride = kMaxCols;              // state tile row stride (floats)
+  static constexpr int kMBytes = D * D * 4;
+  static constexpr int kStageBytes = kMBytes + 16;
+  static constexpr int kStages = 2;
+  static constexpr int kTileBytes = D * kColStride * 4;    // one state buffer [D][cols]
+  static constexpr int kBarCount = 2 * kStages + 1;
+  static constexpr int kSmemBytes = 128 + kStages * kStageBytes + 2 * kTileBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+};
+
+struct GdnStageHeader {
+  int32_t c0, c1;  // the unit's partial slots u + c0 .. u + c1
+  float a, beta;
+};
+
+template <int D>
+__global__ void __launch_bounds__(GdnScanCfg<D>::kThreads, 1)
+    gla_gdn_scan_kernel(const GdnScanParams p) {
+  using G = Geo<D>;
+  using C = GdnScanCfg<D>;
+  constexpr int PF = IncCfg<D>::kPartialFloats;
+  constexpr int S = C::kStages;
+  constexpr int RPW = C::kRowsPerWarp;
+  constexpr int CS = C::kColStride;
+  constexpr unsigned kCode = 64u;
+  constexpr int kCW = C::kConsumerWarps;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~uintptr_t(127));
+  auto stage = [&](int s) { return smem + s * C::kStageBytes; };  // [M | hdr]
+  float* sbuf0 = reinterpret_cast<float*>(smem + S * C::kStageBytes);
+  float* sbuf1 = sbuf0 + D * CS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + 2 * C::kTileBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  const uint32_t fdone = bar0 + 8u * (2 * S);  // every consumer warp finished a frame
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + C::kBarCount);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / p.groups;
+  const int grp = blockIdx.x % p.groups;
+  const int j0 = grp * p.cols;
+  const int ncols = (D + 1 - j0 < p.cols) ? D + 1 - j0 : p.cols;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+  const int64_t u0 = static_cast<int64_t>(b) * p.F * p.H + h;
+  const int64_t srow = static_cast<int64_t>(bh) * D * (D + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), kCW);
+    }
+    mbar_init(fdone, kCW);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const bool stream = p.tpu > 0 && p.F > 0;
+  if (warp == kCW) {
+    // ---------------------------------------------------------------- producer
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the increment kernel
+    if (stream) {
+      float gl = 0.f, bl = 0.f;
+      int f = 0;
+      for (; f < p.F; ++f) {
+        if ((f & 31) == 0) {
+          const int ff = f + lane;
+          gl = ff < p.F ? __ldg(p.gate + u0 + static_cast<int64_t>(ff) * p.H) : 0.f;
+          bl = ff < p.F ? __ldg(p.beta + u0 + static_cast<int64_t>(ff) * p.H) : 0.f;
+        }
+        const float g = __shfl_sync(0xffffffffu, gl, f & 31);
+        const float bb = __shfl_sync(0xffffffffu, bl, f & 31);
+        int ok = 1;
+        if (lane == 0) {
+          const int s = f % S;
+          ok = mbar_wait(empty(s), static_cast<uint32_t>(((f / S) & 1) ^ 1), abort, kCode) ? 1 : 0;
+          if (ok) {
+            const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+            int32_t c0, c1;
+            p.wp.slot_range(u, c0, c1);
+            GdnStageHeader* hdr = reinterpret_cast<GdnStageHeader*>(stage(s) + C::kMBytes);
+            hdr->c0 = c0;
+            hdr->c1 = c1;
+            hdr->a = 1.0f / (1.0f + expf(-g));
+            hdr->beta = 1.0f / (1.0f + expf(-bb));
+            mbar_arrive_expect_tx(full(s), C::kMBytes);
+            bulk_load(smem_u32(stage(s)), p.mpartial + (u + c0) * static_cast<int64_t>(D) * D,
+                      C::kMBytes, full(s));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
+      if (lane == 0)
+        for (int k = (f > S ? f - S : 0); k < f; ++k)
+          mbar_wait_drain(full(k % S), static_cast<uint32_t>((k / S) & 1));
+    }
+  } else {
+    // --------------------------------------------------------------- consumers
+    float* sprev = sbuf0;
+    float* snext = sbuf1;
+    // state_in columns j0 .. j0+ncols-1 -> sprev[i][jl]
+    for (int idx = threadIdx.x; idx < D * ncols; idx += C::kConsumers) {
+      const int jl = idx % ncols, i = idx / ncols;
+      sprev[i * CS + jl] =
+          p.state_in != nullptr ? p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl]
+                                : 0.f;
+    }
+    named_bar_sync(1, C::kConsumers);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int CPA = G::kAtomElems / 8;
+    const int i0 = warp * RPW;             // this warp's rows
+    const bool has0 = lane < ncols;        // column lane
+    const bool has1 = lane + 32 < ncols;   // column lane + 32
+    for (int f = 0; f < p.F; ++f) {
+      const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+      float a, beta;
+      int32_t c0 = 0, c1 = 0;
+      const float* mst = nullptr;
+      if (stream) {
+        const int s = f % S;
+        if (!warp_wait(full(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
+        const GdnStageHeader hd = *reinterpret_cast<const GdnStageHeader*>(stage(s) + C::kMBytes);
+        a = hd.a;
+        beta = hd.beta;
+        c0 = hd.c0;
+        c1 = hd.c1;
+        mst = reinterpret_cast<const float*>(stage(s));
+      } else {
+        // frames without tokens: no write, the state only decays
+        a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));
+        beta = 0.f;
+      }
+      float acc0[RPW], acc1[RPW], ds0[RPW], ds1[RPW];
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) acc0[r] = acc1[r] = ds0[r] = ds1[r] = 0.f;
+      if (stream) {
+        // dS_f rows of this lane's columns, issued before the contraction
+        for (int cc = c0; cc <= c1; ++cc) {
+          const float* base = p.partial + (u + cc) * PF + i0;
+          if (has0) {
+            const float4* x = reinterpret_cast<const float4*>(base + static_cast<int64_t>(j0 + lane) * D);
+#pragma unroll
+            for (int r4 = 0; r4 < RPW / 4; ++r4) {
+              const float4 v4 = __ldg(x + r4);
+              ds0[4 * r4] += v4.x; ds0[4 * r4 + 1] += v4.y; ds0[4 * r4 + 2] += v4.z; ds0[4 * r4 + 3] += v4.w;
+            }
+          }
+          if (has1) {
+            const float4* x =
+                reinterpret_cast<const float4*>(base + static_cast<int64_t>(j0 + lane + 32) * D);
+#pragma unroll
+            for (int r4 = 0; r4 < RPW / 4; ++r4) {
+              const float4 v4 = __ldg(x + r4);
+              ds1[4 * r4] += v4.x; ds1[4 * r4 + 1] += v4.y; ds1[4 * r4 + 2] += v4.z; ds1[4 * r4 + 3] += v4.w;
+            }
+          }
+        }
+        // (M_f S_{f-1})[i0 .. i0+RPW-1, j]; M symmetric: row k of M is column k.
+        // The second column of each lane is only formed when the block has one.
+        auto contract = [&](const float* mrow, bool from_smem, auto two) {
+#pragma unroll 2
+          for (int k = 0; k < D; ++k) {
+            float m[RPW];
+            const float4* mk = reinterpret_cast<const float4*>(mrow + k * D + i0);
+#pragma unroll
+            for (int r4 = 0; r4 < RPW / 4; ++r4) {
+              const float4 v4 = from_smem ? mk[r4] : __ldg(mk + r4);
+              m[4 * r4] = v4.x; m[4 * r4 + 1] = v4.y; m[4 * r4 + 2] = v4.z; m[4 * r4 + 3] = v4.w;
+            }
+            const float s0 = has0 ? sprev[k * CS + lane] : 0.f;
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) acc0[r] = fmaf(m[r], s0, acc0[r]);
+            if constexpr (decltype(two)::value) {
+              const float s1 = has1 ? sprev[k * CS + lane + 32] : 0.f;
+#pragma unroll
+              for (int r = 0; r < RPW; ++r) acc1[r] = fmaf(m[r], s1, acc1[r]);
+            }
+          }
+        };
+        for (int cc = c0; cc <= c1; ++cc) {
+          const float* mrow = cc == c0 ? mst : p.mpartial + (u + cc) * static_cast<int64_t>(D) * D;
+          if (ncols > 32)
+            contract(mrow, cc == c0, std::true_type{});
+          else
+            contract(mrow, cc == c0, std::false_type{});
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(f % S));
+      }
+      // S_f = a (S_{f-1} - beta M S_{f-1}) + beta dS_f, this lane's columns
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const bool has = half == 0 ? has0 : has1;
+        if (!has) continue;
+        const int jl = lane + 32 * half;
+        float sn[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const float sp = sprev[(i0 + r) * CS + jl];
+          const float ac = half == 0 ? acc0[r] : acc1[r];
+          const float dd = half == 0 ? ds0[r] : ds1[r];
+          sn[r] = a * fmaf(-beta, ac, sp) + beta * dd;
+          snext[(i0 + r) * CS + jl] = sn[r];
+        }
+        if (p.image != nullptr) {
+          const int j = j0 + jl;
+#pragma unroll
+          for (int q8 = 0; q8 < RPW / 8; ++q8) {
+            const int ch = i0 / 8 + q8;  // 8-feature chunk of row j of S_f^T
+            uint4 w;
+            w.x = pack_bf16x2(sn[8 * q8 + 0], sn[8 * q8 + 1]);
+            w.y = pack_bf16x2(sn[8 * q8 + 2], sn[8 * q8 + 3]);
+            w.z = pack_bf16x2(sn[8 * q8 + 4], sn[8 * q8 + 5]);
+            w.w = pack_bf16x2(sn[8 * q8 + 6], sn[8 * q8 + 7]);
+            *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes +
+                                      (ch / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
+                                      G::swz(j, ch % CPA) * 16) = w;
+          }
+        }
+      }
+      // hand the frame over: every warp must have read sprev and written snext
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fdone);
+      if (!warp_wait(fdone, static_cast<uint32_t>(f & 1), abort, kCode)) break;
+      float* t = sprev;
+      sprev = snext;
+      snext = t;
+    }
+    if (p.state_out != nullptr) {
+      for (int idx = threadIdx.x; idx < D * ncols; idx += C::kConsumers) {
+        const int jl = idx % ncols, i = idx / ncols;
+        p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl] = sprev[i * CS + jl];
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace gla

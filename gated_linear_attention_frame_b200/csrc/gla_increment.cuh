@@ -30,7 +30,7 @@
 
 namespace gla {
 
-template <int D, bool kRope = false>
+template <int D, bool kRope = false, bool kGram = false>
 struct IncCfg {
   using G = Geo<D>;
   static constexpr int kStages = (D == 128) ? 3 : 4;
@@ -38,7 +38,9 @@ struct IncCfg {
   static constexpr int kABytes = kAAtoms * G::kAtomTileBytes;   // 32 KB
   static constexpr int kVBytes = G::kTileBytes;
   static constexpr int kStageBytes = kABytes + kVBytes;
-  static constexpr int kTmemCols = 2 * D;                       // two fp32 accumulators of N = D
+  // two buffers of [dS (N = D) | M (N = D, Gram variant)] fp32 accumulators
+  static constexpr int kAccCols = kGram ? 2 * D : D;
+  static constexpr int kTmemCols = 2 * kAccCols;
   static constexpr int kPartialRows = D + 1;
   static constexpr int kPartialFloats = kPartialRows * D;
   static constexpr int kReluWarps = kRope ? 8 : 4;
@@ -54,6 +56,8 @@ struct IncParams {
   int H, F;         // heads, frames
   int T;            // tokens per frame (rotary variant)
   RopeGeo rope;     // rotary variant only
+  float* mpartial;  // Gram variant: [(units + gridDim.x) slots][d][d] fp32 partials of
+                    // M_f = phi(K_f)^T phi(K_f), rows as the increment partials
 };
 
 // (b, f, h) of unit u = (b * F + f) * H + h.
@@ -77,12 +81,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // kRope: the rotary variant (gla_rope.cuh): phi(K) is rotated in shared
 // memory after its normaliser sums are taken, so the contraction forms
 // (R phi(K))^T V while row d keeps sum phi(k).
-template <int D, bool kRope = false>
-__global__ void __launch_bounds__(IncCfg<D, kRope>::kThreads, 1)
+// kGram: the delta-rule variant also forms M_f = phi(K_f)^T phi(K_f) from the
+// same shared-memory tile (B = phi(K) read MN-major like A), a second
+// accumulator beside dS_f, written as a second fp32 partial.
+template <int D, bool kRope = false, bool kGram = false>
+__global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
     gla_increment_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const IncParams p) {
   using G = Geo<D>;
-  using C = IncCfg<D, kRope>;
+  static_assert(!(kRope && kGram), "one variant at a time");
+  using C = IncCfg<D, kRope, kGram>;
+  constexpr int AC = C::kAccCols;
   constexpr int RW = C::kReluWarps;
   constexpr int kTmaWarp = 4 + RW, kMmaWarp = 5 + RW;
   constexpr int S = C::kStages;
@@ -193,7 +202,9 @@ __global__ void __launch_bounds__(IncCfg<D, kRope>::kThreads, 1)
                                         G::kGroupBytes, G::kLayout);
           const uint64_t bd = smem_desc(v_buf(s) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
                                         G::kGroupBytes, G::kLayout);
-          mma_bf16(tmem + ab * D, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+          mma_bf16(tmem + ab * AC, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+          if constexpr (kGram)  // M = phi(K)^T phi(K): B is the A tile itself (N = D)
+            mma_bf16(tmem + ab * AC + D, ad, ad, idesc, (first && kk == 0) ? 0u : 1u);
         }
         mma_commit(empty(s));
         if (last) {
@@ -308,10 +319,22 @@ __global__ void __launch_bounds__(IncCfg<D, kRope>::kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
-          tmem_ld_32cols(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * D + cc * 32, r);
+          tmem_ld_32cols(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * AC + cc * 32, r);
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+        }
+        if constexpr (kGram) {
+          float* mdst = p.mpartial + cur.slot() * static_cast<int64_t>(D) * D + row;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld_32cols(
+                tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * AC + D + cc * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) mdst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+          }
         }
       }
       tc_fence_before();

@@ -148,6 +148,39 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v,
 size_t gla_noalloc_scratch_bytes(void);
 
 /*
+ * gla_forward_gdn -- the frame-wise gated delta-rule variant (Gated DeltaNet).
+ *
+ * The SANA-WM pages (paper analysis: abstract, method components) describe
+ * the layer as frame-wise Gated DeltaNet: the SANA-Video linear attention
+ * whose recurrent state gets decay gates and delta-rule corrections, with
+ * keys scaled by 1/sqrt(D S).  No formula is printed; this library reads it
+ * as the layer above with the frame's write made a delta rule:
+ *   a_f = sigmoid(gate_logits[b, f, h]),  beta_f = sigmoid(beta_logits[b, f, h])
+ *   S_f = a_f S_{f-1} + beta_f phi(K_f)^T ([V_f | 1] - a_f phi(K_f) S_{f-1})
+ *   out_t = (phi(q_t) S_f[:, :d]) / (phi(q_t) S_f[:, d] + eps)
+ * (the frame's keys read what the decayed state holds for them and write the
+ * difference).  The key scale is the caller's: the recurrence contracts when
+ * beta_f ||phi(K_f)^T phi(K_f)|| < 2, e.g. k ~ N(0, 1/(d T)).
+ * Arguments as gla_forward plus beta_logits fp32 [B, frames, H] (4-byte
+ * aligned; must not be NULL when B * H * frames > 0).  Workspace: as
+ * gla_forward plus 4 d^2 bytes per (batch, frame, head) and per SM.
+ */
+int gla_forward_gdn(const void* q, const void* k, const void* v,
+                    const float* gate_logits, const float* beta_logits,
+                    const float* state_in, float* state_out,
+                    void* out,
+                    int B, int H, int frames, int tokens_per_frame, int d,
+                    float eps, cudaStream_t stream);
+
+/* gla_forward_gdn with four events recorded as in gla_forward_timed. */
+int gla_forward_gdn_timed(const void* q, const void* k, const void* v,
+                          const float* gate_logits, const float* beta_logits,
+                          const float* state_in, float* state_out,
+                          void* out,
+                          int B, int H, int frames, int tokens_per_frame, int d,
+                          float eps, cudaStream_t stream, cudaEvent_t* events);
+
+/*
  * Rotary position embedding of gla_forward_rope.  The SANA-Video ICLR 2026
  * talk (temporal modelling segment) adds a 3D RoPE to the linear attention
  * without a formula; this library reads it in the RoFormer form for linear
@@ -267,7 +300,8 @@ const char* gla_error_string(int status);
  * kernel gave up a bounded wait (about one second) and returned early; its
  * output is then invalid.  Bit 0: state-increment kernel, bit 1: output
  * kernel, bit 2: forward scan, bit 3: reverse scan, bit 4: key/value
- * gradient kernel, bit 5: query gradient kernel.  `code` is a host pointer.
+ * gradient kernel, bit 5: query gradient kernel, bit 6: delta-rule scan.
+ * `code` is a host pointer.
  * Returns GLA_OK or GLA_ERR_LAUNCH.
  */
 int gla_device_fault(cudaStream_t stream, unsigned int* code);

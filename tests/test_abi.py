@@ -142,6 +142,24 @@ def test_rope_validation_before_any_cuda_call(lib):
                                 ctypes.byref(gl.rope_config(80)), None) == gl.GLA_OK
 
 
+def test_gdn_validation_before_any_cuda_call(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    def call(beta=FAKE, d=128, B=1, **kw):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, out=FAKE)
+        p.update(kw)
+        return lib.gla_forward_gdn(p["q"], p["k"], p["v"], p["g"], beta, None, None, p["out"], B,
+                                   1, 1, 16, d, 1e-6, None)
+
+    assert call(beta=None) == gl.GLA_ERR_NULL
+    assert call(beta=FAKE + 2) == gl.GLA_ERR_ALIGN
+    assert call(d=48) == gl.GLA_ERR_UNSUPPORTED_D
+    assert call(g=None) == gl.GLA_ERR_NULL
+    assert call(B=0) == gl.GLA_OK
+    assert lib.gla_forward_gdn_timed(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 1, 16,
+                                     128, 1e-6, None, None) == gl.GLA_ERR_NULL
+
+
 def test_timed_variant_requires_events(lib):
     import gated_linear_attention_frame_b200 as gl
 

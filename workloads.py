@@ -26,8 +26,8 @@ from dataclasses import dataclass, replace
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "rope_dims",
-           "seed_for"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "make_beta",
+           "gdn_workload", "rope_dims", "seed_for"]
 
 BASE_SEED = 20261202
 
@@ -48,6 +48,8 @@ class Workload:
     calls: int = 1      # consecutive streaming calls (state carried)
     eps: float = 1e-6
     grid_w: int = 1     # latent grid width (token t of a frame sits at row t // grid_w)
+    k_div_tokens: bool = False  # k further divided by sqrt(tokens_per_frame) (delta-rule
+                                # variant: the pages' 1/sqrt(D S) key scale)
 
     @property
     def tokens(self) -> int:
@@ -114,6 +116,8 @@ def make_inputs(w: Workload, call: int = 0, device="cpu", seed: int | None = Non
     k = _normal(shape, gen, dev)
     if w.k_scaled:
         k.mul_(1.0 / math.sqrt(w.d))
+    if w.k_div_tokens and w.tokens_per_frame > 0:
+        k.mul_(1.0 / math.sqrt(w.tokens_per_frame))
     k = k.to(torch.bfloat16)
     v = _normal(shape, gen, dev).to(torch.bfloat16)
     g = _normal((w.B, w.frames, w.H), gen, dev).mul_(w.g_sigma).add_(w.g_mu)
@@ -145,3 +149,18 @@ def make_grads(w: Workload, device="cpu", seed: int | None = None, dstate_out: b
     if dstate_out:
         ds = _normal((w.B, w.H, w.d, w.d + 1), gen, dev).mul_(dstate_scale)
     return dout, ds
+
+
+def gdn_workload(w: Workload) -> Workload:
+    """The delta-rule variant of a workload: keys scaled by 1/sqrt(d T) (the
+    SANA-WM pages' 1/sqrt(D S), S = tokens per frame), same shapes and seeds."""
+    return w.with_(k_scaled=True, k_div_tokens=True)
+
+
+def make_beta(w: Workload, device="cpu", seed: int | None = None):
+    """Write-strength logits of the delta-rule variant: fp32 [B, frames, H]
+    ~ N(0, 1), from a generator seeded with seed_for(w) + 13 (or `seed`)."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed((seed_for(w) if seed is None else seed) + 13)
+    return _normal((w.B, w.frames, w.H), gen, dev)
