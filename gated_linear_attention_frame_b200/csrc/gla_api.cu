@@ -289,7 +289,12 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
     rg.frame_offset = a.rope->frame_offset;
     rg.sec_y = static_cast<int64_t>(a.F) * (rg.dt / 2);
     rg.sec_x = rg.sec_y + static_cast<int64_t>(rg.rows) * (rg.dy / 2);
-    table_pairs = rg.sec_x + static_cast<int64_t>(rg.cols) * (rg.dx / 2);
+    rg.sec_inc = rg.sec_x + static_cast<int64_t>(rg.cols) * (rg.dx / 2);
+    table_pairs = rg.sec_inc + D;  // two increments per pair
+    // token rows between consecutive rows of one ReLU thread (both kernels)
+    static_assert(gla::IncCfg<D, true>::kReluWarps == gla::OutCfg<D, true>::kReluWarps,
+                  "one row stride for the rotary kernels");
+    rg.rpp = gla::IncCfg<D, true>::kReluWarps * 32 / Geo<D>::kChunksPerRow;
   }
   const int64_t table_bytes = align256(table_pairs * 8);
   const int64_t zvec_bytes = (kRope && W > 0) ? align256(units * static_cast<int64_t>(D) * 4) : 0;
@@ -446,6 +451,22 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
     using IC = gla::IncCfg<D, false, true>;
     gla::gla_increment_kernel<D, false, true>
         <<<G1, IC::kThreads, IC::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    check();
+  }
+  // the tail units' Gram partials -> one per unit
+  const int32_t tail_units = W > 0 ? wp.units - wp.full_units() : 0;
+  if (tail_units > 0 && status == GLA_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tail_units), 4);
+    cfg.blockDim = dim3(256);
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gla::gla_gram_reduce_kernel<D>, mpartial, wp) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
     check();
   }
   record(1);

@@ -20,7 +20,9 @@
 // dS_f rows (read from global memory before the contraction, so the loads
 // overlap it), writes the next state to the other buffer and the bf16 S_f^T
 // image that the output kernel reads.  Further partials of a unit that the
-// tile schedule split over several increment CTAs are added from global
+// tile schedule split over several increment CTAs: gla_gram_reduce_kernel
+// first adds their Gram partials into the unit's first slot (the scan then
+// reads one M_f per frame); their dS rows are summed by the scan from global
 // memory.  The warps pass a frame to each other through an mbarrier, so every
 // wait is bounded.
 #pragma once
@@ -240,13 +242,11 @@ __global__ void __launch_bounds__(GdnScanCfg<D>::kThreads, 1)
             }
           }
         };
-        for (int cc = c0; cc <= c1; ++cc) {
-          const float* mrow = cc == c0 ? mst : p.mpartial + (u + cc) * static_cast<int64_t>(D) * D;
-          if (ncols > 32)
-            contract(mrow, cc == c0, std::true_type{});
-          else
-            contract(mrow, cc == c0, std::false_type{});
-        }
+        // the unit's Gram partials were added into slot c0 beforehand
+        if (ncols > 32)
+          contract(mst, true, std::true_type{});
+        else
+          contract(mst, true, std::false_type{});
         __syncwarp();
         if (lane == 0) mbar_arrive(empty(f % S));
       }
@@ -297,6 +297,37 @@ __global__ void __launch_bounds__(GdnScanCfg<D>::kThreads, 1)
     }
   }
   __syncwarp();
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// For the units that the tile schedule split over several increment CTAs
+// (the tail units), add the Gram partials of slots u + c0 + 1 .. u + c1 into
+// slot u + c0, so that the scan streams one M_f per frame.  Grid: (tail units,
+// column blocks); a fixed summation order.  Launched as a programmatic
+// dependent of the increment kernel; the scan depends on it in turn.
+template <int D>
+__global__ void __launch_bounds__(256) gla_gram_reduce_kernel(float* mpartial, WorkPlan wp) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t u = static_cast<int64_t>(wp.full_units()) + blockIdx.x;
+  int32_t c0, c1;
+  wp.slot_range(u, c0, c1);
+  if (c1 > c0) {
+    float4* dst = reinterpret_cast<float4*>(mpartial + (u + c0) * static_cast<int64_t>(D) * D);
+    for (int x = blockIdx.y * blockDim.x + threadIdx.x; x < D * D / 4;
+         x += gridDim.y * blockDim.x) {
+      float4 acc = dst[x];
+      for (int cc = c0 + 1; cc <= c1; ++cc) {
+        const float4 v =
+            reinterpret_cast<const float4*>(mpartial + (u + cc) * static_cast<int64_t>(D) * D)[x];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      dst[x] = acc;
+    }
+  }
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

@@ -232,8 +232,12 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
     int64_t i = 0;
     uint32_t zround = 0;
     RopeChunk rc{};
+    RopeStep st{};
     int frame = 0;
-    if constexpr (kRope) rc = rope_chunk(p.rope, c);
+    if constexpr (kRope) {
+      rc = rope_chunk(p.rope, c);
+      rope_step_init(p.rope, c, D / 2, st);
+    }
     for (; cur.valid(); cur.advance(), ++i) {
       const int s = static_cast<int>(i % S);
       if (!warp_wait(full(s), static_cast<uint32_t>((i / S) & 1), abort, kCode)) break;
@@ -242,6 +246,7 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
       if constexpr (kRope) {
         if (cur.first) frame = static_cast<int>((cur.u / p.H) % p.F);
         rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
+        rope_coeffs(p.rope, rc, frame, rp, p.T, st.cs01, st.cs23);  // first row of the tile
       }
 #pragma unroll
       for (int m = 0; m < kPasses; ++m) {
@@ -250,10 +255,9 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
         relu8(w);
         if constexpr (kRope) {
           uint4 wr = w;
-          float4 cs01, cs23;
-          rope_coeffs(p.rope, rc, frame, rp, p.T, cs01, cs23);
-          rotate8(wr, cs01, cs23);
+          rotate8(wr, st.cs01, st.cs23);
           st_shared_v4(addr, wr);
+          rope_step_next(st, rp, p.rope.grid_w);
           rp.next(RPP, p.rope.grid_w);
         } else {
           st_shared_v4(addr, w);

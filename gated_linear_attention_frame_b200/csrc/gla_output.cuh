@@ -239,12 +239,14 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
     const uint32_t off0 =
         (c / CPA) * G::kAtomTileBytes + r0 * G::kRowBytes + G::swz(r0, c % CPA) * 16;
     RopeChunk rc{};
+    RopeStep st{};
     int frame = 0;
     float zc[8];  // rotary: S_f[8c .. 8c+7, d] of the current unit
 #pragma unroll
     for (int e = 0; e < 8; ++e) zc[e] = 0.f;
     if constexpr (kRope) {
       rc = rope_chunk(p.rope, c);
+      rope_step_init(p.rope, c, D / 2, st);
       asm volatile("griddepcontrol.wait;" ::: "memory");  // zvec comes from the scan kernel
     }
     int64_t i = 0;
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
         }
         RopeRowPos rp;
         rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
+        rope_coeffs(p.rope, rc, frame, rp, p.T, st.cs01, st.cs23);  // first row of the tile
         float* den = den_ring + mr * kTileTokens;
 #pragma unroll
         for (int m = 0; m < kPasses; ++m) {
@@ -292,10 +295,9 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
 #pragma unroll
           for (int o = CPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
           if (c == 0) den[r0 + m * RPP] = part;
-          float4 cs01, cs23;
-          rope_coeffs(p.rope, rc, frame, rp, p.T, cs01, cs23);
-          rotate8(w, cs01, cs23);
+          rotate8(w, st.cs01, st.cs23);
           st_shared_v4(addr, w);
+          rope_step_next(st, rp, p.rope.grid_w);
           rp.next(RPP, p.rope.grid_w);
         }
         __syncwarp();

@@ -10,12 +10,20 @@
 //   the normaliser keeps the un-rotated phi(q_t) . sum phi(k).
 //
 // Since every block is a multiple of 8 features, each 16-byte chunk of a
-// token row (8 bf16, 4 pairs) belongs to one block: a thread that owns chunk
-// c of its rows reads 4 (cos, sin) pairs per row from a small fp32 table:
+// token row (8 bf16, 4 pairs) belongs to one block.  A thread owns chunk c of
+// the rows r0, r0 + P, r0 + 2P, ... of a tile (P = rows per pass of the ReLU
+// warps).  It reads the (cos, sin) of its 4 pairs for its first row from a
+// small fp32 table and steps to the next rows by angle addition: from one row
+// to the next the column advances by P mod grid_w or by that minus grid_w
+// (wrapping to the next latent row), and the row index by floor(P / grid_w)
+// or one more; the (cos, sin) of both increments of every pair are in the
+// table too.  Table (built once per call by gla_rope_table_kernel in fp64,
+// rounded to fp32):
 //   section t: [frames][d_t / 2]   (positions frame_offset .. frame_offset + F - 1)
 //   section y: [rows][d_y / 2]     (rows = ceil(T / grid_w))
 //   section x: [cols][d_x / 2]     (cols = min(T, grid_w))
-// built once per call by gla_rope_table_kernel in fp64 and rounded to fp32.
+//   section inc: [2][d / 2]        (per pair: the no-wrap and the wrap increment;
+//                                   (1, 0) for the temporal block)
 #pragma once
 
 #include <cstdint>
@@ -32,6 +40,8 @@ struct RopeGeo {
   int frames;           // positions of the temporal section
   int frame_offset;
   int64_t sec_y, sec_x; // start of the height / width sections, in (cos, sin) pairs
+  int64_t sec_inc;      // start of the increment section
+  int rpp;              // token rows between a thread's consecutive rows
 };
 
 // The block of chunk c (features 8c .. 8c+7) and where its pairs sit.
@@ -94,17 +104,75 @@ __device__ __forceinline__ void rope_coeffs(const RopeGeo& g, const RopeChunk& r
   cs23 = __ldg(g.table + idx + 1);
 }
 
+// (cos, sin) of a thread's 4 pairs on its current row, and the two
+// increments that lead to its next row.
+struct RopeStep {
+  float4 cs01, cs23;  // current row
+  float4 ia01, ia23;  // next row on the same latent row (no wrap)
+  float4 ib01, ib23;  // next row after a wrap
+  int step_mod;       // rpp mod grid_w
+};
+
+// Once per thread: the increments of chunk c (pairs 4c .. 4c+3).
+__device__ __forceinline__ void rope_step_init(const RopeGeo& g, int c, int half_d, RopeStep& st) {
+  const int64_t ia = (g.sec_inc + 4 * c) >> 1;
+  const int64_t ib = (g.sec_inc + half_d + 4 * c) >> 1;
+  st.ia01 = __ldg(g.table + ia);
+  st.ia23 = __ldg(g.table + ia + 1);
+  st.ib01 = __ldg(g.table + ib);
+  st.ib23 = __ldg(g.table + ib + 1);
+  st.step_mod = g.rpp % g.grid_w;
+}
+
+__device__ __forceinline__ float4 cmul2(const float4& a, const float4& b) {
+  return make_float4(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x, a.z * b.z - a.w * b.w,
+                     a.z * b.w + a.w * b.z);
+}
+
+// Move to the next row (rp still describes the current row).
+__device__ __forceinline__ void rope_step_next(RopeStep& st, const RopeRowPos& rp, int grid_w) {
+  const bool wrap = rp.x + st.step_mod >= grid_w;
+  st.cs01 = cmul2(st.cs01, wrap ? st.ib01 : st.ia01);
+  st.cs23 = cmul2(st.cs23, wrap ? st.ib23 : st.ia23);
+}
+
 // One thread per (cos, sin) entry of the three sections, in fp64.
 __global__ void __launch_bounds__(256) gla_rope_table_kernel(float2* table, RopeGeo g,
                                                              double log2_theta) {
   const int64_t nt = static_cast<int64_t>(g.frames) * (g.dt / 2);
   const int64_t ny = static_cast<int64_t>(g.rows) * (g.dy / 2);
   const int64_t nx = static_cast<int64_t>(g.cols) * (g.dx / 2);
-  const int64_t total = nt + ny + nx;
+  const int half_d = (g.dt + g.dy + g.dx) / 2;
+  const int64_t total = nt + ny + nx + 2 * half_d;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     int64_t k = i;
     int n, pos, j;
+    if (k >= nt + ny + nx) {
+      // increments: which = 0 (no wrap) or 1 (wrap), pair pp of the head dim
+      k -= nt + ny + nx;
+      const int which = static_cast<int>(k / half_d);
+      const int pp = static_cast<int>(k % half_d);
+      const int step_mod = g.rpp % g.grid_w, step_div = g.rpp / g.grid_w;
+      int delta = 0;
+      if (2 * pp < g.dt) {
+        n = g.dt;
+        j = pp;
+      } else if (2 * pp < g.dt + g.dy) {
+        n = g.dy;
+        j = pp - g.dt / 2;
+        delta = step_div + which;
+      } else {
+        n = g.dx;
+        j = pp - (g.dt + g.dy) / 2;
+        delta = which ? step_mod - g.grid_w : step_mod;
+      }
+      const double freq = exp2(-2.0 * j / n * log2_theta);
+      double s, c;
+      sincos(static_cast<double>(delta) * freq, &s, &c);
+      table[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
+      continue;
+    }
     if (k < nt) {
       n = g.dt;
       pos = g.frame_offset + static_cast<int>(k / (n / 2));
