@@ -494,6 +494,12 @@ def run_gpu(args, w, dist, rank, local_rank, world):
 
     if rope or gdn:
         roof["traffic"] = None  # the counters were taken on the plain kernels
+    # kernels per call: increment, scan, output; + the rotary table kernel; +
+    # the Gram reduction when the tile schedule has tail units (delta rule)
+    units = w.B * w.frames * w.H
+    ctas = min(units * -(-w.tokens_per_frame // 128),
+               torch.cuda.get_device_properties(dev).multi_processor_count)
+    launches_per_step = 3 + int(rope) + int(gdn and ctas > 0 and units % ctas != 0)
     metric = METRIC
     if rope:
         metric = METRIC.replace("attention", "attention + 3D RoPE", 1)
@@ -513,7 +519,8 @@ def run_gpu(args, w, dist, rank, local_rank, world):
                    **({"rope": {"grid_w": w.grid_w, "dims": list(rope_dims(w.d)),
                                 "theta": 10000.0}} if rope else {}),
                    **({"keys": "N(0,1)/sqrt(d T)", "beta_logits": "N(0,1)"} if gdn else {})},
-        "roofline": roof, "layer_roofline": layer, "gpu_launches": (4 if rope else 3) * K,
+        "roofline": roof, "layer_roofline": layer,
+        "gpu_launches": launches_per_step * K,
         "e2e": e2e,
         "clocks": clocks.summary(), "device_fault": fault,
         "gpu": torch.cuda.get_device_name(dev),
