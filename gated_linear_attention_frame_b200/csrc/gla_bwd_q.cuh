@@ -26,7 +26,9 @@
 // of D would put their error near the tolerance; dq uses D_hi alone.
 // The ReLU warps keep a byte mask of q > 0 for the dq epilogue, so a q stage
 // is released as soon as MMA3 has read it.
-// Warp roles: 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
+// Warp roles: 0-3 D builders (and the L_f partials), 4-7 ReLU, 8 TMA, 9 MMA,
+// 10-13 dq writers.  The dq writers take the dq epilogue off the path that
+// links one tile's D to the next.
 #pragma once
 
 #include "gla_common.cuh"
@@ -51,7 +53,7 @@ struct BwdQCfg {
   static constexpr int kAcc2 = 160;  // dq~          : N = d
   static constexpr int kAcc3 = 288;  // L_f          : N = d + 16
   static constexpr int kTmemCols = 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 448;
   static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing + 1;
   static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + 2 * kDBytes +
                                     2 * kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 +
@@ -68,7 +70,7 @@ struct BwdQParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     gla_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_dout,
                      const __grid_constant__ CUtensorMap tm_dq, const BwdQParams p) {
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(320, 1)
       mma_commit(done_bar);
       mbar_wait_drain(done_bar, 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------------ ReLU
     constexpr int CPR = G::kChunksPerRow;
     constexpr int RPP = kTileTokens / CPR;
@@ -338,16 +340,14 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(maskfull(mr));
       }
     }
-  } else {
-    // ------------------------------------------------------------- epilogue
+  } else if (warp < 4) {
+    // ------------------------------------------- D builders and L_f partials
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // token within the tile (= key feature for L_f)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     int64_t i = 0, seg = 0;
-    int b = 0, f = 0, h = 0;
     for (; cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
-      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       const int tok = cur.t * kTileTokens + row;
       const bool valid_tok = tok < p.T;
       // ---- Epi1: D = [dout / den | -(dout . num) / den^2]
@@ -356,15 +356,17 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const uint32_t t1 = tmem + lane_base + C::kAcc1;
       uint32_t dr;
+      uint32_t r[2][32];
       tmem_ld_1col(t1 + D, dr);
+      tmem_ld_32cols(t1, r[0]);
       tmem_wait_ld();
       const float rden = 1.0f / (__uint_as_float(dr) + p.eps);
-      float dot = 0.f;
+      float dot4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32cols(t1 + cc * 32, r);
-        tmem_wait_ld();
+        // the next 32 columns load while these are processed
+        if (cc + 1 < D / 32) tmem_ld_32cols(t1 + (cc + 1) * 32, r[(cc + 1) & 1]);
+        const uint32_t* rc = r[cc & 1];
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
           const int chunk = cc * 4 + ch;
@@ -377,8 +379,8 @@ __global__ void __launch_bounds__(320, 1)
           for (int e2 = 0; e2 < 4; ++e2) {
             const uint32_t wpair = dw[e2];
             const float d0 = bf16lo_to_f32(wpair), d1 = bf16hi_to_f32(wpair);
-            dot = fmaf(d0, __uint_as_float(r[8 * ch + 2 * e2]), dot);
-            dot = fmaf(d1, __uint_as_float(r[8 * ch + 2 * e2 + 1]), dot);
+            dot4[e2] = fmaf(d0, __uint_as_float(rc[8 * ch + 2 * e2]), dot4[e2]);
+            dot4[e2] = fmaf(d1, __uint_as_float(rc[8 * ch + 2 * e2 + 1]), dot4[e2]);
             const float x0 = d0 * rden, x1 = d1 * rden;
             w[e2] = pack_bf16x2(x0, x1);
             wl[e2] = pack_bf16x2(x0 - bf16lo_to_f32(w[e2]), x1 - bf16hi_to_f32(w[e2]));
@@ -386,8 +388,10 @@ __global__ void __launch_bounds__(320, 1)
           st_shared_v4(d_buf + off, make_uint4(w[0], w[1], w[2], w[3]));
           st_shared_v4(l_buf + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
         }
+        if (cc + 1 < D / 32) tmem_wait_ld();
       }
       tc_fence_before();
+      const float dot = (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
       const float dden = valid_tok ? -dot * rden * rden : 0.f;
       const uint32_t dden_hi = pack_bf16x2(dden, 0.f);
       const float dden_lo = dden - bf16lo_to_f32(dden_hi);
@@ -401,7 +405,40 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(acc1_free);
         mbar_arrive(dfull);
       }
-
+      // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
+      if (cur.last) {
+        if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        tc_fence_after();
+        float* dst = p.partial + cur.slot() * static_cast<int64_t>(PF) + row;
+        const uint32_t t3 = tmem + lane_base + C::kAcc3;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r3[32];
+          tmem_ld_32cols(t3 + cc * 32, r3);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r3[jj]);
+        }
+        uint32_t zr;
+        tmem_ld_1col(t3 + D, zr);
+        tmem_wait_ld();
+        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc3_free);
+        ++seg;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dq writers
+    const int q4 = warp & 3;          // TMEM lanes 32 q4 .. 32 q4 + 31
+    const int row = q4 * 32 + lane;   // token within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int64_t i = 0;
+    int b = 0, f = 0, h = 0;
+    for (; cur.valid(); cur.advance(), ++i) {
+      const uint32_t ph = static_cast<uint32_t>(i & 1);
+      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       // ---- Epi2: dq = 1[q > 0] * dq~
       if (!warp_wait(acc2_full, ph, abort, kCode)) break;
       const int mr = static_cast<int>(i % R);
@@ -453,29 +490,6 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc2_free);
-      // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
-      if (cur.last) {
-        if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
-        tc_fence_after();
-        float* dst = p.partial + cur.slot() * static_cast<int64_t>(PF) + row;
-        const uint32_t t3 = tmem + lane_base + C::kAcc3;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld_32cols(t3 + cc * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
-        }
-        uint32_t zr;
-        tmem_ld_1col(t3 + D, zr);
-        tmem_wait_ld();
-        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc3_free);
-        ++seg;
-      }
     }
     if (lane == 0) bulk_wait_group<0>();
   }
