@@ -118,6 +118,12 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(gla::gla_gdn_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::GdnScanCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
+  if constexpr (D == 128) {
+    e = cudaFuncSetAttribute(gla::gla_gdn_scan_tc_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gla::GdnTcCfg<128>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
   e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::IncCfg<D, true>::kSmemBytes);
@@ -407,7 +413,9 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   // state columns per scan block: as many blocks per (b, h) as fill the SMs
   // once, at least ceil((D + 1) / kMaxCols) and at most one per 8 columns
   const int64_t bh = static_cast<int64_t>(a.B) * a.H;
-  const int min_groups = (D + 1 + GC::kMaxCols - 1) / GC::kMaxCols;
+  // d = 128: the tensor-core scan (columns per block <= 48); else CUDA cores
+  constexpr int kMaxCols = (D == 128) ? 48 : GC::kMaxCols;
+  const int min_groups = (D + 1 + kMaxCols - 1) / kMaxCols;
   const int max_groups = (D + 1 + 7) / 8;
   int64_t want = bh > 0 ? di.sms / bh : 1;
   const int groups0 = static_cast<int>(want < min_groups ? min_groups
@@ -473,10 +481,15 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
     gla::GdnScanParams sp{partial, mpartial, a.g, a.beta, a.s_in, a.s_out, image, wp,
                           a.H, a.F, tpu, groups, cols};
-    if (launch_dependent(gla::gla_gdn_scan_kernel<D>,
-                         static_cast<unsigned>(groups) * static_cast<unsigned>(bh), GC::kThreads,
-                         GC::kSmemBytes, a.stream, sp) != cudaSuccess)
-      status = GLA_ERR_LAUNCH;
+    const unsigned grid = static_cast<unsigned>(groups) * static_cast<unsigned>(bh);
+    cudaError_t e;
+    if constexpr (D == 128)
+      e = launch_dependent(gla::gla_gdn_scan_tc_kernel<128>, grid, gla::GdnTcCfg<128>::kThreads,
+                           gla::GdnTcCfg<128>::kSmemBytes, a.stream, sp);
+    else
+      e = launch_dependent(gla::gla_gdn_scan_kernel<D>, grid, GC::kThreads, GC::kSmemBytes,
+                           a.stream, sp);
+    if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
   }
   record(2);

@@ -333,3 +333,279 @@ __global__ void __launch_bounds__(256) gla_gram_reduce_kernel(float* mpartial, W
 }
 
 }  // namespace gla
+
+namespace gla {
+
+// ---------------------------------------------------------------------------
+// Tensor-core delta scan (d = 128).  Same recurrence as gla_gdn_scan_kernel;
+// the per-frame product M_f S_{f-1}[:, J] of a block's column group J runs on
+// tcgen05 with a bf16 hi/lo split of both factors (Mh Sh + Mh Sl + Ml Sh into
+// an fp32 TMEM accumulator, the dropped Ml Sl term is ~2^-16 relative):
+//   A = M_f hi / lo   [M = 128 rows i, K = 128]  K-major, 128-byte swizzle
+//                     (built in shared memory from the fp32 Gram matrix)
+//   B = S_{f-1} hi / lo [N = group columns padded to 16, K = 128 rows k]
+//                     MN-major, 32-byte swizzle atoms of 16 columns
+// Thread i of the four consumer warps owns row i of the group's state (TMEM
+// lane i): it converts row i of M_f (M is symmetric, so the row is read as a
+// column, conflict-free), reads back row i of the product, updates its fp32
+// state row and writes the bf16 image and the next frame's B operand.  A
+// producer warp streams M_f; one thread issues the MMAs.
+template <int D>
+struct GdnTcCfg {
+  static_assert(D == 128, "tensor-core delta scan is built for d = 128");
+  static constexpr int kMaxCols = 48;              // three blocks cover d + 1 columns
+  static constexpr int kConsumers = 128;
+  static constexpr int kThreads = kConsumers + 64; // + producer warp + MMA warp
+  static constexpr int kMBytes = D * D * 4;        // fp32 Gram matrix
+  static constexpr int kAImgBytes = D * D * 2;     // one bf16 copy (hi or lo)
+  static constexpr int kBAtomBytes = D * 32;       // 16 columns x 128 rows
+  static constexpr int kBImgBytes = (kMaxCols / 16) * kBAtomBytes;
+  static constexpr int kSTileBytes = D * kMaxCols * 4;
+  static constexpr int kTmemCols = 64;
+  static constexpr int kBarCount = 6;
+  static constexpr int kSmemBytes = 1024 + kMBytes + 16 + 2 * kAImgBytes + 2 * kBImgBytes +
+                                    kSTileBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanParams p) {
+  using G = Geo<D>;
+  using C = GdnTcCfg<D>;
+  constexpr int PF = IncCfg<D>::kPartialFloats;
+  constexpr unsigned kCode = 64u;
+  constexpr int CPA = G::kAtomElems / 8;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t a_hi = sbase;                                  // 1024-aligned
+  const uint32_t a_lo = a_hi + C::kAImgBytes;
+  const uint32_t b_hi = a_lo + C::kAImgBytes;
+  const uint32_t b_lo = b_hi + C::kBImgBytes;
+  float* mst = reinterpret_cast<float*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes);
+  GdnStageHeader* hdr = reinterpret_cast<GdnStageHeader*>(
+      smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes + C::kMBytes);
+  float* stile = reinterpret_cast<float*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes +
+                                          C::kMBytes + 16);   // [row i][kMaxCols]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes +
+                                               C::kMBytes + 16 + C::kSTileBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t mfull = bar0;             // M_f landed (producer)
+  const uint32_t mempty = bar0 + 8;        // M_f converted (4 consumer warps)
+  const uint32_t opready = bar0 + 16;      // A and B operands of a frame written (4 warps)
+  const uint32_t accfull = bar0 + 24;      // product in TMEM (MMA commit)
+  const uint32_t done_bar = bar0 + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / p.groups;
+  const int grp = blockIdx.x % p.groups;
+  const int j0 = grp * p.cols;
+  const int ncols = (D + 1 - j0 < p.cols) ? D + 1 - j0 : p.cols;
+  const int np = (ncols + 15) & ~15;  // MMA N
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+  const int64_t u0 = static_cast<int64_t>(b) * p.F * p.H + h;
+  const int64_t srow = static_cast<int64_t>(bh) * D * (D + 1);
+  const bool stream = p.tpu > 0 && p.F > 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(mfull, 1);
+    mbar_init(mempty, 4);
+    mbar_init(opready, 4);
+    mbar_init(accfull, 1);
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  {
+    // zero the B operands (columns past the group's stay zero)
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int o = threadIdx.x * 16; o < 2 * C::kBImgBytes; o += C::kThreads * 16)
+      st_shared_v4(b_hi + o, z);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // Gram partials
+      int f = 0;
+      if (stream) {
+        for (; f < p.F; ++f) {
+          if (!mbar_wait(mempty, static_cast<uint32_t>((f & 1) ^ 1), abort, kCode)) break;
+          const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+          int32_t c0, c1;
+          p.wp.slot_range(u, c0, c1);
+          hdr->c0 = c0;
+          hdr->c1 = c1;
+          hdr->a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));
+          hdr->beta = 1.0f / (1.0f + expf(-__ldg(p.beta + u)));
+          mbar_arrive_expect_tx(mfull, C::kMBytes);
+          bulk_load(smem_u32(mst), p.mpartial + (u + c0) * static_cast<int64_t>(D) * D,
+                    C::kMBytes, mfull);
+        }
+        if (f > 0) mbar_wait_drain(mfull, static_cast<uint32_t>((f - 1) & 1));
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && stream) {
+      const uint32_t idesc = idesc_bf16_f32(128, np, false, true);
+      int f = 0;
+      for (; f < p.F; ++f) {
+        if (!mbar_wait(opready, static_cast<uint32_t>(f & 1), abort, kCode)) break;
+        tc_fence_after();
+        // Mh Sh + Mh Sl + Ml Sh over K = 128 (8 steps of 16)
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+          const uint32_t abase = pass == 2 ? a_lo : a_hi;
+          const uint32_t bbase = pass == 1 ? b_lo : b_hi;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int at = kk / 4, w = kk % 4;
+            const uint64_t ad = smem_desc(abase + at * (128 * G::kRowBytes) + w * 32, 16,
+                                          G::kGroupBytes, kLayoutSW128);
+            const uint64_t bd = smem_desc(bbase + kk * 512, C::kBAtomBytes, 256, kLayoutSW32);
+            mma_bf16(tmem, ad, bd, idesc, (pass > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(accfull);
+      }
+      mma_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else {
+    // --------------------------------------------------------------- consumers
+    const int i = threadIdx.x;  // state row / TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float* srow_s = stile + i * C::kMaxCols;
+    // B operand element (k = i, column jl): atom jl / 16, 32-byte row i,
+    // 16-byte chunk (jl % 16) / 8 swizzled with bit 2 of the row
+    auto b_off = [&](int jl) {
+      return (jl >> 4) * C::kBAtomBytes + i * 32 + ((((jl >> 3) & 1) ^ ((i >> 2) & 1)) << 4);
+    };
+    auto write_b = [&](const float* s) {  // all of the group's columns of row i
+      for (int jc = 0; jc < np; jc += 8) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = (jc + e < ncols) ? s[jc + e] : 0.f;
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          hw[e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
+          lw[e2] = pack_bf16x2(x[2 * e2] - bf16lo_to_f32(hw[e2]),
+                               x[2 * e2 + 1] - bf16hi_to_f32(hw[e2]));
+        }
+        st_shared_v4(b_hi + b_off(jc), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        st_shared_v4(b_lo + b_off(jc), make_uint4(lw[0], lw[1], lw[2], lw[3]));
+      }
+    };
+    // S_{-1}: row i of the group's columns
+    for (int jl = 0; jl < ncols; ++jl)
+      srow_s[jl] = p.state_in != nullptr
+                       ? p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl]
+                       : 0.f;
+    if (stream) write_b(srow_s);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int f = 0; f < p.F; ++f) {
+      const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+      float a, beta;
+      if (stream) {
+        if (!warp_wait(mfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
+        a = hdr->a;
+        beta = hdr->beta;
+        const int32_t c0 = hdr->c0, c1 = hdr->c1;
+        // A operands: row i of M_f (= column i, M symmetric), hi and lo
+#pragma unroll 2
+        for (int ch = 0; ch < D / 8; ++ch) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = mst[(ch * 8 + e) * D + i];
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            hw[e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
+            lw[e2] = pack_bf16x2(x[2 * e2] - bf16lo_to_f32(hw[e2]),
+                                 x[2 * e2 + 1] - bf16hi_to_f32(hw[e2]));
+          }
+          const uint32_t off = (ch / CPA) * (128 * G::kRowBytes) + i * G::kRowBytes +
+                               G::swz(i, ch % CPA) * 16;
+          st_shared_v4(a_hi + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+          st_shared_v4(a_lo + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(mempty);   // the producer may load the next frame's M
+          mbar_arrive(opready);  // A of this frame and B (written last frame) ready
+        }
+        // this frame's dS rows, loaded while the product runs
+        float ds[C::kMaxCols];
+#pragma unroll
+        for (int jl = 0; jl < C::kMaxCols; ++jl) ds[jl] = 0.f;
+        for (int cc = c0; cc <= c1; ++cc) {
+          const float* src = p.partial + (u + cc) * PF + static_cast<int64_t>(j0) * D + i;
+#pragma unroll
+          for (int jl = 0; jl < C::kMaxCols; ++jl)
+            if (jl < ncols) ds[jl] += __ldg(src + static_cast<int64_t>(jl) * D);
+        }
+        if (!warp_wait(accfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
+        tc_fence_after();
+        uint32_t r[2][32];
+        tmem_ld_32cols(tmem + lane_base, r[0]);
+        tmem_ld_32cols(tmem + lane_base + 32, r[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int jl = 0; jl < C::kMaxCols; ++jl) {
+          if (jl < ncols) {
+            const float acc = __uint_as_float(r[jl >> 5][jl & 31]);
+            srow_s[jl] = a * fmaf(-beta, acc, srow_s[jl]) + beta * ds[jl];
+          }
+        }
+      } else {
+        a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));  // no tokens: the state only decays
+        for (int jl = 0; jl < ncols; ++jl) srow_s[jl] *= a;
+      }
+      // bf16 image of S_f^T: row j = j0 + jl, element i
+      if (p.image != nullptr) {
+        uint16_t* img = reinterpret_cast<uint16_t*>(p.image + u * G::kImageBytes);
+        const int ci = i / 8;
+        for (int jl = 0; jl < ncols; ++jl) {
+          const int j = j0 + jl;
+          const int64_t off = (ci / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
+                              G::swz(j, ci % CPA) * 16 + (i % 8) * 2;
+          img[off / 2] = static_cast<uint16_t>(pack_bf16x2(srow_s[jl], 0.f) & 0xFFFFu);
+        }
+      }
+      if (stream && f + 1 < p.F) {
+        write_b(srow_s);  // next frame's B
+      }
+    }
+    if (p.state_out != nullptr)
+      for (int jl = 0; jl < ncols; ++jl)
+        p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl] = srow_s[jl];
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace gla

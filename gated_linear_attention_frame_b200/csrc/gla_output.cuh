@@ -36,8 +36,9 @@ struct OutCfg {
   static constexpr int kTmemCols = (2 * G::kNPad <= 128) ? 128 : (2 * G::kNPad <= 256) ? 256 : 512;
   static constexpr int kReluWarps = kRope ? 8 : 4;
   static constexpr int kThreads = (kReluWarps + 6) * 32;
-  static constexpr int kDenRing = kRope ? 8 : 0;                          // per-tile normalisers
-  static constexpr int kDenBytes = kDenRing * kTileTokens * 4;
+  // per-tile normaliser partial sums [token][16-byte chunk of the row]
+  static constexpr int kDenRing = kRope ? 2 : 0;
+  static constexpr int kDenBytes = kDenRing * kTileTokens * G::kChunksPerRow * 4;
   static constexpr int kBarCount = 3 * kStages + 9 + 2 * kDenRing;
   static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + 2 * kSBufBytes +
                                     2 * kStageOutBytes + kDenBytes + kBarCount * 8 + 16;
@@ -55,9 +56,10 @@ struct OutParams {
 
 // kRope: the rotary variant (gla_rope.cuh).  The ReLU warps rotate phi(Q) in
 // shared memory for the contraction (only its d value columns are used) and
-// form the un-rotated normaliser phi(q_t) . S_f[:, d] themselves, from the
-// scan's fp32 copy of S_f[:, d]; they pass it to the epilogue through a ring
-// of per-tile arrays in shared memory.
+// form the un-rotated normaliser phi(q_t) . S_f[:, d] from the scan's fp32
+// copy of S_f[:, d]: each thread stores the partial dot product of its 8
+// features of a token in a [token][chunk] array of a small ring, and the
+// epilogue thread of the token adds that row.
 template <int D, bool kRope = false>
 __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
     gla_output_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
         RopeRowPos rp;
         rp.start(cur.t * kTileTokens + r0, p.rope.grid_w);
         rope_coeffs(p.rope, rc, frame, rp, p.T, st.cs01, st.cs23);  // first row of the tile
-        float* den = den_ring + mr * kTileTokens;
+        float* den = den_ring + mr * kTileTokens * CPR;
 #pragma unroll
         for (int m = 0; m < kPasses; ++m) {
           const uint32_t addr = base + m * RPP * G::kRowBytes;
@@ -292,9 +294,7 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
           part = fmaf(bf16hi_to_f32(w.z), zc[5], part);
           part = fmaf(bf16lo_to_f32(w.w), zc[6], part);
           part = fmaf(bf16hi_to_f32(w.w), zc[7], part);
-#pragma unroll
-          for (int o = CPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-          if (c == 0) den[r0 + m * RPP] = part;
+          den[(r0 + m * RPP) * CPR + c] = part;
           rotate8(w, st.cs01, st.cs23);
           st_shared_v4(addr, w);
           rope_step_next(st, rp, p.rope.grid_w);
@@ -323,7 +323,20 @@ __global__ void __launch_bounds__(OutCfg<D, kRope>::kThreads, 1)
       if constexpr (kRope) {
         const int mr = static_cast<int>(i % R);
         if (!warp_wait(denfull(mr), static_cast<uint32_t>((i / R) & 1), abort, kCode)) break;
-        den = den_ring[mr * kTileTokens + row];
+        {
+          constexpr int CPR = G::kChunksPerRow;
+          const float4* dp = reinterpret_cast<const float4*>(den_ring + (mr * kTileTokens + row) * CPR);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int x = 0; x < CPR / 4; ++x) {
+            const float4 v = dp[x];
+            s4[0] += v.x;
+            s4[1] += v.y;
+            s4[2] += v.z;
+            s4[3] += v.w;
+          }
+          den = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(denfree(mr));
       } else {
