@@ -357,14 +357,14 @@ struct GdnTcCfg {
   static constexpr int kConsumers = 128;
   static constexpr int kThreads = kConsumers + 64; // + producer warp + MMA warp
   static constexpr int kMBytes = D * D * 4;        // fp32 Gram matrix
+  static constexpr int kStages = 2;                // M_{f+1} streams in during frame f
   static constexpr int kAImgBytes = D * D * 2;     // one bf16 copy (hi or lo)
   static constexpr int kBAtomBytes = D * 32;       // 16 columns x 128 rows
   static constexpr int kBImgBytes = (kMaxCols / 16) * kBAtomBytes;
-  static constexpr int kSTileBytes = D * kMaxCols * 4;
   static constexpr int kTmemCols = 64;
-  static constexpr int kBarCount = 6;
-  static constexpr int kSmemBytes = 1024 + kMBytes + 16 + 2 * kAImgBytes + 2 * kBImgBytes +
-                                    kSTileBytes + kBarCount * 8 + 16;
+  static constexpr int kBarCount = 2 * kStages + 3;
+  static constexpr int kSmemBytes = 1024 + 2 * kAImgBytes + 2 * kBImgBytes +
+                                    kStages * (kMBytes + 16) + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
 };
 
@@ -375,6 +375,8 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   constexpr int PF = IncCfg<D>::kPartialFloats;
   constexpr unsigned kCode = 64u;
   constexpr int CPA = G::kAtomElems / 8;
+  constexpr int S = C::kStages;
+  constexpr int MC = C::kMaxCols;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -384,19 +386,18 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   const uint32_t a_lo = a_hi + C::kAImgBytes;
   const uint32_t b_hi = a_lo + C::kAImgBytes;
   const uint32_t b_lo = b_hi + C::kBImgBytes;
-  float* mst = reinterpret_cast<float*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes);
-  GdnStageHeader* hdr = reinterpret_cast<GdnStageHeader*>(
-      smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes + C::kMBytes);
-  float* stile = reinterpret_cast<float*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes +
-                                          C::kMBytes + 16);   // [row i][kMaxCols]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes +
-                                               C::kMBytes + 16 + C::kSTileBytes);
+  uint8_t* mbase = smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes;
+  auto mst = [&](int s) { return reinterpret_cast<float*>(mbase + s * (C::kMBytes + 16)); };
+  auto hdr = [&](int s) {
+    return reinterpret_cast<GdnStageHeader*>(mbase + s * (C::kMBytes + 16) + C::kMBytes);
+  };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mbase + S * (C::kMBytes + 16));
   const uint32_t bar0 = smem_u32(bars);
-  const uint32_t mfull = bar0;             // M_f landed (producer)
-  const uint32_t mempty = bar0 + 8;        // M_f converted (4 consumer warps)
-  const uint32_t opready = bar0 + 16;      // A and B operands of a frame written (4 warps)
-  const uint32_t accfull = bar0 + 24;      // product in TMEM (MMA commit)
-  const uint32_t done_bar = bar0 + 32;
+  auto mfull = [&](int s) { return bar0 + 8u * s; };        // M_f landed (producer)
+  auto mempty = [&](int s) { return bar0 + 8u * (S + s); }; // M_f converted (4 warps)
+  const uint32_t opready = bar0 + 8u * (2 * S);     // A and B operands of a frame written
+  const uint32_t accfull = bar0 + 8u * (2 * S + 1); // product in TMEM (MMA commit)
+  const uint32_t done_bar = bar0 + 8u * (2 * S + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -414,8 +415,10 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   const bool stream = p.tpu > 0 && p.F > 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(mfull, 1);
-    mbar_init(mempty, 4);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(mfull(s), 1);
+      mbar_init(mempty(s), 4);
+    }
     mbar_init(opready, 4);
     mbar_init(accfull, 1);
     mbar_init(done_bar, 1);
@@ -439,25 +442,43 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // Gram partials
+    // The whole warp loads the gate and write-strength logits of 32 frames at
+    // a time (one lane per frame); lane 0 streams M_f.
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // Gram partials
+    if (stream) {
+      float gl = 0.f, bl = 0.f;
       int f = 0;
-      if (stream) {
-        for (; f < p.F; ++f) {
-          if (!mbar_wait(mempty, static_cast<uint32_t>((f & 1) ^ 1), abort, kCode)) break;
-          const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
-          int32_t c0, c1;
-          p.wp.slot_range(u, c0, c1);
-          hdr->c0 = c0;
-          hdr->c1 = c1;
-          hdr->a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));
-          hdr->beta = 1.0f / (1.0f + expf(-__ldg(p.beta + u)));
-          mbar_arrive_expect_tx(mfull, C::kMBytes);
-          bulk_load(smem_u32(mst), p.mpartial + (u + c0) * static_cast<int64_t>(D) * D,
-                    C::kMBytes, mfull);
+      for (; f < p.F; ++f) {
+        if ((f & 31) == 0) {
+          const int ff = f + lane;
+          gl = ff < p.F ? __ldg(p.gate + u0 + static_cast<int64_t>(ff) * p.H) : 0.f;
+          bl = ff < p.F ? __ldg(p.beta + u0 + static_cast<int64_t>(ff) * p.H) : 0.f;
         }
-        if (f > 0) mbar_wait_drain(mfull, static_cast<uint32_t>((f - 1) & 1));
+        const float g = __shfl_sync(0xffffffffu, gl, f & 31);
+        const float bb = __shfl_sync(0xffffffffu, bl, f & 31);
+        int ok = 1;
+        if (lane == 0) {
+          const int s = f % S;
+          ok = mbar_wait(mempty(s), static_cast<uint32_t>(((f / S) & 1) ^ 1), abort, kCode) ? 1 : 0;
+          if (ok) {
+            const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
+            int32_t c0, c1;
+            p.wp.slot_range(u, c0, c1);
+            GdnStageHeader* hd = hdr(s);
+            hd->c0 = c0;
+            hd->c1 = c1;
+            hd->a = 1.0f / (1.0f + expf(-g));
+            hd->beta = 1.0f / (1.0f + expf(-bb));
+            mbar_arrive_expect_tx(mfull(s), C::kMBytes);
+            bulk_load(smem_u32(mst(s)), p.mpartial + (u + c0) * static_cast<int64_t>(D) * D,
+                      C::kMBytes, mfull(s));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
+      if (lane == 0)
+        for (int k = (f > S ? f - S : 0); k < f; ++k)
+          mbar_wait_drain(mfull(k % S), static_cast<uint32_t>((k / S) & 1));
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issuer
@@ -486,53 +507,57 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
       mma_commit(done_bar);
       mbar_wait_drain(done_bar, 0);
     }
-  } else {
+  } else if (warp < 4) {
     // --------------------------------------------------------------- consumers
     const int i = threadIdx.x;  // state row / TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float* srow_s = stile + i * C::kMaxCols;
+    float sr[MC];  // row i of the group's columns of the state, fp32
     // B operand element (k = i, column jl): atom jl / 16, 32-byte row i,
     // 16-byte chunk (jl % 16) / 8 swizzled with bit 2 of the row
     auto b_off = [&](int jl) {
       return (jl >> 4) * C::kBAtomBytes + i * 32 + ((((jl >> 3) & 1) ^ ((i >> 2) & 1)) << 4);
     };
-    auto write_b = [&](const float* s) {  // all of the group's columns of row i
-      for (int jc = 0; jc < np; jc += 8) {
-        float x[8];
+    auto write_b = [&]() {  // the group's columns of row i, hi and lo
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = (jc + e < ncols) ? s[jc + e] : 0.f;
-        uint32_t hw[4], lw[4];
+      for (int jc = 0; jc < MC; jc += 8) {
+        if (jc < np) {
+          uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          hw[e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
-          lw[e2] = pack_bf16x2(x[2 * e2] - bf16lo_to_f32(hw[e2]),
-                               x[2 * e2 + 1] - bf16hi_to_f32(hw[e2]));
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float x0 = (jc + 2 * e2 < ncols) ? sr[jc + 2 * e2] : 0.f;
+            const float x1 = (jc + 2 * e2 + 1 < ncols) ? sr[jc + 2 * e2 + 1] : 0.f;
+            hw[e2] = pack_bf16x2(x0, x1);
+            lw[e2] = pack_bf16x2(x0 - bf16lo_to_f32(hw[e2]), x1 - bf16hi_to_f32(hw[e2]));
+          }
+          st_shared_v4(b_hi + b_off(jc), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+          st_shared_v4(b_lo + b_off(jc), make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
-        st_shared_v4(b_hi + b_off(jc), make_uint4(hw[0], hw[1], hw[2], hw[3]));
-        st_shared_v4(b_lo + b_off(jc), make_uint4(lw[0], lw[1], lw[2], lw[3]));
       }
     };
     // S_{-1}: row i of the group's columns
-    for (int jl = 0; jl < ncols; ++jl)
-      srow_s[jl] = p.state_in != nullptr
-                       ? p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl]
-                       : 0.f;
-    if (stream) write_b(srow_s);
+#pragma unroll
+    for (int jl = 0; jl < MC; ++jl)
+      sr[jl] = (jl < ncols && p.state_in != nullptr)
+                   ? p.state_in[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl]
+                   : 0.f;
+    if (stream) write_b();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int f = 0; f < p.F; ++f) {
       const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
       float a, beta;
       if (stream) {
-        if (!warp_wait(mfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
-        a = hdr->a;
-        beta = hdr->beta;
-        const int32_t c0 = hdr->c0, c1 = hdr->c1;
+        const int s = f % S;
+        if (!warp_wait(mfull(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
+        const GdnStageHeader hd = *hdr(s);
+        a = hd.a;
+        beta = hd.beta;
         // A operands: row i of M_f (= column i, M symmetric), hi and lo
+        const float* m = mst(s);
 #pragma unroll 2
         for (int ch = 0; ch < D / 8; ++ch) {
           float x[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = mst[(ch * 8 + e) * D + i];
+          for (int e = 0; e < 8; ++e) x[e] = m[(ch * 8 + e) * D + i];
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
@@ -548,17 +573,17 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(mempty);   // the producer may load the next frame's M
-          mbar_arrive(opready);  // A of this frame and B (written last frame) ready
+          mbar_arrive(mempty(s));  // the producer may load M_{f+2} into this stage
+          mbar_arrive(opready);    // A of this frame and B (written last frame) ready
         }
         // this frame's dS rows, loaded while the product runs
-        float ds[C::kMaxCols];
+        float ds[MC];
 #pragma unroll
-        for (int jl = 0; jl < C::kMaxCols; ++jl) ds[jl] = 0.f;
-        for (int cc = c0; cc <= c1; ++cc) {
+        for (int jl = 0; jl < MC; ++jl) ds[jl] = 0.f;
+        for (int cc = hd.c0; cc <= hd.c1; ++cc) {
           const float* src = p.partial + (u + cc) * PF + static_cast<int64_t>(j0) * D + i;
 #pragma unroll
-          for (int jl = 0; jl < C::kMaxCols; ++jl)
+          for (int jl = 0; jl < MC; ++jl)
             if (jl < ncols) ds[jl] += __ldg(src + static_cast<int64_t>(jl) * D);
         }
         if (!warp_wait(accfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
@@ -569,34 +594,35 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
         tmem_wait_ld();
         tc_fence_before();
 #pragma unroll
-        for (int jl = 0; jl < C::kMaxCols; ++jl) {
-          if (jl < ncols) {
-            const float acc = __uint_as_float(r[jl >> 5][jl & 31]);
-            srow_s[jl] = a * fmaf(-beta, acc, srow_s[jl]) + beta * ds[jl];
-          }
-        }
+        for (int jl = 0; jl < MC; ++jl)
+          if (jl < ncols)
+            sr[jl] = a * fmaf(-beta, __uint_as_float(r[jl >> 5][jl & 31]), sr[jl]) + beta * ds[jl];
       } else {
         a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));  // no tokens: the state only decays
-        for (int jl = 0; jl < ncols; ++jl) srow_s[jl] *= a;
+#pragma unroll
+        for (int jl = 0; jl < MC; ++jl) sr[jl] *= a;
       }
       // bf16 image of S_f^T: row j = j0 + jl, element i
       if (p.image != nullptr) {
         uint16_t* img = reinterpret_cast<uint16_t*>(p.image + u * G::kImageBytes);
         const int ci = i / 8;
-        for (int jl = 0; jl < ncols; ++jl) {
-          const int j = j0 + jl;
-          const int64_t off = (ci / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
-                              G::swz(j, ci % CPA) * 16 + (i % 8) * 2;
-          img[off / 2] = static_cast<uint16_t>(pack_bf16x2(srow_s[jl], 0.f) & 0xFFFFu);
+#pragma unroll
+        for (int jl = 0; jl < MC; ++jl) {
+          if (jl < ncols) {
+            const int j = j0 + jl;
+            const int64_t off = (ci / CPA) * G::kImageAtomBytes + j * G::kRowBytes +
+                                G::swz(j, ci % CPA) * 16 + (i % 8) * 2;
+            img[off / 2] = static_cast<uint16_t>(pack_bf16x2(sr[jl], 0.f) & 0xFFFFu);
+          }
         }
       }
-      if (stream && f + 1 < p.F) {
-        write_b(srow_s);  // next frame's B
-      }
+      if (stream && f + 1 < p.F) write_b();  // next frame's B
     }
-    if (p.state_out != nullptr)
-      for (int jl = 0; jl < ncols; ++jl)
-        p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl] = srow_s[jl];
+    if (p.state_out != nullptr) {
+#pragma unroll
+      for (int jl = 0; jl < MC; ++jl)
+        if (jl < ncols) p.state_out[srow + static_cast<int64_t>(i) * (D + 1) + j0 + jl] = sr[jl];
+    }
   }
   __syncwarp();
   tc_fence_before();
