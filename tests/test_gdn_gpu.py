@@ -133,3 +133,15 @@ def test_full_size_720p_5s_sampled_heads():
                                         bl[b, :, h].cpu().numpy(), w.tokens_per_frame, None, w.eps)
         assert_close(sl(out), ref, "out[b=%d,h=%d]" % (b, h))
         assert_close(so[b, h].cpu().numpy(), sref, "state_out[b=%d,h=%d]" % (b, h))
+
+
+def test_streamed_calls_match_one_call():
+    """Chunking through state_out -> state_in equals one call (the delta rule
+    depends on the carried state through M_f S_{f-1})."""
+    q, k, v, g, bl, s = case(1, 3, 5, 150, 128, True, 31)
+    full, s_full = run_gpu(q, k, v, g, bl, s)
+    n = 2 * 150
+    o1, s1 = run_gpu(q[:, :n], k[:, :n], v[:, :n], g[:, :2], bl[:, :2], s)
+    o2, s2 = run_gpu(q[:, n:], k[:, n:], v[:, n:], g[:, 2:], bl[:, 2:], torch.from_numpy(s1))
+    assert_close(np.concatenate([o1, o2], axis=1), full, "out")
+    assert_close(s2, s_full, "state_out")
