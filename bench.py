@@ -41,6 +41,17 @@ from workloads import (WORKLOADS, gdn_workload, make_beta, make_grads, make_inpu
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
+
+
+def metric_for(mode: str, variant: str) -> str:
+    """The metric string of the timed path (the same for both arms)."""
+    if mode == "backward":
+        return METRIC_BWD
+    if variant == "rope":
+        return METRIC.replace("attention", "attention + 3D RoPE", 1)
+    if variant == "gdn":
+        return METRIC.replace("gated linear attention", "frame-wise gated delta rule", 1)
+    return METRIC
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "720p-5s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
@@ -269,11 +280,35 @@ def oracle_head_slices(w, heads, seed_device="cpu"):
     return out
 
 
-def time_oracle(w, budget_s: float, max_heads: int | None = None, device="cpu") -> dict:
-    """Time the fp64 oracle on (b, h) slices of the workload until `budget_s`
-    of CPU work has been done; tokens/s counts full-layer tokens (all heads)."""
+def oracle_head_call(w, variant: str):
+    """The fp64 oracle of one (b, h) slice for the layer or a variant:
+    (workload whose inputs it takes, f(q, k, v, g, b, h, s_in_bh), label)."""
     import oracle
 
+    if variant == "rope":
+        def f(q, k, v, g, b, h, s):
+            oracle.gla_rope_head(q, k, v, g, w.tokens_per_frame, w.grid_w, 0, rope_dims(w.d),
+                                 10000.0, s, w.eps)
+        return w, f, "3D-RoPE oracle"
+    if variant == "gdn":
+        wg = gdn_workload(w)
+        beta = make_beta(wg)
+
+        def f(q, k, v, g, b, h, s):
+            oracle.gla_gdn_head(q, k, v, g, beta[b, :, h], wg.tokens_per_frame, s, wg.eps)
+        return wg, f, "delta-rule oracle"
+
+    def f(q, k, v, g, b, h, s):
+        oracle.gla_head(q, k, v, g, w.tokens_per_frame, s, w.eps)
+    return w, f, "oracle"
+
+
+def time_oracle(w, budget_s: float, max_heads: int | None = None, device="cpu",
+                variant: str = "plain") -> dict:
+    """Time the fp64 oracle (of the layer or of the variant) on (b, h) slices
+    of the workload until `budget_s` of CPU work has been done; tokens/s
+    counts full-layer tokens (all heads)."""
+    w, head_fn, label = oracle_head_call(w, variant)
     pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
     if max_heads:
         pairs = pairs[:max_heads]
@@ -285,16 +320,15 @@ def time_oracle(w, budget_s: float, max_heads: int | None = None, device="cpu") 
         i = done % len(slices)
         b, h = pairs[i]
         q, k, v, g = slices[i]
-        oracle.gla_head(q, k, v, g, w.tokens_per_frame,
-                        None if s_in is None else s_in[b, h], w.eps)
+        head_fn(q, k, v, g, b, h, None if s_in is None else s_in[b, h])
         done += 1
         el = time.perf_counter() - t0
         if el >= budget_s or done >= 4 * len(pairs):
             break
     tokens = done * w.tokens / w.H * 1.0  # head-slices -> full-layer tokens
     return {"value": tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": "%d (batch, head) slices of %s (%d frames x %d tokens each), fp64 numpy, "
-                      "%.1f s wall" % (done, w.name, w.frames, w.tokens_per_frame, el),
+            "sample": "%d (batch, head) slices of %s (%d frames x %d tokens each), fp64 numpy "
+                      "%s, %.1f s wall" % (done, w.name, w.frames, w.tokens_per_frame, label, el),
             "seconds": round(el, 3)}
 
 
@@ -500,11 +534,7 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     ctas = min(units * -(-w.tokens_per_frame // 128),
                torch.cuda.get_device_properties(dev).multi_processor_count)
     launches_per_step = 3 + int(rope) + int(gdn and ctas > 0 and units % ctas != 0)
-    metric = METRIC
-    if rope:
-        metric = METRIC.replace("attention", "attention + 3D RoPE", 1)
-    elif gdn:
-        metric = METRIC.replace("gated linear attention", "frame-wise gated delta rule", 1)
+    metric = metric_for("forward", args.variant)
     res = {
         "metric": metric,
         "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -669,18 +699,28 @@ def time_oracle_backward(w, budget_s: float) -> dict:
 
 
 def run_reference(args, w):
-    """fp64 CPU oracle, one (batch, head) slice per step."""
+    """fp64 CPU oracle of the timed path (the layer, a variant or the
+    gradients), one (batch, head) slice per step."""
     import oracle
 
+    backward = args.mode == "backward"
+    w, head_fn, label = oracle_head_call(w, "plain" if backward else args.variant)
     pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
     slices = oracle_head_slices(w, pairs[:4])
     s_in = make_state(w)
+    if backward:
+        dout, _ = make_grads(w)
+        douts = [dout[b, :, h].clone() for (b, h) in pairs[:4]]
+        del dout
 
     def step(i):
         b, h = pairs[i % 4]
         q, k, v, g = slices[i % 4]
-        oracle.gla_head(q, k, v, g, w.tokens_per_frame, None if s_in is None else s_in[b, h],
-                        w.eps)
+        if backward:
+            oracle.gla_backward_head_manual(q, k, v, g, w.tokens_per_frame, douts[i % 4], None,
+                                            None, w.eps)
+        else:
+            head_fn(q, k, v, g, b, h, None if s_in is None else s_in[b, h])
 
     for i in range(args.warmup):
         step(i)
@@ -689,10 +729,12 @@ def run_reference(args, w):
         step(i)
     el = time.perf_counter() - t0
     value = args.steps * w.tokens / w.H / el
-    sample = ("one (batch, head) slice of %s per step (%d frames x %d tokens), fp64 numpy oracle"
-              % (w.name, w.frames, w.tokens_per_frame))
+    sample = ("one (batch, head) slice of %s per step (%d frames x %d tokens), fp64 numpy %s"
+              % (w.name, w.frames, w.tokens_per_frame,
+                 "gradient oracle" if backward else label))
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "impl": "reference", "metric": metric_for(args.mode, args.variant), "value": round(value, 1),
+        "unit": UNIT,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -744,7 +786,8 @@ def main(argv=None):
             res = run_gpu(args, w, dist, rank, local_rank, world)
         if rank == 0 and world == 1 and args.cpu_budget > 0:
             res["cpu_baseline"] = (time_oracle_backward(w, args.cpu_budget)
-                                   if args.mode == "backward" else time_oracle(w, args.cpu_budget))
+                                   if args.mode == "backward"
+                                   else time_oracle(w, args.cpu_budget, variant=args.variant))
         elif rank == 0:
             res["cpu_baseline"] = None
         if rank == 0:
