@@ -26,11 +26,7 @@
 // of D would put their error near the tolerance; dq uses D_hi alone.
 // The ReLU warps keep a byte mask of q > 0 for the dq epilogue, so a q stage
 // is released as soon as MMA3 has read it.
-// Warp roles: 0-3 group A, 4-7 ReLU, 8 TMA, 9 MMA, 10-13 group B.  Building D
-// is on the path that links one tile to the next, so both groups build it:
-// A the dnum columns of the first swizzle atom and the dden column, B those
-// of the second atom (B hands A its half of dout . num through shared
-// memory).  Group B then writes dq; group A writes the L_f partials.
+// Warp roles: 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
 #pragma once
 
 #include "gla_common.cuh"
@@ -55,11 +51,11 @@ struct BwdQCfg {
   static constexpr int kAcc2 = 160;  // dq~          : N = d
   static constexpr int kAcc3 = 288;  // L_f          : N = d + 16
   static constexpr int kTmemCols = 512;
-  static constexpr int kThreads = 448;
-  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing + 2;
+  static constexpr int kThreads = 320;
+  static constexpr int kBarCount = 3 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kMaskRing + 1;
   static constexpr int kSmemBytes = 1024 + kStages * G::kTileBytes + kSBufBytes + 2 * kDBytes +
-                                    2 * kStageOutBytes + kMaskRing * kMaskBytes + kTileTokens * 4 +
-                                    kBarCount * 8 + 16;
+                                    2 * kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 +
+                                    16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -72,7 +68,7 @@ struct BwdQParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(320, 1)
     gla_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_dout,
                      const __grid_constant__ CUtensorMap tm_dq, const BwdQParams p) {
@@ -95,8 +91,7 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t o_base = l_buf + C::kDBytes;
   uint8_t* mask_ring = smem + S * G::kTileBytes + C::kSBufBytes + 2 * C::kDBytes +
                        2 * C::kStageOutBytes;
-  float* dotb = reinterpret_cast<float*>(mask_ring + C::kMaskRing * C::kMaskBytes);  // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(dotb + kTileTokens);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + C::kMaskRing * C::kMaskBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto qfull = [&](int s) { return bar0 + 8u * s; };
   auto qrelu = [&](int s) { return bar0 + 8u * (S + s); };
@@ -116,7 +111,6 @@ __global__ void __launch_bounds__(448, 1)
   auto maskfull = [&](int m) { return bar0 + 8u * (3 * S + 11 + m); };
   auto maskfree = [&](int m) { return bar0 + 8u * (3 * S + 11 + R + m); };
   const uint32_t doutfull = bar0 + 8u * (3 * S + 11 + 2 * R);  // dout tile landed in D_hi
-  const uint32_t dotfull = bar0 + 8u * (3 * S + 12 + 2 * R);   // group B's half of dout . num
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -138,9 +132,8 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(sfull, 1);
     mbar_init(sempty, 1);
     mbar_init(acc1_full, 1);
-    mbar_init(acc1_free, 8);
-    mbar_init(dfull, 8);
-    mbar_init(dotfull, 4);
+    mbar_init(acc1_free, 4);
+    mbar_init(dfull, 4);
     mbar_init(dfree, 1);
     mbar_init(doutfull, 1);
     mbar_init(acc2_full, 1);
@@ -179,53 +172,6 @@ __global__ void __launch_bounds__(448, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // Building D for one swizzle atom (64 columns) of dnum: thread `row` of a
-  // 4-warp group reads the den column and its 64 num columns from TMEM and its
-  // dout row from D_hi, writes dnum (hi, lo) in place and returns its part of
-  // dout . num.  Also sets rden_row.  Issued by group A (atom 0) and group B
-  // (atom 1) of the same tile; each thread touches only its own row.
-  float rden_row = 0.f;
-  auto build_dnum_half = [&](int atom) -> float {
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
-    const uint32_t t1 = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kAcc1;
-    uint32_t dr;
-    uint32_t r[2][32];
-    tmem_ld_1col(t1 + D, dr);
-    tmem_ld_32cols(t1 + atom * 64, r[0]);
-    tmem_wait_ld();
-    rden_row = 1.0f / (__uint_as_float(dr) + p.eps);
-    const float rden = rden_row;
-    float dot4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      if (cc == 0) tmem_ld_32cols(t1 + atom * 64 + 32, r[1]);  // loads while cc = 0 runs
-      const uint32_t* rc = r[cc];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
-        const int cin = cc * 4 + ch;
-        const uint32_t off = atom * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16;
-        const uint4 dq4 = ld_shared_v4(d_buf + off);  // dout (zero past the frame's end)
-        const uint32_t dw[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
-        uint32_t w[4], wl[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float d0 = bf16lo_to_f32(dw[e2]), d1 = bf16hi_to_f32(dw[e2]);
-          dot4[e2] = fmaf(d0, __uint_as_float(rc[8 * ch + 2 * e2]), dot4[e2]);
-          dot4[e2] = fmaf(d1, __uint_as_float(rc[8 * ch + 2 * e2 + 1]), dot4[e2]);
-          const float x0 = d0 * rden, x1 = d1 * rden;
-          w[e2] = pack_bf16x2(x0, x1);
-          wl[e2] = pack_bf16x2(x0 - bf16lo_to_f32(w[e2]), x1 - bf16hi_to_f32(w[e2]));
-        }
-        st_shared_v4(d_buf + off, make_uint4(w[0], w[1], w[2], w[3]));
-        st_shared_v4(l_buf + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
-      }
-      if (cc == 0) tmem_wait_ld();
-    }
-    tc_fence_before();
-    return (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
-  };
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -351,7 +297,7 @@ __global__ void __launch_bounds__(448, 1)
       mma_commit(done_bar);
       mbar_wait_drain(done_bar, 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ ReLU
     constexpr int CPR = G::kChunksPerRow;
     constexpr int RPP = kTileTokens / CPR;
@@ -392,26 +338,57 @@ __global__ void __launch_bounds__(448, 1)
         mbar_arrive(maskfull(mr));
       }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------- D builders and L_f partials
+  } else {
+    // ------------------------------------------------------------- epilogue
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // token within the tile (= key feature for L_f)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     int64_t i = 0, seg = 0;
+    int b = 0, f = 0, h = 0;
     for (; cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
+      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       const int tok = cur.t * kTileTokens + row;
       const bool valid_tok = tok < p.T;
-      // ---- Epi1 (atom 0 of dnum, then dden): D = [dout / den | -(dout . num) / den^2]
+      // ---- Epi1: D = [dout / den | -(dout . num) / den^2]
       if (!warp_wait(acc1_full, ph, abort, kCode)) break;
       if (!warp_wait(doutfull, ph, abort, kCode)) break;  // dout in D_hi (previous D read)
       tc_fence_after();
-      const float dot_a = build_dnum_half(0);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc1_free);  // both halves of acc1 read once group B arrives
-      if (!warp_wait(dotfull, ph, abort, kCode)) break;    // group B's half of the dot
-      const float dot = dot_a + dotb[row];
-      const float rden = rden_row;
+      const uint32_t t1 = tmem + lane_base + C::kAcc1;
+      uint32_t dr;
+      tmem_ld_1col(t1 + D, dr);
+      tmem_wait_ld();
+      const float rden = 1.0f / (__uint_as_float(dr) + p.eps);
+      float dot4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld_32cols(t1 + cc * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {  // 8 columns = one 16-byte chunk of D
+          const int chunk = cc * 4 + ch;
+          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
+          const uint32_t off = a * G::kAtomTileBytes + row * G::kRowBytes + G::swz(row, cin) * 16;
+          const uint4 dq4 = ld_shared_v4(d_buf + off);  // dout (zero past the frame's end)
+          const uint32_t dw[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+          uint32_t w[4], wl[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint32_t wpair = dw[e2];
+            const float d0 = bf16lo_to_f32(wpair), d1 = bf16hi_to_f32(wpair);
+            dot4[e2] = fmaf(d0, __uint_as_float(r[8 * ch + 2 * e2]), dot4[e2]);
+            dot4[e2] = fmaf(d1, __uint_as_float(r[8 * ch + 2 * e2 + 1]), dot4[e2]);
+            const float x0 = d0 * rden, x1 = d1 * rden;
+            w[e2] = pack_bf16x2(x0, x1);
+            wl[e2] = pack_bf16x2(x0 - bf16lo_to_f32(w[e2]), x1 - bf16hi_to_f32(w[e2]));
+          }
+          st_shared_v4(d_buf + off, make_uint4(w[0], w[1], w[2], w[3]));
+          st_shared_v4(l_buf + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+        }
+      }
+      tc_fence_before();
+      const float dot = (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
       const float dden = valid_tok ? -dot * rden * rden : 0.f;
       const uint32_t dden_hi = pack_bf16x2(dden, 0.f);
       const float dden_lo = dden - bf16lo_to_f32(dden_hi);
@@ -421,54 +398,11 @@ __global__ void __launch_bounds__(448, 1)
       st_shared_v4(l_pad + poff, make_uint4(pack_bf16x2(dden_lo, 0.f), 0u, 0u, 0u));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dfull);
-      // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
-      if (cur.last) {
-        if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
-        tc_fence_after();
-        float* dst = p.partial + cur.slot() * static_cast<int64_t>(PF) + row;
-        const uint32_t t3 = tmem + lane_base + C::kAcc3;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r3[32];
-          tmem_ld_32cols(t3 + cc * 32, r3);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r3[jj]);
-        }
-        uint32_t zr;
-        tmem_ld_1col(t3 + D, zr);
-        tmem_wait_ld();
-        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc3_free);
-        ++seg;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ dq writers
-    const int q4 = warp & 3;          // TMEM lanes 32 q4 .. 32 q4 + 31
-    const int row = q4 * 32 + lane;   // token within the tile
-    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    int64_t i = 0;
-    int b = 0, f = 0, h = 0;
-    for (; cur.valid(); cur.advance(), ++i) {
-      const uint32_t ph = static_cast<uint32_t>(i & 1);
-      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
-      // ---- Epi1 (atom 1 of dnum): D's second half and half of dout . num
-      if (!warp_wait(acc1_full, ph, abort, kCode)) break;
-      if (!warp_wait(doutfull, ph, abort, kCode)) break;
-      tc_fence_after();
-      const float dot_b = build_dnum_half(1);
-      dotb[row] = dot_b;
-      fence_proxy_async_smem();
-      __syncwarp();
       if (lane == 0) {
-        mbar_arrive(dotfull);
         mbar_arrive(acc1_free);
         mbar_arrive(dfull);
       }
+
       // ---- Epi2: dq = 1[q > 0] * dq~
       if (!warp_wait(acc2_full, ph, abort, kCode)) break;
       const int mr = static_cast<int>(i % R);
@@ -520,6 +454,29 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc2_free);
+      // ---- Epi3 (unit end): L_f partial, row j = state column, column i = row
+      if (cur.last) {
+        if (!warp_wait(acc3_full, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        tc_fence_after();
+        float* dst = p.partial + cur.slot() * static_cast<int64_t>(PF) + row;
+        const uint32_t t3 = tmem + lane_base + C::kAcc3;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(t3 + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+        }
+        uint32_t zr;
+        tmem_ld_1col(t3 + D, zr);
+        tmem_wait_ld();
+        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc3_free);
+        ++seg;
+      }
     }
     if (lane == 0) bulk_wait_group<0>();
   }

@@ -111,6 +111,7 @@ struct RopeStep {
   float4 ia01, ia23;  // next row on the same latent row (no wrap)
   float4 ib01, ib23;  // next row after a wrap
   int step_mod;       // rpp mod grid_w
+  bool moving;        // false for the temporal block (one angle per frame)
 };
 
 // Once per thread: the increments of chunk c (pairs 4c .. 4c+3).
@@ -122,6 +123,7 @@ __device__ __forceinline__ void rope_step_init(const RopeGeo& g, int c, int half
   st.ib01 = __ldg(g.table + ib);
   st.ib23 = __ldg(g.table + ib + 1);
   st.step_mod = g.rpp % g.grid_w;
+  st.moving = 8 * c >= g.dt;
 }
 
 __device__ __forceinline__ float4 cmul2(const float4& a, const float4& b) {
@@ -131,6 +133,7 @@ __device__ __forceinline__ float4 cmul2(const float4& a, const float4& b) {
 
 // Move to the next row (rp still describes the current row).
 __device__ __forceinline__ void rope_step_next(RopeStep& st, const RopeRowPos& rp, int grid_w) {
+  if (!st.moving) return;
   const bool wrap = rp.x + st.step_mod >= grid_w;
   st.cs01 = cmul2(st.cs01, wrap ? st.ib01 : st.ia01);
   st.cs23 = cmul2(st.cs23, wrap ? st.ib23 : st.ia23);
