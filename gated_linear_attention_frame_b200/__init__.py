@@ -30,11 +30,14 @@ from ._binding import (  # noqa: F401
     gla_forward_rope,
     gla_forward_rope_timed,
     gla_forward_timed,
+    gla_softmax_anchor,
+    gla_softmax_anchor_timed,
     gla_noalloc_scratch_bytes,
     gla_trim_workspace,
     gla_version,
     load_library,
     rope_config,
+    softmax_anchor,
 )
 
 # Every entry point loads libgla.so on first use and raises ImportError when

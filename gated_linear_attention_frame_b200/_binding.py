@@ -28,6 +28,7 @@ GLA_ERR_ROPE = 9
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
             "gla_forward_rope", "gla_forward_rope_timed", "gla_forward_gdn", "gla_forward_gdn_timed",
+            "gla_softmax_anchor", "gla_softmax_anchor_timed",
             "gla_backward", "gla_backward_timed",
             "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
 
@@ -74,6 +75,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_forward_timed.restype = i32
     lib.gla_forward_noalloc.argtypes = fwd
     lib.gla_forward_noalloc.restype = i32
+    anc = [vp] * 5 + [i32] * 7 + [vp]
+    lib.gla_softmax_anchor.argtypes = anc
+    lib.gla_softmax_anchor.restype = i32
+    lib.gla_softmax_anchor_timed.argtypes = anc + [ctypes.POINTER(vp)]
+    lib.gla_softmax_anchor_timed.restype = i32
     gdn = fwd[:4] + [vp] + fwd[4:]
     lib.gla_forward_gdn.argtypes = gdn
     lib.gla_forward_gdn.restype = i32
@@ -183,6 +189,49 @@ def gla_forward_noalloc(q, k, v, gate_logits, state_in, state_out, out, B, H, fr
                                  int(tokens_per_frame), int(d), float(eps), _stream(stream))
     if st != GLA_OK:
         raise GLAError(st, "gla_forward_noalloc")
+
+
+def gla_softmax_anchor(q, k, v, gate_z, out, B, H, frames, tokens_per_frame, d, window_frames,
+                       n_sink, stream=None) -> None:
+    """The softmax anchor layer: attention sinks + a local window of frames,
+    optional sigmoid output gate (see include/gla.h; d = 128)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("gate_z", gate_z), ("out", out)):
+        if isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+            raise TypeError("gla: %s must be torch.bfloat16, got %s" % (name, t.dtype))
+    st = load_library().gla_softmax_anchor(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(out),
+                                           int(B), int(H), int(frames), int(tokens_per_frame),
+                                           int(d), int(window_frames), int(n_sink),
+                                           _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_softmax_anchor")
+
+
+def gla_softmax_anchor_timed(q, k, v, gate_z, out, B, H, frames, tokens_per_frame, d,
+                             window_frames, n_sink, stream, events) -> None:
+    """gla_softmax_anchor with 2 CUDA events around the kernel."""
+    lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 2)(*[e.cuda_event for e in events])
+    st = lib.gla_softmax_anchor_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(out), int(B),
+                                      int(H), int(frames), int(tokens_per_frame), int(d),
+                                      int(window_frames), int(n_sink), _stream(stream),
+                                      ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_softmax_anchor_timed")
+
+
+def softmax_anchor(q, k, v, frames, window_frames, n_sink=0, gate_z=None, out=None, stream=None):
+    """Convenience wrapper of gla_softmax_anchor; returns out."""
+    B, N, H, d = q.shape
+    T = N // frames if frames else 0
+    if frames and N % frames:
+        raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+    if out is None:
+        out = torch.empty_like(q)
+    gla_softmax_anchor(q, k, v, gate_z, out, B, H, frames, T, d, window_frames, n_sink, stream)
+    return out
 
 
 def gla_forward_gdn(q, k, v, gate_logits, beta_logits, state_in, state_out, out, B, H, frames,

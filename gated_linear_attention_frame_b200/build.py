@@ -22,7 +22,7 @@ DEPENDS = SOURCES + [
     os.path.join(CSRC, n)
     for n in ("sm100_ptx.cuh", "gla_common.cuh", "gla_increment.cuh", "gla_scan.cuh",
               "gla_output.cuh", "gla_bwd_q.cuh", "gla_scan_bwd.cuh", "gla_bwd_kv.cuh",
-              "gla_rope.cuh", "gla_gdn_scan.cuh")
+              "gla_rope.cuh", "gla_gdn_scan.cuh", "gla_softmax_anchor.cuh")
 ] + [os.path.join(INCLUDE, "gla.h")]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -18,6 +18,8 @@
 //   1. gla_increment_kernel  dS_f and M_f = phi(K_f)^T phi(K_f) partials (tcgen05)
 //   2. gla_gdn_scan_kernel   S_f = a_f (S_{f-1} - beta_f M_f S_{f-1}) + beta_f dS_f
 //   3. gla_output_kernel     as gla_forward
+// gla_softmax_anchor (d = 128) runs gla_softmax_anchor_kernel: two passes of
+// tcgen05 Q K^T over the key tiles of sinks + window, P V into TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -37,6 +39,7 @@
 #include "gla_rope.cuh"
 #include "gla_scan.cuh"
 #include "gla_scan_bwd.cuh"
+#include "gla_softmax_anchor.cuh"
 #include "sm100_ptx.cuh"
 
 namespace {
@@ -119,6 +122,10 @@ cudaError_t set_smem_attrs() {
                            gla::GdnScanCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   if constexpr (D == 128) {
+    e = cudaFuncSetAttribute(gla::gla_softmax_anchor_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gla::AnchorCfg<128>::kSmemBytes);
+    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gla::gla_gdn_scan_tc_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gla::GdnTcCfg<128>::kSmemBytes);
@@ -738,6 +745,46 @@ int backward_impl(const BwdArgs& a, cudaEvent_t* ev) {
   return run_backward(a, di, ev);
 }
 
+// The softmax anchor layer (d = 128).
+int anchor_impl(const void* q, const void* k, const void* v, const void* z, void* out, int B,
+                int H, int F, int T, int d, int window, int n_sink, cudaStream_t stream,
+                cudaEvent_t* ev) {
+  if (d != 128) return GLA_ERR_UNSUPPORTED_D;
+  Args chk{q, k, v, nullptr, nullptr, nullptr, out, B, H, F, T, d, 0.f, stream};
+  const int64_t units0 = static_cast<int64_t>(B) * F * H;
+  static const float kNone = 0.f;  // the validator wants gate logits when units > 0
+  chk.g = units0 > 0 ? &kNone : nullptr;
+  int st = validate(chk);
+  if (st != GLA_OK) return st;
+  if (window < 1 || n_sink < 0) return GLA_ERR_SHAPE;
+  if (z != nullptr && !aligned(z, 16)) return GLA_ERR_ALIGN;
+  const int tpf = (T + gla::kTileTokens - 1) / gla::kTileTokens;
+  const int64_t units = units0 * tpf;
+  if (units > INT32_MAX) return GLA_ERR_SHAPE;
+  if (units == 0) return GLA_OK;
+  DeviceInfo di;
+  if ((st = device_setup(&di)) != GLA_OK) return st;
+  CUtensorMap tm_q, tm_k, tm_v, tm_z, tm_out;
+  if ((st = encode_map(&tm_q, q, d, H, T, F, B, gla::kTileTokens)) != GLA_OK) return st;
+  if ((st = encode_map(&tm_k, k, d, H, T, F, B, gla::kTileTokens)) != GLA_OK) return st;
+  if ((st = encode_map(&tm_v, v, d, H, T, F, B, gla::kTileTokens)) != GLA_OK) return st;
+  if ((st = encode_map(&tm_z, z != nullptr ? z : q, d, H, T, F, B, gla::kTileTokens)) != GLA_OK)
+    return st;
+  if ((st = encode_map(&tm_out, out, d, H, T, F, B, 32)) != GLA_OK) return st;
+  gla::AnchorParams ap{H, F, T, window, n_sink, static_cast<int>(units),
+                       static_cast<float>(1.4426950408889634 / std::sqrt(128.0)), z != nullptr};
+  const int grid = static_cast<int>(units < di.sms ? units : di.sms);
+  int status = GLA_OK;
+  if (ev != nullptr && cudaEventRecord(ev[0], stream) != cudaSuccess) return GLA_ERR_LAUNCH;
+  gla::gla_softmax_anchor_kernel<128>
+      <<<grid, gla::AnchorCfg<128>::kThreads, gla::AnchorCfg<128>::kSmemBytes, stream>>>(
+          tm_q, tm_k, tm_v, tm_z, tm_out, ap);
+  if (cudaGetLastError() != cudaSuccess) status = GLA_ERR_LAUNCH;
+  if (ev != nullptr && status == GLA_OK && cudaEventRecord(ev[1], stream) != cudaSuccess)
+    status = GLA_ERR_LAUNCH;
+  return status;
+}
+
 }  // namespace
 
 extern "C" {
@@ -769,6 +816,22 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v, const float
 }
 
 size_t gla_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int gla_softmax_anchor(const void* q, const void* k, const void* v, const void* gate_z,
+                       void* out, int B, int H, int frames, int tokens_per_frame, int d,
+                       int window_frames, int n_sink, cudaStream_t stream) {
+  return anchor_impl(q, k, v, gate_z, out, B, H, frames, tokens_per_frame, d, window_frames,
+                     n_sink, stream, nullptr);
+}
+
+int gla_softmax_anchor_timed(const void* q, const void* k, const void* v, const void* gate_z,
+                             void* out, int B, int H, int frames, int tokens_per_frame, int d,
+                             int window_frames, int n_sink, cudaStream_t stream,
+                             cudaEvent_t* events) {
+  if (events == nullptr) return GLA_ERR_NULL;
+  return anchor_impl(q, k, v, gate_z, out, B, H, frames, tokens_per_frame, d, window_frames,
+                     n_sink, stream, events);
+}
 
 int gla_forward_gdn(const void* q, const void* k, const void* v, const float* gate_logits,
                     const float* beta_logits, const float* state_in, float* state_out, void* out,

@@ -1,0 +1,464 @@
+// gla_softmax_anchor.cuh -- the softmax anchor layer (attention sinks + a
+// local window of frames) on tcgen05.
+//
+// The SANA-Video 2.0 pages put a gated-softmax anchor after every three
+// linear layers; the SANA-WM pages give the softmax layers attention-sink
+// tokens and a local temporal window so that memory and per-chunk latency stay
+// constant over long rollouts.  This library's reading, per (b, h): the
+// queries of frame f attend to all tokens of frames max(0, f-W+1) .. f and to
+// the first n_sink tokens of the sequence that precede that window, with
+// scores q . k / sqrt(d); out = sigmoid(z) * softmax-weighted sum of v (z an
+// optional per-element gate).
+//
+// One work unit = 128 query tokens of one (b, f, h).  Its key tiles (128 keys
+// of one frame, the frame's last tile ragged) are walked twice:
+//   pass 1  S = Q K^T into TMEM (double-buffered); the softmax warps keep the
+//           running row maximum m (invalid key rows masked to -inf);
+//   pass 2  S = Q K^T again; the softmax warps write P = exp(S - m) in bf16 to
+//           shared memory and sum l = sum P; O += P V accumulates in TMEM.
+// Two passes cost one more Q K^T per tile but need no rescaling of the TMEM
+// accumulator when the maximum grows.  The epilogue writes sigmoid(z) O / l.
+//   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
+//   PV: A = P [M = 128 queries, K = 128 keys] K-major, B = V tile [N = d] MN-major
+// Warp roles: 0-3 softmax / epilogue (thread = query row), 4 TMA, 5 MMA.
+#pragma once
+
+#include "gla_common.cuh"
+#include "gla_increment.cuh"  // warp_wait, unit_coords
+#include "sm100_ptx.cuh"
+
+namespace gla {
+
+struct AnchorParams {
+  int H, F, T;       // heads, frames, tokens per frame
+  int window;        // W >= 1 frames
+  int n_sink;        // sink tokens at the start of the sequence
+  int units;         // B * F * H * tiles per frame
+  float scale_log2;  // log2(e) / sqrt(d)
+  int has_gate;
+};
+
+// The key tiles of the queries of frame f, in order: the sink tokens that
+// precede the window (frames 0 .., the last one possibly partial), then the
+// window's frames.  Each tile is (frame, first token t0, valid rows).
+struct KeyTiles {
+  int T, f, w_lo_frame, s_hi;  // s_hi: sink tokens [0, s_hi), s_hi <= w_lo_frame * T
+  int fr, t0, valid, end_t;    // current tile
+  bool in_sink, done;
+
+  __device__ void init(int T_, int f_, int window, int n_sink) {
+    T = T_;
+    f = f_;
+    w_lo_frame = f - window + 1 > 0 ? f - window + 1 : 0;
+    const int w_lo = w_lo_frame * T;
+    s_hi = n_sink < w_lo ? n_sink : w_lo;
+    done = false;
+    if (s_hi > 0) {
+      in_sink = true;
+      fr = 0;
+    } else {
+      in_sink = false;
+      fr = w_lo_frame;
+    }
+    t0 = 0;
+    set_end();
+    if (end_t <= 0) done = true;  // T == 0
+    valid = end_t - t0 < kTileTokens ? end_t - t0 : kTileTokens;
+  }
+  __device__ void set_end() {
+    end_t = in_sink ? ((s_hi - fr * T) < T ? s_hi - fr * T : T) : T;
+  }
+  __device__ void advance() {
+    t0 += kTileTokens;
+    if (t0 >= end_t) {
+      t0 = 0;
+      ++fr;
+      if (in_sink && fr * T >= s_hi) {
+        in_sink = false;
+        fr = w_lo_frame;
+      }
+      if (!in_sink && fr > f) {
+        done = true;
+        return;
+      }
+      set_end();
+    }
+    valid = end_t - t0 < kTileTokens ? end_t - t0 : kTileTokens;
+  }
+};
+
+template <int D>
+struct AnchorCfg {
+  using G = Geo<D>;
+  static_assert(D == 128, "the softmax anchor kernel is built for d = 128");
+  static constexpr int kStages = 3;                 // K / V tile ring
+  static constexpr int kTileBytes = G::kTileBytes;  // 32 KB
+  static constexpr int kThreads = 192;
+  static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128)
+  static constexpr int kAccO = 256;
+  static constexpr int kBarCount = 2 * kStages + 14;
+  static constexpr int kSmemBytes = 1024 + (3 + kStages) * kTileBytes + kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    gla_softmax_anchor_kernel(const __grid_constant__ CUtensorMap tm_q,
+                              const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v,
+                              const __grid_constant__ CUtensorMap tm_z,
+                              const __grid_constant__ CUtensorMap tm_out, const AnchorParams p) {
+  using G = Geo<D>;
+  using C = AnchorCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr unsigned kCode = 128u;
+  constexpr int KPA = G::kAtomElems / 16;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t q_buf = sbase;
+  const uint32_t p_buf = sbase + C::kTileBytes;
+  const uint32_t o_buf = sbase + 2 * C::kTileBytes;  // gate in, output out
+  auto ring = [&](int s) { return sbase + (3 + s) * C::kTileBytes; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (3 + S) * C::kTileBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto rfull = [&](int s) { return bar0 + 8u * s; };
+  auto rempty = [&](int s) { return bar0 + 8u * (S + s); };
+  const uint32_t qfull = bar0 + 8u * (2 * S + 0);
+  const uint32_t qempty = bar0 + 8u * (2 * S + 1);
+  auto sfull = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+  auto sfree = [&](int b) { return bar0 + 8u * (2 * S + 4 + b); };
+  const uint32_t pfull = bar0 + 8u * (2 * S + 6);
+  const uint32_t pfree = bar0 + 8u * (2 * S + 7);
+  const uint32_t ofull = bar0 + 8u * (2 * S + 8);
+  const uint32_t ofree = bar0 + 8u * (2 * S + 9);
+  const uint32_t zfull = bar0 + 8u * (2 * S + 10);
+  const uint32_t zfree = bar0 + 8u * (2 * S + 11);
+  const uint32_t done_bar = bar0 + 8u * (2 * S + 12);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tpf = (p.T + kTileTokens - 1) / kTileTokens;  // query tiles per frame
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(rfull(s), 1);
+      mbar_init(rempty(s), 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sfull(b), 1);
+      mbar_init(sfree(b), 4);
+    }
+    mbar_init(pfull, 4);
+    mbar_init(pfree, 1);
+    mbar_init(ofull, 1);
+    mbar_init(ofree, 4);
+    mbar_init(zfull, 1);
+    mbar_init(zfree, 4);
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // unit -> (b, f, h, query tile): unit = ((b * F + f) * H + h) * tpf + qt
+  auto coords = [&](int unit, int& b, int& f, int& h, int& qt) {
+    qt = unit % tpf;
+    const int u = unit / tpf;
+    unit_coords(u, p.H, p.F, b, f, h);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int64_t n = 0;  // ring tiles issued
+      int64_t it = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++it) {
+        int b, f, h, qt;
+        coords(unit, b, f, h, qt);
+        const uint32_t ph = static_cast<uint32_t>(it & 1);
+        if (!mbar_wait(qempty, ph ^ 1u, abort, kCode)) break;
+        mbar_arrive_expect_tx(qfull, G::kTileBytes);
+        for (int a = 0; a < G::kAtoms; ++a)
+          tma_load_5d(q_buf + a * G::kAtomTileBytes, &tm_q, qfull, a * G::kAtomElems, h,
+                      qt * kTileTokens, f, b);
+        if (p.has_gate) {
+          if (!mbar_wait(zfree, ph ^ 1u, abort, kCode)) break;
+          mbar_arrive_expect_tx(zfull, G::kTileBytes);
+          for (int a = 0; a < G::kAtoms; ++a)
+            tma_load_5d(o_buf + a * G::kAtomTileBytes, &tm_z, zfull, a * G::kAtomElems, h,
+                        qt * kTileTokens, f, b);
+        }
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          KeyTiles kt;
+          kt.init(p.T, f, p.window, p.n_sink);
+          for (; !kt.done; kt.advance()) {
+            for (int which = 0; which < pass + 1; ++which) {  // pass 2: K then V
+              const int s = static_cast<int>(n % S);
+              if (!mbar_wait(rempty(s), static_cast<uint32_t>(((n / S) & 1) ^ 1), abort, kCode)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(rfull(s), G::kTileBytes);
+              const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
+              for (int a = 0; a < G::kAtoms; ++a)
+                tma_load_5d(ring(s) + a * G::kAtomTileBytes, tm, rfull(s), a * G::kAtomElems, h,
+                            kt.t0, kt.fr, b);
+              ++n;
+            }
+            if (!ok) break;
+          }
+        }
+      }
+      for (int64_t i = (n > S ? n - S : 0); i < n; ++i)
+        mbar_wait_drain(rfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileTokens, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      int64_t n = 0, ns = 0, np = 0;  // ring tiles consumed, S tiles, P tiles
+      int64_t it = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++it) {
+        int b, f, h, qt;
+        coords(unit, b, f, h, qt);
+        const uint32_t ph = static_cast<uint32_t>(it & 1);
+        if (!mbar_wait(qfull, ph, abort, kCode)) break;
+        bool first_pv = true;
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          KeyTiles kt;
+          kt.init(p.T, f, p.window, p.n_sink);
+          for (; !kt.done; kt.advance()) {
+            // S = Q K^T into buffer ns % 2
+            const int sb = static_cast<int>(ns & 1);
+            const int s = static_cast<int>(n % S);
+            if (!mbar_wait(sfree(sb), static_cast<uint32_t>(((ns >> 1) & 1) ^ 1), abort, kCode) ||
+                !mbar_wait(rfull(s), static_cast<uint32_t>((n / S) & 1), abort, kCode)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int a = kk / KPA, w = kk % KPA;
+              const uint64_t ad = smem_desc(q_buf + a * G::kAtomTileBytes + w * 32, 16,
+                                            G::kGroupBytes, G::kLayout);
+              const uint64_t bd = smem_desc(ring(s) + a * G::kAtomTileBytes + w * 32, 16,
+                                            G::kGroupBytes, G::kLayout);
+              mma_bf16(tmem + sb * kTileTokens, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(sfull(sb));
+            mma_commit(rempty(s));
+            ++n;
+            ++ns;
+            if (pass == 1) {
+              // O += P V once the softmax warps wrote P of this tile
+              const int sv = static_cast<int>(n % S);
+              if (!mbar_wait(pfull, static_cast<uint32_t>(np & 1), abort, kCode) ||
+                  !mbar_wait(rfull(sv), static_cast<uint32_t>((n / S) & 1), abort, kCode)) {
+                ok = false;
+                break;
+              }
+              if (first_pv && !mbar_wait(ofree, ph ^ 1u, abort, kCode)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+                const int a = kk / KPA, w = kk % KPA;
+                const uint64_t ad = smem_desc(p_buf + a * G::kAtomTileBytes + w * 32, 16,
+                                              G::kGroupBytes, G::kLayout);
+                const uint64_t bd = smem_desc(ring(sv) + kk * 2 * G::kGroupBytes,
+                                              G::kAtomTileBytes, G::kGroupBytes, G::kLayout);
+                mma_bf16(tmem + C::kAccO, ad, bd, idesc_o, (first_pv && kk == 0) ? 0u : 1u);
+              }
+              first_pv = false;
+              mma_commit(pfree);
+              mma_commit(rempty(sv));
+              ++n;
+              ++np;
+            }
+          }
+        }
+        if (!ok) break;
+        mma_commit(qempty);  // Q no longer read
+        mma_commit(ofull);   // O of this unit complete
+      }
+      mma_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else {
+    // -------------------------------------------------- softmax and epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // query within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int64_t ns = 0, np = 0, it = 0;
+    for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x, ++it) {
+      int b, f, h, qt;
+      coords(unit, b, f, h, qt);
+      const uint32_t ph = static_cast<uint32_t>(it & 1);
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        KeyTiles kt;
+        kt.init(p.T, f, p.window, p.n_sink);
+        for (; !kt.done; kt.advance()) {
+          const int sb = static_cast<int>(ns & 1);
+          if (!warp_wait(sfull(sb), static_cast<uint32_t>((ns >> 1) & 1), abort, kCode)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ts = tmem + lane_base + sb * kTileTokens;
+          if (pass == 0) {
+            float mx = m;
+#pragma unroll
+            for (int cc = 0; cc < kTileTokens / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(ts + cc * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (cc * 32 + e < kt.valid) mx = fmaxf(mx, __uint_as_float(r[e]));
+            }
+            m = mx;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sfree(sb));
+          } else {
+            // P = exp2((S - m) * scale log2 e) for valid keys, 0 past them
+            if (!warp_wait(pfree, static_cast<uint32_t>((np & 1) ^ 1), abort, kCode)) {
+              ok = false;
+              break;
+            }
+            const float ms = m * p.scale_log2;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int cc = 0; cc < kTileTokens / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(ts + cc * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int ch = 0; ch < 4; ++ch) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int col = cc * 32 + ch * 8 + e;
+                  x[e] = col < kt.valid ? exp2f(fmaf(__uint_as_float(r[ch * 8 + e]),
+                                                     p.scale_log2, -ms))
+                                        : 0.f;
+                  ls[e & 3] += x[e];
+                }
+                uint4 w;
+                w.x = pack_bf16x2(x[0], x[1]);
+                w.y = pack_bf16x2(x[2], x[3]);
+                w.z = pack_bf16x2(x[4], x[5]);
+                w.w = pack_bf16x2(x[6], x[7]);
+                const int chunk = cc * 4 + ch;
+                const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
+                st_shared_v4(p_buf + a * G::kAtomTileBytes + row * G::kRowBytes +
+                                 G::swz(row, cin) * 16,
+                             w);
+              }
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(sfree(sb));
+              mbar_arrive(pfull);
+            }
+            ++np;
+          }
+          ++ns;
+        }
+      }
+      if (!ok) break;
+      // ---- epilogue: out = sigmoid(z) * O / l
+      if (!warp_wait(ofull, ph, abort, kCode)) break;
+      if (p.has_gate && !warp_wait(zfull, ph, abort, kCode)) break;
+      tc_fence_after();
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous output left o_buf
+      __syncwarp();
+      const float rl = 1.0f / l;
+      const uint32_t to = tmem + lane_base + C::kAccO;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld_32cols(to + cc * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = cc * 4 + ch;
+          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
+          const uint32_t addr = o_buf + a * G::kAtomTileBytes + row * G::kRowBytes +
+                                G::swz(row, cin) * 16;
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[ch * 8 + e]) * rl;
+          if (p.has_gate) {
+            const uint4 zw = ld_shared_v4(addr);
+            const uint32_t zz[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float z = (e & 1) ? bf16hi_to_f32(zz[e >> 1]) : bf16lo_to_f32(zz[e >> 1]);
+              x[e] *= 1.0f / (1.0f + expf(-z));
+            }
+          }
+          uint4 w;
+          w.x = pack_bf16x2(x[0], x[1]);
+          w.y = pack_bf16x2(x[2], x[3]);
+          w.z = pack_bf16x2(x[4], x[5]);
+          w.w = pack_bf16x2(x[6], x[7]);
+          st_shared_v4(addr, w);
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(ofree);
+        const int tok0 = qt * kTileTokens + q4 * 32;
+        if (tok0 < p.T)
+          for (int a = 0; a < G::kAtoms; ++a)
+            tma_store_5d(&tm_out, o_buf + a * G::kAtomTileBytes + q4 * 32 * G::kRowBytes,
+                         a * G::kAtomElems, h, tok0, f, b);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();  // the next unit's gate may land in o_buf
+        if (p.has_gate) mbar_arrive(zfree);
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace gla

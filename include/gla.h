@@ -148,6 +148,35 @@ int gla_forward_noalloc(const void* q, const void* k, const void* v,
 size_t gla_noalloc_scratch_bytes(void);
 
 /*
+ * gla_softmax_anchor -- the softmax anchor layer with attention sinks and a
+ * local window of frames (d = 128 only).
+ *
+ * The SANA-Video 2.0 pages interleave gated-softmax anchors with the linear
+ * layers (one in four); the SANA-WM pages add attention-sink tokens and local
+ * temporal windows to the softmax layers so that their memory and per-chunk
+ * latency stay constant over long rollouts.  No formula is printed; this
+ * library reads it, per (b, h), frames f of tokens_per_frame tokens, as:
+ *   keys of the queries of frame f = all tokens of frames
+ *       max(0, f - window_frames + 1) .. f, plus the first n_sink tokens of
+ *       the sequence that precede that window (never a later frame)
+ *   out_t = sigmoid(gate_z_t) * sum_s softmax_s(q_t . k_s / sqrt(d)) v_s
+ * Arguments: q, k, v, out bf16 [B, frames * tokens_per_frame, H, d]
+ * (16-byte aligned, out not overlapping the inputs); gate_z bf16 of the same
+ * shape or NULL (no gate); window_frames >= 1; n_sink >= 0.  No workspace.
+ * Returns the gla_forward codes (GLA_ERR_SHAPE for window_frames < 1 or
+ * n_sink < 0).
+ */
+int gla_softmax_anchor(const void* q, const void* k, const void* v, const void* gate_z,
+                       void* out, int B, int H, int frames, int tokens_per_frame, int d,
+                       int window_frames, int n_sink, cudaStream_t stream);
+
+/* gla_softmax_anchor with events[0] / events[1] recorded around the kernel. */
+int gla_softmax_anchor_timed(const void* q, const void* k, const void* v, const void* gate_z,
+                             void* out, int B, int H, int frames, int tokens_per_frame, int d,
+                             int window_frames, int n_sink, cudaStream_t stream,
+                             cudaEvent_t* events);
+
+/*
  * gla_forward_gdn -- the frame-wise gated delta-rule variant (Gated DeltaNet).
  *
  * The SANA-WM pages (paper analysis: abstract, method components) describe
@@ -300,7 +329,8 @@ const char* gla_error_string(int status);
  * kernel gave up a bounded wait (about one second) and returned early; its
  * output is then invalid.  Bit 0: state-increment kernel, bit 1: output
  * kernel, bit 2: forward scan, bit 3: reverse scan, bit 4: key/value
- * gradient kernel, bit 5: query gradient kernel, bit 6: delta-rule scan.
+ * gradient kernel, bit 5: query gradient kernel, bit 6: delta-rule scan,
+ * bit 7: softmax anchor kernel.
  * `code` is a host pointer.
  * Returns GLA_OK or GLA_ERR_LAUNCH.
  */

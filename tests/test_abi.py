@@ -160,6 +160,23 @@ def test_gdn_validation_before_any_cuda_call(lib):
                                      128, 1e-6, None, None) == gl.GLA_ERR_NULL
 
 
+def test_softmax_anchor_validation_before_any_cuda_call(lib):
+    import gated_linear_attention_frame_b200 as gl
+
+    def call(d=128, W=2, S=0, q=FAKE, out=FAKE, z=None, B=1):
+        return lib.gla_softmax_anchor(q, FAKE, FAKE, z, out, B, 1, 2, 16, d, W, S, None)
+
+    assert call(d=64) == gl.GLA_ERR_UNSUPPORTED_D
+    assert call(W=0) == gl.GLA_ERR_SHAPE
+    assert call(S=-1) == gl.GLA_ERR_SHAPE
+    assert call(q=None) == gl.GLA_ERR_NULL
+    assert call(out=FAKE + 8) == gl.GLA_ERR_ALIGN
+    assert call(z=FAKE + 8) == gl.GLA_ERR_ALIGN
+    assert call(B=0) == gl.GLA_OK
+    assert lib.gla_softmax_anchor_timed(FAKE, FAKE, FAKE, None, FAKE, 1, 1, 2, 16, 128, 2, 0, None,
+                                        None) == gl.GLA_ERR_NULL
+
+
 def test_timed_variant_requires_events(lib):
     import gated_linear_attention_frame_b200 as gl
 
