@@ -37,16 +37,32 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from workloads import (WORKLOADS, gdn_workload, make_beta, make_grads, make_inputs,  # noqa: E402
-                       make_state, rope_dims)
+                       make_state, rope_dims, seed_for)
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
+
+
+ANCHOR_WINDOW = 2  # softmax anchor: frames in the local window; sinks = the first frame
+
+
+def anchor_pairs(w, window: int, n_sink: int) -> int:
+    """(query, key) pairs of the softmax anchor layer over the whole batch."""
+    T = w.tokens_per_frame
+    per_bh = 0
+    for f in range(w.frames):
+        w_lo = max(0, f - window + 1) * T
+        per_bh += T * (min(n_sink, w_lo) + (f + 1) * T - w_lo)
+    return per_bh * w.B * w.H
 
 
 def metric_for(mode: str, variant: str) -> str:
     """The metric string of the timed path (the same for both arms)."""
     if mode == "backward":
         return METRIC_BWD
+    if variant == "softmax":
+        return ("softmax anchor tokens/s (sinks + %d-frame window, bf16, 720p shapes); "
+                "%% of roofline on 1 B200" % ANCHOR_WINDOW)
     if variant == "rope":
         return METRIC.replace("attention", "attention + 3D RoPE", 1)
     if variant == "gdn":
@@ -290,6 +306,11 @@ def oracle_head_call(w, variant: str):
             oracle.gla_rope_head(q, k, v, g, w.tokens_per_frame, w.grid_w, 0, rope_dims(w.d),
                                  10000.0, s, w.eps)
         return w, f, "3D-RoPE oracle"
+    if variant == "softmax":
+        def f(q, k, v, g, b, h, s):
+            oracle.softmax_anchor_head(q, k, v, w.tokens_per_frame, ANCHOR_WINDOW,
+                                       w.tokens_per_frame)
+        return w, f, "softmax-anchor oracle"
     if variant == "gdn":
         wg = gdn_workload(w)
         beta = make_beta(wg)
@@ -669,6 +690,91 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
     }
 
 
+def run_gpu_anchor(args, w, dist, rank, local_rank, world):
+    """One step = one gla_softmax_anchor call (sinks = the first frame, a
+    window of ANCHOR_WINDOW frames, sigmoid output gate) over one batch."""
+    import gated_linear_attention_frame_b200 as gla
+
+    if w.d != 128:
+        raise SystemExit("the softmax anchor kernel is built for d = 128")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    q, k, v, _ = make_inputs(w, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed_for(w) + 17)
+    z = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    T, W = w.tokens_per_frame, ANCHOR_WINDOW
+    pairs = anchor_pairs(w, W, T)
+    flops = 4 * w.d * pairs                         # Q K^T and P V
+    nbytes = w.B * w.tokens * w.H * w.d * 2 * 5     # q, k, v, z read; out written
+
+    def step(events=None):
+        a = (q, k, v, z, out, w.B, w.H, w.frames, T, w.d, W, T)
+        if events is None:
+            gla.gla_softmax_anchor(*a, stream)
+        else:
+            gla.gla_softmax_anchor_timed(*a, stream, events)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_device_fault(stream) == 0
+    K = args.steps
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with clocks:
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_step = reduce_max(t0.elapsed_time(t1), dist, dev) / K
+    fault = gla.gla_device_fault(stream)
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": "gla_softmax_anchor_kernel", "achieved": round(achieved, 1),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+            "algorithmic_flops_per_launch": flops,
+            "flops_note": "4 d per (query, key) pair; the two-pass kernel issues 6 d",
+            "peak_source": peaks["source"] + " (bf16_tflops)"}
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    layer = {"algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+             "roofline_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_step, 4)}
+    e2e = None
+    if not args.no_e2e:
+        host_in = [x.cpu().pin_memory() for x in (q, k, v, z)]
+
+        def call(bi, bo):
+            gla.gla_softmax_anchor(bi[0], bi[1], bi[2], bi[3], bo[0], w.B, w.H, w.frames, T,
+                                   w.d, W, T, stream)
+
+        e2e = e2e_pipelined(dev, stream, dist, world, host_in, [out], call,
+                            max(2, min(K, args.e2e_steps)), w.total_tokens)
+    return {
+        "metric": metric_for("forward", "softmax"), "value": round(world * w.total_tokens /
+                                                                 (ms_step * 1e-3), 1),
+        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.frames,
+                   "tokens_per_frame": T, "window_frames": W, "n_sink": T, "gate": True,
+                   "tokens_per_step_per_gpu": w.total_tokens,
+                   "l2": "inputs larger than L2; no flush",
+                   "parallelism": "dp%d (independent sequences per GPU)" % world},
+        "roofline": roof, "layer_roofline": layer, "gpu_launches": K, "e2e": e2e,
+        "clocks": clocks.summary(), "device_fault": fault,
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+
+
 def time_oracle_backward(w, budget_s: float) -> dict:
     """Time the fp64 gradient oracle on (b, h) slices until `budget_s` of CPU
     work; tokens/s counts full-layer tokens (all heads)."""
@@ -755,9 +861,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
                     help="time gla_forward (the layer metric) or gla_backward")
-    ap.add_argument("--variant", choices=["plain", "rope", "gdn"], default="plain",
-                    help="forward only: the plain layer, gla_forward_rope (3D RoPE) or "
-                         "gla_forward_gdn (frame-wise gated delta rule)")
+    ap.add_argument("--variant", choices=["plain", "rope", "gdn", "softmax"], default="plain",
+                    help="forward only: the plain layer, gla_forward_rope (3D RoPE), "
+                         "gla_forward_gdn (frame-wise gated delta rule) or gla_softmax_anchor")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=0,
                     help="override the workload's frame count (small profiling cases)")
@@ -782,6 +888,8 @@ def main(argv=None):
     try:
         if args.mode == "backward":
             res = run_gpu_backward(args, w, dist, rank, local_rank, world)
+        elif args.variant == "softmax":
+            res = run_gpu_anchor(args, w, dist, rank, local_rank, world)
         else:
             res = run_gpu(args, w, dist, rank, local_rank, world)
         if rank == 0 and world == 1 and args.cpu_budget > 0:
