@@ -1,11 +1,12 @@
 """Benchmark of the gated linear attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
-                    [--mode forward|backward]
+                    [--mode forward|backward] [--variant plain|rope|gdn|softmax]
 
 One step = one gla_forward call (increment -> gated scan -> output kernels)
 over one batch of the workload, inputs resident in HBM; with --mode backward,
-one gla_backward call (d = 128) instead.  With N > 1 (torchrun,
+one gla_backward call (d = 128) instead; with --variant, one call of
+gla_forward_rope, gla_forward_gdn or gla_softmax_anchor.  With N > 1 (torchrun,
 one process per GPU) every rank runs its own independent copy of the workload
 (heads and sequences are independent: weak scaling, no data-path
 collective); the timed region is bracketed by a barrier and a device
@@ -37,7 +38,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from workloads import (WORKLOADS, gdn_workload, make_beta, make_grads, make_inputs,  # noqa: E402
-                       make_state, rope_dims, seed_for)
+                       make_state, rope_dims, anchor_workload, make_anchor_gate)
 
 METRIC = "gated linear attention tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
 METRIC_BWD = "gated linear attention backward tokens/s (bf16, 720p shapes); % of roofline on 1 B200"
@@ -68,6 +69,8 @@ def metric_for(mode: str, variant: str) -> str:
     if variant == "gdn":
         return METRIC.replace("gated linear attention", "frame-wise gated delta rule", 1)
     return METRIC
+
+
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "720p-5s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
@@ -307,10 +310,13 @@ def oracle_head_call(w, variant: str):
                                  10000.0, s, w.eps)
         return w, f, "3D-RoPE oracle"
     if variant == "softmax":
+        wa = anchor_workload(w)
+        z = make_anchor_gate(wa)
+
         def f(q, k, v, g, b, h, s):
-            oracle.softmax_anchor_head(q, k, v, w.tokens_per_frame, ANCHOR_WINDOW,
-                                       w.tokens_per_frame)
-        return w, f, "softmax-anchor oracle"
+            oracle.softmax_anchor_head(q, k, v, wa.tokens_per_frame, ANCHOR_WINDOW,
+                                       wa.tokens_per_frame, z[b, :, h])
+        return wa, f, "softmax-anchor oracle"
     if variant == "gdn":
         wg = gdn_workload(w)
         beta = make_beta(wg)
@@ -697,14 +703,13 @@ def run_gpu_anchor(args, w, dist, rank, local_rank, world):
 
     if w.d != 128:
         raise SystemExit("the softmax anchor kernel is built for d = 128")
+    w = anchor_workload(w)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peaks = load_peaks()
     q, k, v, _ = make_inputs(w, device=dev)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(seed_for(w) + 17)
-    z = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+    z = make_anchor_gate(w, device=dev)
     out = torch.empty_like(q)
     T, W = w.tokens_per_frame, ANCHOR_WINDOW
     pairs = anchor_pairs(w, W, T)

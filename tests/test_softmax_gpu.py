@@ -4,8 +4,8 @@ Tolerance as the linear layers: max|gpu - oracle| <= 1e-2 max|oracle| and
 rel-L2 <= 5e-3.  Small shapes cover ragged key and query tiles, sinks shorter
 than, equal to and longer than a frame, windows of 1 to all frames, the
 output gate, several units per CTA; the 720p-5s shape runs at full size (a
-window of 2 frames, the first frame as sinks) and is compared on sampled
-(batch, head) slices.
+window of 2 frames, the first frame as sinks, the output gate: the benchmark's
+launch) and is compared on sampled (batch, head) slices.
 """
 
 import numpy as np
@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from workloads import WORKLOADS, make_inputs
+from workloads import WORKLOADS, anchor_workload, make_anchor_gate, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -92,13 +92,14 @@ def test_small_shapes_full_compare(B, H, F, T, W, S, gate):
 def test_full_size_720p_5s_sampled_heads():
     import gated_linear_attention_frame_b200 as gla
 
-    w = WORKLOADS["720p-5s"]
+    w = anchor_workload(WORKLOADS["720p-5s"])
     dev = torch.device("cuda")
     q, k, v, _ = make_inputs(w, device=dev)
+    z = make_anchor_gate(w, device=dev)
     T = w.tokens_per_frame
-    out = gla.softmax_anchor(q, k, v, w.frames, 2, T)
+    out = gla.softmax_anchor(q, k, v, w.frames, 2, T, z)
     torch.cuda.synchronize()
     for b, h in [(0, 0), (1, 17)]:
         sl = lambda x: x[b, :, h].float().cpu().numpy()  # noqa: E731
-        ref = oracle.softmax_anchor_head(sl(q), sl(k), sl(v), T, 2, T)
+        ref = oracle.softmax_anchor_head(sl(q), sl(k), sl(v), T, 2, T, sl(z))
         assert_close(sl(out), ref, "out[b=%d,h=%d]" % (b, h))

@@ -27,7 +27,7 @@ from dataclasses import dataclass, replace
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_state", "make_grads", "make_beta",
-           "gdn_workload", "rope_dims", "seed_for"]
+           "gdn_workload", "rope_dims", "seed_for", "anchor_workload", "make_anchor_gate"]
 
 BASE_SEED = 20261202
 
@@ -164,3 +164,20 @@ def make_beta(w: Workload, device="cpu", seed: int | None = None):
     gen = torch.Generator(device=dev)
     gen.manual_seed((seed_for(w) if seed is None else seed) + 13)
     return _normal((w.B, w.frames, w.H), gen, dev)
+
+
+def anchor_workload(w: Workload) -> Workload:
+    """The softmax anchor layer's inputs for a workload: the same shapes and
+    seeds with q, k ~ N(0, 1) unscaled, so that the scores q . k / sqrt(d) are
+    ~ N(0, 1)."""
+    return w.with_(k_scaled=False, k_div_tokens=False)
+
+
+def make_anchor_gate(w: Workload, device="cpu", seed: int | None = None):
+    """Output-gate logits z of the softmax anchor layer: bf16 [B, tokens, H, d]
+    ~ N(0, 1) rounded to nearest even, from a generator seeded with
+    seed_for(w) + 17 (or `seed`)."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed((seed_for(w) if seed is None else seed) + 17)
+    return _normal((w.B, w.tokens, w.H, w.d), gen, dev).to(torch.bfloat16)
