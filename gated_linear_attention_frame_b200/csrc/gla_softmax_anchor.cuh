@@ -15,9 +15,14 @@
 //   pass 1  S = Q K^T into TMEM (double-buffered); the softmax warps keep the
 //           running row maximum m (invalid key rows masked to -inf);
 //   pass 2  S = Q K^T again; the softmax warps write P = exp(S - m) in bf16 to
-//           shared memory and sum l = sum P; O += P V accumulates in TMEM.
+//           shared memory (two buffers) and sum l = sum P; O += P V
+//           accumulates in TMEM.  The MMA issuer runs one tile ahead: S of
+//           tile j+1 is issued before P V of tile j, so the tensor core
+//           computes the next scores while the softmax warps exponentiate.
 // Two passes cost one more Q K^T per tile but need no rescaling of the TMEM
 // accumulator when the maximum grows.  The epilogue writes sigmoid(z) O / l.
+// Ring order of the key/value tiles: pass 1 K0 K1 ..; pass 2 K0 K1 V0 K2 V1 ..
+// K(n-1) V(n-2) V(n-1), the order in which the MMA issuer consumes them.
 //   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
 //   PV: A = P [M = 128 queries, K = 128 keys] K-major, B = V tile [N = d] MN-major
 // Warp roles: 0-3 softmax / epilogue (thread = query row), 4 TMA, 5 MMA.
@@ -96,8 +101,9 @@ struct AnchorCfg {
   static constexpr int kThreads = 192;
   static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128)
   static constexpr int kAccO = 256;
-  static constexpr int kBarCount = 2 * kStages + 14;
-  static constexpr int kSmemBytes = 1024 + (3 + kStages) * kTileBytes + kBarCount * 8 + 16;
+  static constexpr int kBarCount = 2 * kStages + 16;
+  // Q, P x 2, gate / output, ring
+  static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -119,10 +125,10 @@ __global__ void __launch_bounds__(192, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t q_buf = sbase;
-  const uint32_t p_buf = sbase + C::kTileBytes;
-  const uint32_t o_buf = sbase + 2 * C::kTileBytes;  // gate in, output out
-  auto ring = [&](int s) { return sbase + (3 + s) * C::kTileBytes; };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (3 + S) * C::kTileBytes);
+  auto p_buf = [&](int i) { return sbase + (1 + i) * C::kTileBytes; };
+  const uint32_t o_buf = sbase + 3 * C::kTileBytes;  // gate in, output out
+  auto ring = [&](int s) { return sbase + (4 + s) * C::kTileBytes; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (4 + S) * C::kTileBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto rfull = [&](int s) { return bar0 + 8u * s; };
   auto rempty = [&](int s) { return bar0 + 8u * (S + s); };
@@ -130,13 +136,13 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t qempty = bar0 + 8u * (2 * S + 1);
   auto sfull = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
   auto sfree = [&](int b) { return bar0 + 8u * (2 * S + 4 + b); };
-  const uint32_t pfull = bar0 + 8u * (2 * S + 6);
-  const uint32_t pfree = bar0 + 8u * (2 * S + 7);
-  const uint32_t ofull = bar0 + 8u * (2 * S + 8);
-  const uint32_t ofree = bar0 + 8u * (2 * S + 9);
-  const uint32_t zfull = bar0 + 8u * (2 * S + 10);
-  const uint32_t zfree = bar0 + 8u * (2 * S + 11);
-  const uint32_t done_bar = bar0 + 8u * (2 * S + 12);
+  auto pfull = [&](int i) { return bar0 + 8u * (2 * S + 6 + i); };
+  auto pfree = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
+  const uint32_t ofull = bar0 + 8u * (2 * S + 10);
+  const uint32_t ofree = bar0 + 8u * (2 * S + 11);
+  const uint32_t zfull = bar0 + 8u * (2 * S + 12);
+  const uint32_t zfree = bar0 + 8u * (2 * S + 13);
+  const uint32_t done_bar = bar0 + 8u * (2 * S + 14);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -154,9 +160,9 @@ __global__ void __launch_bounds__(192, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(sfull(b), 1);
       mbar_init(sfree(b), 4);
+      mbar_init(pfull(b), 4);
+      mbar_init(pfree(b), 1);
     }
-    mbar_init(pfull, 4);
-    mbar_init(pfree, 1);
     mbar_init(ofull, 1);
     mbar_init(ofree, 4);
     mbar_init(zfull, 1);
@@ -206,26 +212,29 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_5d(o_buf + a * G::kAtomTileBytes, &tm_z, zfull, a * G::kAtomElems, h,
                         qt * kTileTokens, f, b);
         }
-        for (int pass = 0; pass < 2 && ok; ++pass) {
-          KeyTiles kt;
-          kt.init(p.T, f, p.window, p.n_sink);
-          for (; !kt.done; kt.advance()) {
-            for (int which = 0; which < pass + 1; ++which) {  // pass 2: K then V
-              const int s = static_cast<int>(n % S);
-              if (!mbar_wait(rempty(s), static_cast<uint32_t>(((n / S) & 1) ^ 1), abort, kCode)) {
-                ok = false;
-                break;
-              }
-              mbar_arrive_expect_tx(rfull(s), G::kTileBytes);
-              const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
-              for (int a = 0; a < G::kAtoms; ++a)
-                tma_load_5d(ring(s) + a * G::kAtomTileBytes, tm, rfull(s), a * G::kAtomElems, h,
-                            kt.t0, kt.fr, b);
-              ++n;
-            }
-            if (!ok) break;
-          }
+        // one ring tile: K or V rows [t0, t0 + 128) of frame fr
+        auto load = [&](const CUtensorMap* tm, int fr, int t0) {
+          const int s = static_cast<int>(n % S);
+          if (!mbar_wait(rempty(s), static_cast<uint32_t>(((n / S) & 1) ^ 1), abort, kCode))
+            return false;
+          mbar_arrive_expect_tx(rfull(s), G::kTileBytes);
+          for (int a = 0; a < G::kAtoms; ++a)
+            tma_load_5d(ring(s) + a * G::kAtomTileBytes, tm, rfull(s), a * G::kAtomElems, h, t0,
+                        fr, b);
+          ++n;
+          return true;
+        };
+        KeyTiles kt;
+        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance())
+          ok = load(&tm_k, kt.fr, kt.t0);
+        int pfr = -1, pt0 = 0;  // the previous tile, whose V follows this tile's K
+        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance()) {
+          ok = load(&tm_k, kt.fr, kt.t0);
+          if (ok && pfr >= 0) ok = load(&tm_v, pfr, pt0);
+          pfr = kt.fr;
+          pt0 = kt.t0;
         }
+        if (ok && pfr >= 0) ok = load(&tm_v, pfr, pt0);
       }
       for (int64_t i = (n > S ? n - S : 0); i < n; ++i)
         mbar_wait_drain(rfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
@@ -243,61 +252,64 @@ __global__ void __launch_bounds__(192, 1)
         coords(unit, b, f, h, qt);
         const uint32_t ph = static_cast<uint32_t>(it & 1);
         if (!mbar_wait(qfull, ph, abort, kCode)) break;
-        bool first_pv = true;
-        for (int pass = 0; pass < 2 && ok; ++pass) {
-          KeyTiles kt;
-          kt.init(p.T, f, p.window, p.n_sink);
-          for (; !kt.done; kt.advance()) {
-            // S = Q K^T into buffer ns % 2
-            const int sb = static_cast<int>(ns & 1);
-            const int s = static_cast<int>(n % S);
-            if (!mbar_wait(sfree(sb), static_cast<uint32_t>(((ns >> 1) & 1) ^ 1), abort, kCode) ||
-                !mbar_wait(rfull(s), static_cast<uint32_t>((n / S) & 1), abort, kCode)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+        // S = Q K^T of the next ring tile into S buffer ns % 2
+        auto issue_s = [&]() {
+          const int sb = static_cast<int>(ns & 1);
+          const int s = static_cast<int>(n % S);
+          if (!mbar_wait(sfree(sb), static_cast<uint32_t>(((ns >> 1) & 1) ^ 1), abort, kCode) ||
+              !mbar_wait(rfull(s), static_cast<uint32_t>((n / S) & 1), abort, kCode))
+            return false;
+          tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int a = kk / KPA, w = kk % KPA;
-              const uint64_t ad = smem_desc(q_buf + a * G::kAtomTileBytes + w * 32, 16,
-                                            G::kGroupBytes, G::kLayout);
-              const uint64_t bd = smem_desc(ring(s) + a * G::kAtomTileBytes + w * 32, 16,
-                                            G::kGroupBytes, G::kLayout);
-              mma_bf16(tmem + sb * kTileTokens, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(sfull(sb));
-            mma_commit(rempty(s));
-            ++n;
-            ++ns;
-            if (pass == 1) {
-              // O += P V once the softmax warps wrote P of this tile
-              const int sv = static_cast<int>(n % S);
-              if (!mbar_wait(pfull, static_cast<uint32_t>(np & 1), abort, kCode) ||
-                  !mbar_wait(rfull(sv), static_cast<uint32_t>((n / S) & 1), abort, kCode)) {
-                ok = false;
-                break;
-              }
-              if (first_pv && !mbar_wait(ofree, ph ^ 1u, abort, kCode)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int a = kk / KPA, w = kk % KPA;
+            const uint64_t ad = smem_desc(q_buf + a * G::kAtomTileBytes + w * 32, 16,
+                                          G::kGroupBytes, G::kLayout);
+            const uint64_t bd = smem_desc(ring(s) + a * G::kAtomTileBytes + w * 32, 16,
+                                          G::kGroupBytes, G::kLayout);
+            mma_bf16(tmem + sb * kTileTokens, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(sfull(sb));
+          mma_commit(rempty(s));
+          ++n;
+          ++ns;
+          return true;
+        };
+        // O += P V with P from buffer np % 2 and V the next ring tile
+        auto issue_pv = [&](bool first) {
+          const int pb = static_cast<int>(np & 1);
+          const int sv = static_cast<int>(n % S);
+          if (!mbar_wait(pfull(pb), static_cast<uint32_t>((np >> 1) & 1), abort, kCode) ||
+              !mbar_wait(rfull(sv), static_cast<uint32_t>((n / S) & 1), abort, kCode))
+            return false;
+          if (first && !mbar_wait(ofree, ph ^ 1u, abort, kCode)) return false;
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-                const int a = kk / KPA, w = kk % KPA;
-                const uint64_t ad = smem_desc(p_buf + a * G::kAtomTileBytes + w * 32, 16,
-                                              G::kGroupBytes, G::kLayout);
-                const uint64_t bd = smem_desc(ring(sv) + kk * 2 * G::kGroupBytes,
-                                              G::kAtomTileBytes, G::kGroupBytes, G::kLayout);
-                mma_bf16(tmem + C::kAccO, ad, bd, idesc_o, (first_pv && kk == 0) ? 0u : 1u);
-              }
-              first_pv = false;
-              mma_commit(pfree);
-              mma_commit(rempty(sv));
-              ++n;
-              ++np;
-            }
+          for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+            const int a = kk / KPA, w = kk % KPA;
+            const uint64_t ad = smem_desc(p_buf(pb) + a * G::kAtomTileBytes + w * 32, 16,
+                                          G::kGroupBytes, G::kLayout);
+            const uint64_t bd = smem_desc(ring(sv) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
+                                          G::kGroupBytes, G::kLayout);
+            mma_bf16(tmem + C::kAccO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(pfree(pb));
+          mma_commit(rempty(sv));
+          ++n;
+          ++np;
+          return true;
+        };
+        KeyTiles kt;
+        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance()) ok = issue_s();
+        kt.init(p.T, f, p.window, p.n_sink);
+        if (ok && !kt.done) {
+          ok = issue_s();
+          for (bool first = true; ok; first = false) {
+            kt.advance();
+            const bool more = !kt.done;
+            if (more) ok = issue_s();
+            if (ok) ok = issue_pv(first);
+            if (!more) break;
           }
         }
         if (!ok) break;
@@ -330,43 +342,54 @@ __global__ void __launch_bounds__(192, 1)
           }
           tc_fence_after();
           const uint32_t ts = tmem + lane_base + sb * kTileTokens;
+          const bool full = kt.valid == kTileTokens;  // warp-uniform
           if (pass == 0) {
-            float mx = m;
+            float mx[4] = {m, m, m, m};
 #pragma unroll
             for (int cc = 0; cc < kTileTokens / 32; ++cc) {
               uint32_t r[32];
               tmem_ld_32cols(ts + cc * 32, r);
               tmem_wait_ld();
+              if (full) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (cc * 32 + e < kt.valid) mx = fmaxf(mx, __uint_as_float(r[e]));
+                for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  mx[e & 3] = fmaxf(mx[e & 3],
+                                    cc * 32 + e < kt.valid ? __uint_as_float(r[e]) : -INFINITY);
+              }
             }
-            m = mx;
+            m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sfree(sb));
           } else {
-            // P = exp2((S - m) * scale log2 e) for valid keys, 0 past them
-            if (!warp_wait(pfree, static_cast<uint32_t>((np & 1) ^ 1), abort, kCode)) {
+            // P = 2^((S - m) scale log2 e); keys past the tile's end get S = -inf, P = 0
+            const int pb = static_cast<int>(np & 1);
+            if (!warp_wait(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort, kCode)) {
               ok = false;
               break;
             }
             const float ms = m * p.scale_log2;
+            const uint32_t pbase = p_buf(pb) + row * G::kRowBytes;
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int cc = 0; cc < kTileTokens / 32; ++cc) {
               uint32_t r[32];
               tmem_ld_32cols(ts + cc * 32, r);
               tmem_wait_ld();
+              if (!full) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (cc * 32 + e >= kt.valid) r[e] = __float_as_uint(-INFINITY);
+              }
 #pragma unroll
               for (int ch = 0; ch < 4; ++ch) {
                 float x[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                  const int col = cc * 32 + ch * 8 + e;
-                  x[e] = col < kt.valid ? exp2f(fmaf(__uint_as_float(r[ch * 8 + e]),
-                                                     p.scale_log2, -ms))
-                                        : 0.f;
+                  x[e] = ex2_approx(fmaf(__uint_as_float(r[ch * 8 + e]), p.scale_log2, -ms));
                   ls[e & 3] += x[e];
                 }
                 uint4 w;
@@ -376,9 +399,7 @@ __global__ void __launch_bounds__(192, 1)
                 w.w = pack_bf16x2(x[6], x[7]);
                 const int chunk = cc * 4 + ch;
                 const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
-                st_shared_v4(p_buf + a * G::kAtomTileBytes + row * G::kRowBytes +
-                                 G::swz(row, cin) * 16,
-                             w);
+                st_shared_v4(pbase + a * G::kAtomTileBytes + G::swz(row, cin) * 16, w);
               }
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
@@ -387,7 +408,7 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) {
               mbar_arrive(sfree(sb));
-              mbar_arrive(pfull);
+              mbar_arrive(pfull(pb));
             }
             ++np;
           }
