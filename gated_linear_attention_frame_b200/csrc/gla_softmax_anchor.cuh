@@ -25,7 +25,10 @@
 // K(n-1) V(n-2) V(n-1), the order in which the MMA issuer consumes them.
 //   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
 //   PV: A = P [M = 128 queries, K = 128 keys] K-major, B = V tile [N = d] MN-major
-// Warp roles: 0-3 softmax / epilogue (thread = query row), 4 TMA, 5 MMA.
+// Warp roles: 0-7 softmax / epilogue, 8 TMA, 9 MMA.  Softmax warp w owns the
+// query rows 32 (w % 4) .. + 31 (its TMEM lane quarter) and the key / output
+// columns 64 (w / 4) .. + 63 of every tile; the two warps of a row quarter
+// exchange their partial row maximum and row sum through spare TMEM columns.
 #pragma once
 
 #include "gla_common.cuh"
@@ -98,9 +101,11 @@ struct AnchorCfg {
   static_assert(D == 128, "the softmax anchor kernel is built for d = 128");
   static constexpr int kStages = 3;                 // K / V tile ring
   static constexpr int kTileBytes = G::kTileBytes;  // 32 KB
-  static constexpr int kThreads = 192;
-  static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128)
+  static constexpr int kThreads = 320;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128) + exchange
   static constexpr int kAccO = 256;
+  static constexpr int kXchg = 384;                 // m of half c at +c, l of half c at +2+c
   static constexpr int kBarCount = 2 * kStages + 16;
   // Q, P x 2, gate / output, ring
   static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
@@ -108,7 +113,7 @@ struct AnchorCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gla_softmax_anchor_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v,
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t zfull = bar0 + 8u * (2 * S + 12);
   const uint32_t zfree = bar0 + 8u * (2 * S + 13);
   const uint32_t done_bar = bar0 + 8u * (2 * S + 14);
+  const uint32_t xbar = bar0 + 8u * (2 * S + 15);  // row max / row sum exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -159,15 +165,16 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(qempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(sfull(b), 1);
-      mbar_init(sfree(b), 4);
-      mbar_init(pfull(b), 4);
+      mbar_init(sfree(b), C::kSoftmaxWarps);
+      mbar_init(pfull(b), C::kSoftmaxWarps);
       mbar_init(pfree(b), 1);
     }
     mbar_init(ofull, 1);
-    mbar_init(ofree, 4);
+    mbar_init(ofree, C::kSoftmaxWarps);
     mbar_init(zfull, 1);
-    mbar_init(zfree, 4);
+    mbar_init(zfree, C::kSoftmaxWarps);
     mbar_init(done_bar, 1);
+    mbar_init(xbar, C::kSoftmaxWarps);
     *abort = 0;
     fence_mbar_init();
   }
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(192, 1)
     unit_coords(u, p.H, p.F, b, f, h);
   };
 
-  if (warp == 4) {
+  if (warp == C::kSoftmaxWarps) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int64_t i = (n > S ? n - S : 0); i < n; ++i)
         mbar_wait_drain(rfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
     }
-  } else if (warp == 5) {
+  } else if (warp == C::kSoftmaxWarps + 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileTokens, false, false);
@@ -321,10 +328,32 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // -------------------------------------------------- softmax and epilogue
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;  // query within the tile
+    const int q4 = warp & 3;          // TMEM lane quarter: query rows 32 q4 ..
+    const int hc = warp >> 2;         // column half: keys / outputs 64 hc ..
+    const int row = q4 * 32 + lane;   // query within the tile
+    const int c0 = hc * 64;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t tx = tmem + lane_base + C::kXchg;
     int64_t ns = 0, np = 0, it = 0;
+    // the partner warp's partial value through TMEM column kXchg + slot;
+    // .ok (warp-uniform) is false if the wait gave up
+    struct Xchg {
+      float v;
+      bool ok;
+    };
+    auto exchange = [&](float mine, int slot, uint32_t parity) {
+      tmem_st_1col(tx + slot + hc, __float_as_uint(mine));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (!warp_wait(xbar, parity, abort, kCode)) return Xchg{0.f, false};
+      tc_fence_after();
+      uint32_t v;
+      tmem_ld_1col(tx + slot + (hc ^ 1), v);
+      tmem_wait_ld();
+      return Xchg{__uint_as_float(v), true};
+    };
     for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x, ++it) {
       int b, f, h, qt;
       coords(unit, b, f, h, qt);
@@ -341,130 +370,126 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t ts = tmem + lane_base + sb * kTileTokens;
-          const bool full = kt.valid == kTileTokens;  // warp-uniform
+          uint32_t ra[32], rb[32];  // columns c0 .. c0 + 31, c0 + 32 .. c0 + 63
+          const uint32_t ts = tmem + lane_base + sb * kTileTokens + c0;
+          tmem_ld_32cols(ts, ra);
+          tmem_ld_32cols(ts + 32, rb);
+          tmem_wait_ld();
+          if (kt.valid < c0 + 64) {  // keys past the tile's end: S = -inf
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (c0 + e >= kt.valid) ra[e] = __float_as_uint(-INFINITY);
+              if (c0 + 32 + e >= kt.valid) rb[e] = __float_as_uint(-INFINITY);
+            }
+          }
           if (pass == 0) {
             float mx[4] = {m, m, m, m};
 #pragma unroll
-            for (int cc = 0; cc < kTileTokens / 32; ++cc) {
-              uint32_t r[32];
-              tmem_ld_32cols(ts + cc * 32, r);
-              tmem_wait_ld();
-              if (full) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
-              } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  mx[e & 3] = fmaxf(mx[e & 3],
-                                    cc * 32 + e < kt.valid ? __uint_as_float(r[e]) : -INFINITY);
-              }
+            for (int e = 0; e < 32; ++e) {
+              mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(ra[e]));
+              mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(rb[e]));
             }
             m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sfree(sb));
           } else {
-            // P = 2^((S - m) scale log2 e); keys past the tile's end get S = -inf, P = 0
+            // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sfree(sb));  // S read into registers
             const int pb = static_cast<int>(np & 1);
             if (!warp_wait(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort, kCode)) {
               ok = false;
               break;
             }
             const float ms = m * p.scale_log2;
-            const uint32_t pbase = p_buf(pb) + row * G::kRowBytes;
+            const uint32_t pbase = p_buf(pb) + hc * G::kAtomTileBytes + row * G::kRowBytes;
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int cc = 0; cc < kTileTokens / 32; ++cc) {
-              uint32_t r[32];
-              tmem_ld_32cols(ts + cc * 32, r);
-              tmem_wait_ld();
-              if (!full) {
+            for (int ch = 0; ch < 8; ++ch) {
+              float x[8];
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (cc * 32 + e >= kt.valid) r[e] = __float_as_uint(-INFINITY);
+              for (int e = 0; e < 8; ++e) {
+                const uint32_t sv = ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e];
+                x[e] = ex2_approx(fmaf(__uint_as_float(sv), p.scale_log2, -ms));
+                ls[e & 3] += x[e];
               }
-#pragma unroll
-              for (int ch = 0; ch < 4; ++ch) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  x[e] = ex2_approx(fmaf(__uint_as_float(r[ch * 8 + e]), p.scale_log2, -ms));
-                  ls[e & 3] += x[e];
-                }
-                uint4 w;
-                w.x = pack_bf16x2(x[0], x[1]);
-                w.y = pack_bf16x2(x[2], x[3]);
-                w.z = pack_bf16x2(x[4], x[5]);
-                w.w = pack_bf16x2(x[6], x[7]);
-                const int chunk = cc * 4 + ch;
-                const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
-                st_shared_v4(pbase + a * G::kAtomTileBytes + G::swz(row, cin) * 16, w);
-              }
+              uint4 w;
+              w.x = pack_bf16x2(x[0], x[1]);
+              w.y = pack_bf16x2(x[2], x[3]);
+              w.z = pack_bf16x2(x[4], x[5]);
+              w.w = pack_bf16x2(x[6], x[7]);
+              st_shared_v4(pbase + G::swz(row, ch) * 16, w);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             fence_proxy_async_smem();
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-              mbar_arrive(sfree(sb));
-              mbar_arrive(pfull(pb));
-            }
+            if (lane == 0) mbar_arrive(pfull(pb));
             ++np;
           }
           ++ns;
         }
+        if (!ok) break;
+        if (pass == 0) {  // the row maximum over both column halves
+          const Xchg mo = exchange(m, 0, 0u);
+          if (!mo.ok) {
+            ok = false;
+            break;
+          }
+          m = fmaxf(m, mo.v);
+        }
       }
       if (!ok) break;
-      // ---- epilogue: out = sigmoid(z) * O / l
+      const Xchg lo = exchange(l, 2, 1u);
+      if (!lo.ok) break;
+      l += lo.v;
+      // ---- epilogue: out = sigmoid(z) * O / l, columns [c0, c0 + 64)
       if (!warp_wait(ofull, ph, abort, kCode)) break;
       if (p.has_gate && !warp_wait(zfull, ph, abort, kCode)) break;
       tc_fence_after();
       if (lane == 0) bulk_wait_group_read<0>();  // the previous output left o_buf
       __syncwarp();
       const float rl = 1.0f / l;
-      const uint32_t to = tmem + lane_base + C::kAccO;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32cols(to + cc * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = cc * 4 + ch;
-          const int a = chunk / (G::kAtomElems / 8), cin = chunk % (G::kAtomElems / 8);
-          const uint32_t addr = o_buf + a * G::kAtomTileBytes + row * G::kRowBytes +
-                                G::swz(row, cin) * 16;
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[ch * 8 + e]) * rl;
-          if (p.has_gate) {
-            const uint4 zw = ld_shared_v4(addr);
-            const uint32_t zz[4] = {zw.x, zw.y, zw.z, zw.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float z = (e & 1) ? bf16hi_to_f32(zz[e >> 1]) : bf16lo_to_f32(zz[e >> 1]);
-              x[e] *= 1.0f / (1.0f + expf(-z));
-            }
-          }
-          uint4 w;
-          w.x = pack_bf16x2(x[0], x[1]);
-          w.y = pack_bf16x2(x[2], x[3]);
-          w.z = pack_bf16x2(x[4], x[5]);
-          w.w = pack_bf16x2(x[6], x[7]);
-          st_shared_v4(addr, w);
-        }
-      }
+      uint32_t ra[32], rb[32];
+      const uint32_t to = tmem + lane_base + C::kAccO + c0;
+      tmem_ld_32cols(to, ra);
+      tmem_ld_32cols(to + 32, rb);
+      tmem_wait_ld();
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ofree);  // O read into registers
+      const uint32_t obase = o_buf + hc * G::kAtomTileBytes + row * G::kRowBytes;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t addr = obase + G::swz(row, ch) * 16;
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          x[e] = __uint_as_float(ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e]) * rl;
+        if (p.has_gate) {
+          const uint4 zw = ld_shared_v4(addr);
+          const uint32_t zz[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float z = (e & 1) ? bf16hi_to_f32(zz[e >> 1]) : bf16lo_to_f32(zz[e >> 1]);
+            x[e] *= 1.0f / (1.0f + expf(-z));
+          }
+        }
+        uint4 w;
+        w.x = pack_bf16x2(x[0], x[1]);
+        w.y = pack_bf16x2(x[2], x[3]);
+        w.z = pack_bf16x2(x[4], x[5]);
+        w.w = pack_bf16x2(x[6], x[7]);
+        st_shared_v4(addr, w);
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(ofree);
         const int tok0 = qt * kTileTokens + q4 * 32;
         if (tok0 < p.T)
-          for (int a = 0; a < G::kAtoms; ++a)
-            tma_store_5d(&tm_out, o_buf + a * G::kAtomTileBytes + q4 * 32 * G::kRowBytes,
-                         a * G::kAtomElems, h, tok0, f, b);
+          tma_store_5d(&tm_out, o_buf + hc * G::kAtomTileBytes + q4 * 32 * G::kRowBytes,
+                       hc * G::kAtomElems, h, tok0, f, b);
         bulk_commit_group();
         bulk_wait_group_read<0>();  // the next unit's gate may land in o_buf
         if (p.has_gate) mbar_arrive(zfree);
