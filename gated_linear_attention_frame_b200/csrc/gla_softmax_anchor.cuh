@@ -25,7 +25,13 @@
 // K(n-1) V(n-2) V(n-1), the order in which the MMA issuer consumes them.
 //   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
 //   PV: A = P [M = 128 queries, K = 128 keys] K-major, B = V tile [N = d] MN-major
-// Warp roles: 0-7 softmax / epilogue, 8 TMA, 9 MMA.  Softmax warp w owns the
+// Warp roles: 0-7 softmax / epilogue, 8 TMA, 9 and 10 MMA.  A tcgen05.mma
+// issue returns only about when the tensor core takes the instruction, so a
+// lone issuing thread leaves the tensor core idle while it waits on barriers
+// and commits; two issuers overlap that bookkeeping with each other's MMAs.
+// Pass 1: issuer i takes the S tiles of S buffer i.  Pass 2: issuer 0 takes
+// every S = Q K^T, issuer 1 every O += P V (one thread, so the accumulation
+// into O keeps its order).  Softmax warp w owns the
 // query rows 32 (w % 4) .. + 31 (its TMEM lane quarter) and the key / output
 // columns 64 (w / 4) .. + 63 of every tile; the two warps of a row quarter
 // exchange their partial row maximum and row sum through spare TMEM columns.
@@ -101,7 +107,7 @@ struct AnchorCfg {
   static_assert(D == 128, "the softmax anchor kernel is built for d = 128");
   static constexpr int kStages = 3;                 // K / V tile ring
   static constexpr int kTileBytes = G::kTileBytes;  // 32 KB
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128) + exchange
   static constexpr int kAccO = 256;
@@ -113,7 +119,7 @@ struct AnchorCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     gla_softmax_anchor_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v,
@@ -162,7 +168,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(rempty(s), 1);
     }
     mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
+    mbar_init(qempty, 2);
     for (int b = 0; b < 2; ++b) {
       mbar_init(sfull(b), 1);
       mbar_init(sfree(b), C::kSoftmaxWarps);
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(ofree, C::kSoftmaxWarps);
     mbar_init(zfull, 1);
     mbar_init(zfree, C::kSoftmaxWarps);
-    mbar_init(done_bar, 1);
+    mbar_init(done_bar, 2);
     mbar_init(xbar, C::kSoftmaxWarps);
     *abort = 0;
     fence_mbar_init();
@@ -246,12 +252,29 @@ __global__ void __launch_bounds__(320, 1)
       for (int64_t i = (n > S ? n - S : 0); i < n; ++i)
         mbar_wait_drain(rfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
     }
-  } else if (warp == C::kSoftmaxWarps + 1) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == C::kSoftmaxWarps + 1 || warp == C::kSoftmaxWarps + 2) {
+    // ------------------------------------------------------------ MMA issuers
+    const uint32_t me = static_cast<uint32_t>(warp - C::kSoftmaxWarps - 1);
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileTokens, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      int64_t n = 0, ns = 0, np = 0;  // ring tiles consumed, S tiles, P tiles
+      // Operand descriptors are built once; a K step or another buffer only
+      // moves the start address field (address >> 4, low 14 bits), so the
+      // issue loop adds compile-time offsets (shared memory is < 256 KB, no
+      // carry leaves the field).
+      constexpr uint64_t kBufStep = C::kTileBytes >> 4;
+      const uint64_t qd = smem_desc(q_buf, 16, G::kGroupBytes, G::kLayout);
+      const uint64_t kd = smem_desc(ring(0), 16, G::kGroupBytes, G::kLayout);
+      const uint64_t vd = smem_desc(ring(0), G::kAtomTileBytes, G::kGroupBytes, G::kLayout);
+      const uint64_t pd = smem_desc(p_buf(0), 16, G::kGroupBytes, G::kLayout);
+      uint32_t rs = 0, rph = 0;  // ring slot and phase of the next tile consumed
+      uint32_t ns = 0, np = 0;   // S tiles, P tiles
+      auto ring_next = [&]() {
+        if (++rs == static_cast<uint32_t>(S)) {
+          rs = 0;
+          rph ^= 1u;
+        }
+      };
       int64_t it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++it) {
@@ -261,67 +284,77 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(qfull, ph, abort, kCode)) break;
         // S = Q K^T of the next ring tile into S buffer ns % 2
         auto issue_s = [&]() {
-          const int sb = static_cast<int>(ns & 1);
-          const int s = static_cast<int>(n % S);
-          if (!mbar_wait(sfree(sb), static_cast<uint32_t>(((ns >> 1) & 1) ^ 1), abort, kCode) ||
-              !mbar_wait(rfull(s), static_cast<uint32_t>((n / S) & 1), abort, kCode))
+          const uint32_t sb = ns & 1u;
+          if (!mbar_wait(sfree(sb), ((ns >> 1) & 1u) ^ 1u, abort, kCode) ||
+              !mbar_wait(rfull(rs), rph, abort, kCode))
             return false;
           tc_fence_after();
+          const uint64_t bd0 = kd + rs * kBufStep;
+          const uint32_t dt = tmem + sb * kTileTokens;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const int a = kk / KPA, w = kk % KPA;
-            const uint64_t ad = smem_desc(q_buf + a * G::kAtomTileBytes + w * 32, 16,
-                                          G::kGroupBytes, G::kLayout);
-            const uint64_t bd = smem_desc(ring(s) + a * G::kAtomTileBytes + w * 32, 16,
-                                          G::kGroupBytes, G::kLayout);
-            mma_bf16(tmem + sb * kTileTokens, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off =
+                static_cast<uint64_t>(((kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32) >> 4);
+            mma_bf16(dt, qd + off, bd0 + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(sfull(sb));
-          mma_commit(rempty(s));
-          ++n;
+          mma_commit(rempty(rs));
+          ring_next();
           ++ns;
           return true;
         };
         // O += P V with P from buffer np % 2 and V the next ring tile
         auto issue_pv = [&](bool first) {
-          const int pb = static_cast<int>(np & 1);
-          const int sv = static_cast<int>(n % S);
-          if (!mbar_wait(pfull(pb), static_cast<uint32_t>((np >> 1) & 1), abort, kCode) ||
-              !mbar_wait(rfull(sv), static_cast<uint32_t>((n / S) & 1), abort, kCode))
+          const uint32_t pb = np & 1u;
+          if (!mbar_wait(pfull(pb), (np >> 1) & 1u, abort, kCode) ||
+              !mbar_wait(rfull(rs), rph, abort, kCode))
             return false;
           if (first && !mbar_wait(ofree, ph ^ 1u, abort, kCode)) return false;
           tc_fence_after();
+          const uint64_t ad0 = pd + pb * kBufStep;
+          const uint64_t bd0 = vd + rs * kBufStep;
 #pragma unroll
           for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-            const int a = kk / KPA, w = kk % KPA;
-            const uint64_t ad = smem_desc(p_buf(pb) + a * G::kAtomTileBytes + w * 32, 16,
-                                          G::kGroupBytes, G::kLayout);
-            const uint64_t bd = smem_desc(ring(sv) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
-                                          G::kGroupBytes, G::kLayout);
-            mma_bf16(tmem + C::kAccO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+            const uint64_t aoff =
+                static_cast<uint64_t>(((kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32) >> 4);
+            const uint64_t boff = static_cast<uint64_t>((kk * 2 * G::kGroupBytes) >> 4);
+            mma_bf16(tmem + C::kAccO, ad0 + aoff, bd0 + boff, idesc_o,
+                     (first && kk == 0) ? 0u : 1u);
           }
           mma_commit(pfree(pb));
-          mma_commit(rempty(sv));
-          ++n;
+          mma_commit(rempty(rs));
+          ring_next();
+          ++np;
+          return true;
+        };
+        // a tile the other issuer takes: only the counters move
+        auto skip_s = [&]() {
+          ring_next();
+          ++ns;
+          return true;
+        };
+        auto skip_pv = [&]() {
+          ring_next();
           ++np;
           return true;
         };
         KeyTiles kt;
-        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance()) ok = issue_s();
+        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance())
+          ok = (ns & 1u) == me ? issue_s() : skip_s();
         kt.init(p.T, f, p.window, p.n_sink);
         if (ok && !kt.done) {
-          ok = issue_s();
+          ok = me == 0 ? issue_s() : skip_s();
           for (bool first = true; ok; first = false) {
             kt.advance();
             const bool more = !kt.done;
-            if (more) ok = issue_s();
-            if (ok) ok = issue_pv(first);
+            if (more) ok = me == 0 ? issue_s() : skip_s();
+            if (ok) ok = me == 1 ? issue_pv(first) : skip_pv();
             if (!more) break;
           }
         }
         if (!ok) break;
-        mma_commit(qempty);  // Q no longer read
-        mma_commit(ofull);   // O of this unit complete
+        mma_commit(qempty);             // this issuer's reads of Q are done
+        if (me == 1) mma_commit(ofull);  // O of this unit complete
       }
       mma_commit(done_bar);
       mbar_wait_drain(done_bar, 0);
