@@ -11,30 +11,34 @@
 // optional per-element gate).
 //
 // One work unit = 128 query tokens of one (b, f, h).  Its key tiles (128 keys
-// of one frame, the frame's last tile ragged) are walked twice:
-//   pass 1  S = Q K^T into TMEM (double-buffered); the softmax warps keep the
-//           running row maximum m (invalid key rows masked to -inf);
-//   pass 2  S = Q K^T again; the softmax warps write P = exp(S - m) in bf16 to
-//           shared memory (two buffers) and sum l = sum P; O += P V
-//           accumulates in TMEM.  The MMA issuer runs one tile ahead: S of
-//           tile j+1 is issued before P V of tile j, so the tensor core
-//           computes the next scores while the softmax warps exponentiate.
-// Two passes cost one more Q K^T per tile but need no rescaling of the TMEM
-// accumulator when the maximum grows.  The epilogue writes sigmoid(z) O / l.
-// Ring order of the key/value tiles: pass 1 K0 K1 ..; pass 2 K0 K1 V0 K2 V1 ..
-// K(n-1) V(n-2) V(n-1), the order in which the MMA issuer consumes them.
+// of one frame, the frame's last tile ragged) are walked once, online:
+//   S = Q K^T into TMEM (two buffers); the softmax warps write
+//   P = 2^((S - m) log2(e) / sqrt(d)) in bf16 to shared memory (two buffers)
+//   and sum l = sum P; O += P V accumulates in TMEM.
+// The reference maximum m of a row moves lazily: only when a tile's maximum
+// exceeds it by more than 2^kRescaleLog2 in P, and then the row of O and l are
+// scaled by the ratio (after the previous P V has completed); otherwise P is
+// at most 2^kRescaleLog2 and the reference stays.  With scores of unit scale
+// this happens on a handful of tiles per unit.
+// Softmax warp w owns the query rows 32 (w % 4) .. + 31 (its TMEM lane
+// quarter) and the keys 64 (w / 4) .. + 63 of every tile; each key half keeps
+// its own m, l and O accumulator (P V is issued as two K = 64 halves), so the
+// two warps of a row quarter never wait on each other per tile.  They swap
+// (m, l) once per unit, through their own columns of the unit's last S buffer,
+// and the epilogue combines out = sigmoid(z) (O_0 f_0 + O_1 f_1) / (l_0 f_0 +
+// l_1 f_1), f_c = 2^(m_c - max(m_0, m_1)) in the scaled units.
+// The MMA issuers run one tile ahead: S of tile j+1 is issued before P V of
+// tile j, so the tensor core computes the next scores while the softmax warps
+// exponentiate.  Ring order of the key/value tiles: K0 K1 V0 K2 V1 ..
+// K(n-1) V(n-2) V(n-1), the order in which they are consumed.
 //   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
-//   PV: A = P [M = 128 queries, K = 128 keys] K-major, B = V tile [N = d] MN-major
+//   PV: A = P [M = 128 queries, K = 64 keys] K-major, B = V rows [N = d] MN-major
 // Warp roles: 0-7 softmax / epilogue, 8 TMA, 9 and 10 MMA.  A tcgen05.mma
 // issue returns only about when the tensor core takes the instruction, so a
 // lone issuing thread leaves the tensor core idle while it waits on barriers
-// and commits; two issuers overlap that bookkeeping with each other's MMAs.
-// Pass 1: issuer i takes the S tiles of S buffer i.  Pass 2: issuer 0 takes
-// every S = Q K^T, issuer 1 every O += P V (one thread, so the accumulation
-// into O keeps its order).  Softmax warp w owns the
-// query rows 32 (w % 4) .. + 31 (its TMEM lane quarter) and the key / output
-// columns 64 (w / 4) .. + 63 of every tile; the two warps of a row quarter
-// exchange their partial row maximum and row sum through spare TMEM columns.
+// and commits; two issuers overlap that bookkeeping with each other's MMAs:
+// issuer 0 takes every S = Q K^T, issuer 1 every O += P V (one thread, so the
+// accumulation into O keeps its order).
 #pragma once
 
 #include "gla_common.cuh"
@@ -109,9 +113,9 @@ struct AnchorCfg {
   static constexpr int kTileBytes = G::kTileBytes;  // 32 KB
   static constexpr int kThreads = 352;
   static constexpr int kSoftmaxWarps = 8;
-  static constexpr int kTmemCols = 512;             // S x 2 (256) + O (128) + exchange
-  static constexpr int kAccO = 256;
-  static constexpr int kXchg = 384;                 // m of half c at +c, l of half c at +2+c
+  static constexpr int kTmemCols = 512;             // S x 2 (256) + O of each key half (256)
+  static constexpr int kAccO = 256;                 // O of key half c at kAccO + 128 c
+  static constexpr float kRescaleLog2 = 8.0f;       // P <= 2^8 between rescales
   static constexpr int kBarCount = 2 * kStages + 16;
   // Q, P x 2, gate / output, ring
   static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t zfull = bar0 + 8u * (2 * S + 12);
   const uint32_t zfree = bar0 + 8u * (2 * S + 13);
   const uint32_t done_bar = bar0 + 8u * (2 * S + 14);
-  const uint32_t xbar = bar0 + 8u * (2 * S + 15);  // row max / row sum exchange
+  const uint32_t xbar = bar0 + 8u * (2 * S + 15);  // (m, l) exchange of the two key halves
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -238,8 +242,6 @@ __global__ void __launch_bounds__(352, 1)
           return true;
         };
         KeyTiles kt;
-        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance())
-          ok = load(&tm_k, kt.fr, kt.t0);
         int pfr = -1, pt0 = 0;  // the previous tile, whose V follows this tile's K
         for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance()) {
           ok = load(&tm_k, kt.fr, kt.t0);
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(352, 1)
         coords(unit, b, f, h, qt);
         const uint32_t ph = static_cast<uint32_t>(it & 1);
         if (!mbar_wait(qfull, ph, abort, kCode)) break;
-        // S = Q K^T of the next ring tile into S buffer ns % 2
+        // issuer 0: S = Q K^T of the next ring tile into S buffer ns % 2
         auto issue_s = [&]() {
           const uint32_t sb = ns & 1u;
           if (!mbar_wait(sfree(sb), ((ns >> 1) & 1u) ^ 1u, abort, kCode) ||
@@ -303,7 +305,8 @@ __global__ void __launch_bounds__(352, 1)
           ++ns;
           return true;
         };
-        // O += P V with P from buffer np % 2 and V the next ring tile
+        // issuer 1: O_c += P[:, 64 c ..] V[64 c .., :] for both key halves c, P
+        // from buffer np % 2 and V the next ring tile
         auto issue_pv = [&](bool first) {
           const uint32_t pb = np & 1u;
           if (!mbar_wait(pfull(pb), (np >> 1) & 1u, abort, kCode) ||
@@ -318,8 +321,8 @@ __global__ void __launch_bounds__(352, 1)
             const uint64_t aoff =
                 static_cast<uint64_t>(((kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32) >> 4);
             const uint64_t boff = static_cast<uint64_t>((kk * 2 * G::kGroupBytes) >> 4);
-            mma_bf16(tmem + C::kAccO, ad0 + aoff, bd0 + boff, idesc_o,
-                     (first && kk == 0) ? 0u : 1u);
+            mma_bf16(tmem + C::kAccO + (kk / KPA) * D, ad0 + aoff, bd0 + boff, idesc_o,
+                     (first && kk % KPA == 0) ? 0u : 1u);
           }
           mma_commit(pfree(pb));
           mma_commit(rempty(rs));
@@ -339,10 +342,8 @@ __global__ void __launch_bounds__(352, 1)
           return true;
         };
         KeyTiles kt;
-        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance())
-          ok = (ns & 1u) == me ? issue_s() : skip_s();
         kt.init(p.T, f, p.window, p.n_sink);
-        if (ok && !kt.done) {
+        if (!kt.done) {
           ok = me == 0 ? issue_s() : skip_s();
           for (bool first = true; ok; first = false) {
             kt.advance();
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(352, 1)
           }
         }
         if (!ok) break;
-        mma_commit(qempty);             // this issuer's reads of Q are done
+        mma_commit(qempty);              // this issuer's reads of Q are done
         if (me == 1) mma_commit(ofull);  // O of this unit complete
       }
       mma_commit(done_bar);
@@ -362,159 +363,199 @@ __global__ void __launch_bounds__(352, 1)
   } else {
     // -------------------------------------------------- softmax and epilogue
     const int q4 = warp & 3;          // TMEM lane quarter: query rows 32 q4 ..
-    const int hc = warp >> 2;         // column half: keys / outputs 64 hc ..
+    const int hc = warp >> 2;         // key half of the tiles, output columns 64 hc ..
     const int row = q4 * 32 + lane;   // query within the tile
     const int c0 = hc * 64;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t tx = tmem + lane_base + C::kXchg;
+    const float sl2 = p.scale_log2;
     int64_t ns = 0, np = 0, it = 0;
-    // the partner warp's partial value through TMEM column kXchg + slot;
-    // .ok (warp-uniform) is false if the wait gave up
-    struct Xchg {
-      float v;
-      bool ok;
-    };
-    auto exchange = [&](float mine, int slot, uint32_t parity) {
-      tmem_st_1col(tx + slot + hc, __float_as_uint(mine));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      if (!warp_wait(xbar, parity, abort, kCode)) return Xchg{0.f, false};
-      tc_fence_after();
-      uint32_t v;
-      tmem_ld_1col(tx + slot + (hc ^ 1), v);
-      tmem_wait_ld();
-      return Xchg{__uint_as_float(v), true};
-    };
     for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x, ++it) {
       int b, f, h, qt;
       coords(unit, b, f, h, qt);
       const uint32_t ph = static_cast<uint32_t>(it & 1);
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // this key half's reference maximum and sum
+      float mo = -INFINITY, lo = 0.f;  // the other half's, after the exchange
       bool ok = true;
-      for (int pass = 0; pass < 2 && ok; ++pass) {
-        KeyTiles kt;
-        kt.init(p.T, f, p.window, p.n_sink);
-        for (; !kt.done; kt.advance()) {
-          const int sb = static_cast<int>(ns & 1);
-          if (!warp_wait(sfull(sb), static_cast<uint32_t>((ns >> 1) & 1), abort, kCode)) {
+      KeyTiles kt;
+      kt.init(p.T, f, p.window, p.n_sink);
+      for (bool first = true; !kt.done; first = false) {
+        const int sb = static_cast<int>(ns & 1);
+        KeyTiles nx = kt;
+        nx.advance();
+        const bool last = nx.done;
+        if (!warp_wait(sfull(sb), static_cast<uint32_t>((ns >> 1) & 1), abort, kCode)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t ra[32], rb[32];  // keys c0 .. c0 + 31, c0 + 32 .. c0 + 63
+        const uint32_t ts = tmem + lane_base + sb * kTileTokens + c0;
+        tmem_ld_32cols(ts, ra);
+        tmem_ld_32cols(ts + 32, rb);
+        tmem_wait_ld();
+        if (kt.valid < c0 + 64) {  // keys past the tile's end: S = -inf
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (c0 + e >= kt.valid) ra[e] = __float_as_uint(-INFINITY);
+            if (c0 + 32 + e >= kt.valid) rb[e] = __float_as_uint(-INFINITY);
+          }
+        }
+        if (!last) {  // the unit's last S buffer carries the (m, l) exchange
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sfree(sb));
+        }
+        float mt;
+        {
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(ra[e]));
+            mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(rb[e]));
+          }
+          mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        }
+        bool grow = false;
+        if (first || m == -INFINITY)
+          m = mt;  // no P of this row's half has been non-zero yet: O and l are zero
+        else
+          grow = (mt - m) * sl2 > C::kRescaleLog2;
+        if (!first) {  // warp-uniform
+          if (__any_sync(0xffffffffu, grow)) {
+            // scale this warp's rows of O_hc once the previous P V is done
+            const uint32_t pp = static_cast<uint32_t>(np - 1);
+            if (!warp_wait(pfree(static_cast<int>(pp & 1u)), (pp >> 1) & 1u, abort, kCode)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const float fct = grow ? ex2_approx((m - mt) * sl2) : 1.0f;
+            if (grow) {
+              l *= fct;
+              m = mt;
+            }
+            const uint32_t to = tmem + lane_base + C::kAccO + hc * D;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld_32cols(to + cc * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * fct);
+              tmem_st_32cols(to + cc * 32, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0)
+        const int pb = static_cast<int>(np & 1);
+        if (!warp_wait(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort, kCode)) {
+          ok = false;
+          break;
+        }
+        const float ms = m == -INFINITY ? 0.f : m * sl2;
+        const uint32_t pbase = p_buf(pb) + hc * G::kAtomTileBytes + row * G::kRowBytes;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t sv = ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e];
+            x[e] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -ms));
+            ls[e & 3] += x[e];
+          }
+          uint4 w;
+          w.x = pack_bf16x2(x[0], x[1]);
+          w.y = pack_bf16x2(x[2], x[3]);
+          w.z = pack_bf16x2(x[4], x[5]);
+          w.w = pack_bf16x2(x[6], x[7]);
+          st_shared_v4(pbase + G::swz(row, ch) * 16, w);
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        fence_proxy_async_smem();
+        tc_fence_before();  // orders a rescale's TMEM stores before the P V
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pfull(pb));
+        ++np;
+        if (last) {
+          // swap (m, l) with the other key half through this half's own
+          // columns of the S buffer just read, then release it
+          const uint32_t mine = tmem + lane_base + sb * kTileTokens + c0;
+          const uint32_t other = tmem + lane_base + sb * kTileTokens + (c0 ^ 64);
+          tmem_st_1col(mine, __float_as_uint(m));
+          tmem_st_1col(mine + 1, __float_as_uint(l));
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xbar);
+          if (!warp_wait(xbar, ph, abort, kCode)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          uint32_t ra[32], rb[32];  // columns c0 .. c0 + 31, c0 + 32 .. c0 + 63
-          const uint32_t ts = tmem + lane_base + sb * kTileTokens + c0;
-          tmem_ld_32cols(ts, ra);
-          tmem_ld_32cols(ts + 32, rb);
+          uint32_t v0, v1;
+          tmem_ld_1col(other, v0);
+          tmem_ld_1col(other + 1, v1);
           tmem_wait_ld();
-          if (kt.valid < c0 + 64) {  // keys past the tile's end: S = -inf
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (c0 + e >= kt.valid) ra[e] = __float_as_uint(-INFINITY);
-              if (c0 + 32 + e >= kt.valid) rb[e] = __float_as_uint(-INFINITY);
-            }
-          }
-          if (pass == 0) {
-            float mx[4] = {m, m, m, m};
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(ra[e]));
-              mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(rb[e]));
-            }
-            m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sfree(sb));
-          } else {
-            // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0)
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sfree(sb));  // S read into registers
-            const int pb = static_cast<int>(np & 1);
-            if (!warp_wait(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort, kCode)) {
-              ok = false;
-              break;
-            }
-            const float ms = m * p.scale_log2;
-            const uint32_t pbase = p_buf(pb) + hc * G::kAtomTileBytes + row * G::kRowBytes;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              float x[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const uint32_t sv = ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e];
-                x[e] = ex2_approx(fmaf(__uint_as_float(sv), p.scale_log2, -ms));
-                ls[e & 3] += x[e];
-              }
-              uint4 w;
-              w.x = pack_bf16x2(x[0], x[1]);
-              w.y = pack_bf16x2(x[2], x[3]);
-              w.z = pack_bf16x2(x[4], x[5]);
-              w.w = pack_bf16x2(x[6], x[7]);
-              st_shared_v4(pbase + G::swz(row, ch) * 16, w);
-            }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pfull(pb));
-            ++np;
-          }
-          ++ns;
+          mo = __uint_as_float(v0);
+          lo = __uint_as_float(v1);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sfree(sb));
         }
-        if (!ok) break;
-        if (pass == 0) {  // the row maximum over both column halves
-          const Xchg mo = exchange(m, 0, 0u);
-          if (!mo.ok) {
-            ok = false;
-            break;
-          }
-          m = fmaxf(m, mo.v);
-        }
+        ++ns;
+        kt = nx;
       }
       if (!ok) break;
-      const Xchg lo = exchange(l, 2, 1u);
-      if (!lo.ok) break;
-      l += lo.v;
-      // ---- epilogue: out = sigmoid(z) * O / l, columns [c0, c0 + 64)
+      // ---- epilogue: out = sigmoid(z) (O_0 f_0 + O_1 f_1) / (l_0 f_0 + l_1 f_1)
+      const float mm = fmaxf(m, mo);
+      const float f_me = m == -INFINITY ? 0.f : ex2_approx((m - mm) * sl2);
+      const float f_ot = mo == -INFINITY ? 0.f : ex2_approx((mo - mm) * sl2);
+      const float f0 = hc == 0 ? f_me : f_ot, f1 = hc == 0 ? f_ot : f_me;
+      const float rl = 1.0f / (l * f_me + lo * f_ot);
       if (!warp_wait(ofull, ph, abort, kCode)) break;
       if (p.has_gate && !warp_wait(zfull, ph, abort, kCode)) break;
       tc_fence_after();
       if (lane == 0) bulk_wait_group_read<0>();  // the previous output left o_buf
       __syncwarp();
-      const float rl = 1.0f / l;
-      uint32_t ra[32], rb[32];
-      const uint32_t to = tmem + lane_base + C::kAccO + c0;
-      tmem_ld_32cols(to, ra);
-      tmem_ld_32cols(to + 32, rb);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ofree);  // O read into registers
       const uint32_t obase = o_buf + hc * G::kAtomTileBytes + row * G::kRowBytes;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t addr = obase + G::swz(row, ch) * 16;
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          x[e] = __uint_as_float(ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e]) * rl;
-        if (p.has_gate) {
-          const uint4 zw = ld_shared_v4(addr);
-          const uint32_t zz[4] = {zw.x, zw.y, zw.z, zw.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float z = (e & 1) ? bf16hi_to_f32(zz[e >> 1]) : bf16lo_to_f32(zz[e >> 1]);
-            x[e] *= 1.0f / (1.0f + expf(-z));
-          }
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t ra[32], rb[32];  // O_0 and O_1, output columns c0 + 32 cc ..
+        const uint32_t to = tmem + lane_base + C::kAccO + c0 + cc * 32;
+        tmem_ld_32cols(to, ra);
+        tmem_ld_32cols(to + D, rb);
+        tmem_wait_ld();
+        if (cc == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ofree);  // O read into registers
         }
-        uint4 w;
-        w.x = pack_bf16x2(x[0], x[1]);
-        w.y = pack_bf16x2(x[2], x[3]);
-        w.z = pack_bf16x2(x[4], x[5]);
-        w.w = pack_bf16x2(x[6], x[7]);
-        st_shared_v4(addr, w);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t addr = obase + G::swz(row, cc * 4 + ch) * 16;
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            x[e] = (__uint_as_float(ra[ch * 8 + e]) * f0 + __uint_as_float(rb[ch * 8 + e]) * f1) *
+                   rl;
+          if (p.has_gate) {
+            const uint4 zw = ld_shared_v4(addr);
+            const uint32_t zz[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float z = (e & 1) ? bf16hi_to_f32(zz[e >> 1]) : bf16lo_to_f32(zz[e >> 1]);
+              x[e] *= 1.0f / (1.0f + expf(-z));
+            }
+          }
+          uint4 w;
+          w.x = pack_bf16x2(x[0], x[1]);
+          w.y = pack_bf16x2(x[2], x[3]);
+          w.z = pack_bf16x2(x[4], x[5]);
+          w.w = pack_bf16x2(x[6], x[7]);
+          st_shared_v4(addr, w);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();

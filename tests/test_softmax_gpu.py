@@ -103,3 +103,17 @@ def test_full_size_720p_5s_sampled_heads():
         sl = lambda x: x[b, :, h].float().cpu().numpy()  # noqa: E731
         ref = oracle.softmax_anchor_head(sl(q), sl(k), sl(v), T, 2, T, sl(z))
         assert_close(sl(out), ref, "out[b=%d,h=%d]" % (b, h))
+
+
+@pytest.mark.parametrize("gate", [False, True])
+def test_growing_scores_rescale_the_accumulator(gate):
+    """Keys of frame f scaled by 1 + 4 f: with a window over every frame each
+    new frame raises the row maxima far beyond the kernel's rescale threshold,
+    so the running accumulator is rescaled many times per query tile."""
+    B, H, F, T = 1, 2, 4, 200
+    q, k, v, z = case(B, H, F, T, 8100, gate)
+    scale = torch.repeat_interleave(1.0 + 4.0 * torch.arange(F, dtype=torch.float32), T)
+    k = (k.float() * scale[None, :, None, None]).to(torch.bfloat16)
+    out = run_gpu(q, k, v, z, F, F, 0)
+    ref = oracle.softmax_anchor_forward(q, k, v, F, F, 0, z)
+    assert_close(out, ref, "out")
