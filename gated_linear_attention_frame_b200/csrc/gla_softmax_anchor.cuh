@@ -105,6 +105,35 @@ struct KeyTiles {
   }
 };
 
+// 2^x on the FMA pipe, for part of the exponentials of P (the MUFU unit that
+// runs ex2.approx does 16 per clock per SM and bounds the softmax otherwise).
+// Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer n in the
+// low mantissa bits, r = x - n lies in [-1/2, 1/2]; 2^r by a degree-3
+// polynomial fitted to 2^r on that interval (iteratively reweighted least
+// squares towards the minimax relative error: 7.5e-5, far below the bf16
+// rounding of P); n is added to the exponent field.  x is clamped at -126, so
+// masked keys (x = -inf) give about 1e-38 instead of 0, which no sum notices.
+constexpr float kExp2C0 = 0.9999281167984009f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.24261054396629333f;
+constexpr float kExp2C3 = 0.05517132207751274f;
+
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23
+  const float r = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, r, kExp2C2), r, kExp2C1), r, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// A wait on a phase that has most likely completed already: one vote of the
+// warp on a single try_wait, the bounded warp_wait otherwise.
+__device__ __forceinline__ bool warp_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               unsigned int code) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return warp_wait(bar, parity, abort, code);
+}
+
 template <int D>
 struct AnchorCfg {
   using G = Geo<D>;
@@ -116,6 +145,7 @@ struct AnchorCfg {
   static constexpr int kTmemCols = 512;             // S x 2 (256) + O of each key half (256)
   static constexpr int kAccO = 256;                 // O of key half c at kAccO + 128 c
   static constexpr float kRescaleLog2 = 8.0f;       // P <= 2^8 between rescales
+  static constexpr int kPolyPerChunk = 3;           // of each 8 exponentials, on the FMA pipe
   static constexpr int kBarCount = 2 * kStages + 16;
   // Q, P x 2, gate / output, ring
   static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
@@ -383,7 +413,7 @@ __global__ void __launch_bounds__(352, 1)
         KeyTiles nx = kt;
         nx.advance();
         const bool last = nx.done;
-        if (!warp_wait(sfull(sb), static_cast<uint32_t>((ns >> 1) & 1), abort, kCode)) {
+        if (!warp_wait_fast(sfull(sb), static_cast<uint32_t>((ns >> 1) & 1), abort, kCode)) {
           ok = false;
           break;
         }
@@ -449,7 +479,8 @@ __global__ void __launch_bounds__(352, 1)
         }
         // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0)
         const int pb = static_cast<int>(np & 1);
-        if (!warp_wait(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort, kCode)) {
+        if (!warp_wait_fast(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort,
+                            kCode)) {
           ok = false;
           break;
         }
@@ -462,7 +493,8 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t sv = ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e];
-            x[e] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -ms));
+            const float arg = fmaf(__uint_as_float(sv), sl2, -ms);
+            x[e] = e < C::kPolyPerChunk ? exp2_poly3(arg) : ex2_approx(arg);
             ls[e & 3] += x[e];
           }
           uint4 w;
