@@ -145,7 +145,8 @@ struct AnchorCfg {
   static constexpr int kTmemCols = 512;             // S x 2 (256) + O of each key half (256)
   static constexpr int kAccO = 256;                 // O of key half c at kAccO + 128 c
   static constexpr float kRescaleLog2 = 8.0f;       // P <= 2^8 between rescales
-  static constexpr int kPolyPerChunk = 3;           // of each 8 exponentials, on the FMA pipe
+  static constexpr int kPolyPairs = 1;              // of each 4 pairs of exponentials, on the
+                                                    // FMA pipe
   static constexpr int kBarCount = 2 * kStages + 16;
   // Q, P x 2, gate / output, ring
   static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
@@ -439,10 +440,8 @@ __global__ void __launch_bounds__(352, 1)
         {
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(ra[e]));
-            mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(rb[e]));
-          }
+          for (int e = 0; e < 32; ++e)
+            mx[e & 3] = fmax3(mx[e & 3], __uint_as_float(ra[e]), __uint_as_float(rb[e]));
           mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         }
         bool grow = false;
@@ -486,25 +485,36 @@ __global__ void __launch_bounds__(352, 1)
         }
         const float ms = m == -INFINITY ? 0.f : m * sl2;
         const uint32_t pbase = p_buf(pb) + hc * G::kAtomTileBytes + row * G::kRowBytes;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t sc2 = f2_pack(sl2, sl2), sh2 = f2_pack(-ms, -ms);
+        uint64_t ls2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // pair-wise row sums
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          float x[8];
+          uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t sv = ch < 4 ? ra[ch * 8 + e] : rb[(ch - 4) * 8 + e];
-            const float arg = fmaf(__uint_as_float(sv), sl2, -ms);
-            x[e] = e < C::kPolyPerChunk ? exp2_poly3(arg) : ex2_approx(arg);
-            ls[e & 3] += x[e];
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int e = ch * 8 + 2 * e2;
+            const float s0 = __uint_as_float(e < 32 ? ra[e] : rb[e - 32]);
+            const float s1 = __uint_as_float(e < 32 ? ra[e + 1] : rb[e - 31]);
+            float a0, a1, x0, x1;
+            f2_unpack(f2_fma(f2_pack(s0, s1), sc2, sh2), a0, a1);
+            if (e2 < C::kPolyPairs) {
+              x0 = exp2_poly3(a0);
+              x1 = exp2_poly3(a1);
+            } else {
+              x0 = ex2_approx(a0);
+              x1 = ex2_approx(a1);
+            }
+            ls2[e2 & 1] = f2_add(ls2[e2 & 1], f2_pack(x0, x1));
+            w[e2] = pack_bf16x2(x0, x1);
           }
-          uint4 w;
-          w.x = pack_bf16x2(x[0], x[1]);
-          w.y = pack_bf16x2(x[2], x[3]);
-          w.z = pack_bf16x2(x[4], x[5]);
-          w.w = pack_bf16x2(x[6], x[7]);
-          st_shared_v4(pbase + G::swz(row, ch) * 16, w);
+          st_shared_v4(pbase + G::swz(row, ch) * 16, make_uint4(w[0], w[1], w[2], w[3]));
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        {
+          float l0, l1, l2, l3;
+          f2_unpack(ls2[0], l0, l1);
+          f2_unpack(ls2[1], l2, l3);
+          l += (l0 + l1) + (l2 + l3);
+        }
         fence_proxy_async_smem();
         tc_fence_before();  // orders a rescale's TMEM stores before the P V
         __syncwarp();
