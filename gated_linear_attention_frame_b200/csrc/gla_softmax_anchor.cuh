@@ -126,6 +126,21 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// The same for two lanes with the packed pair arithmetic.
+__device__ __forceinline__ void exp2_poly3_x2(float a0, float a1, float& x0, float& x1) {
+  const uint64_t x = f2_pack(fmaxf(a0, -126.0f), fmaxf(a1, -126.0f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t r = f2_sub(x, f2_sub(t, f2_pack(12582912.0f, 12582912.0f)));
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), r, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, r, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, r, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  x0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  x1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // A wait on a phase that has most likely completed already: one vote of the
 // warp on a single try_wait, the bounded warp_wait otherwise.
 __device__ __forceinline__ bool warp_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
@@ -498,8 +513,7 @@ __global__ void __launch_bounds__(352, 1)
             float a0, a1, x0, x1;
             f2_unpack(f2_fma(f2_pack(s0, s1), sc2, sh2), a0, a1);
             if (e2 < C::kPolyPairs) {
-              x0 = exp2_poly3(a0);
-              x1 = exp2_poly3(a1);
+              exp2_poly3_x2(a0, a1, x0, x1);
             } else {
               x0 = ex2_approx(a0);
               x1 = ex2_approx(a1);
