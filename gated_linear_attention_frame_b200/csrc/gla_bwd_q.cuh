@@ -23,7 +23,10 @@
 // D enters MMA3 as a hi/lo pair of bf16 copies (D = D_hi + D_lo, D_lo the
 // bf16 rounding of the remainder): the gate gradient <G_f, S_{f-1}> and dk
 // sum thousands of products of L_f with random signs, and one bf16 rounding
-// of D would put their error near the tolerance; dq uses D_hi alone.
+// of D would put their error near the tolerance; dq uses D_hi alone.  The
+// pad region holds dden's hi part in its column 0 and its lo part in column
+// 1, so one N = 16 MMA per K step gives both (L_f[:, d] = their sum); MMA2
+// meets column 1 only against a zero padding row of the S_f^T image.
 // The ReLU warps keep a byte mask of q > 0 for the dq epilogue, so a q stage
 // is released as soon as MMA3 has read it.
 // Warp roles: 0-3 epilogue, 4-7 ReLU, 8 TMA, 9 MMA.
@@ -87,7 +90,6 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t d_buf = s_buf + C::kSBufBytes;          // D_hi
   const uint32_t d_pad = d_buf + C::kDMainBytes;
   const uint32_t l_buf = d_buf + C::kDBytes;             // D_lo
-  const uint32_t l_pad = l_buf + C::kDMainBytes;
   const uint32_t o_base = l_buf + C::kDBytes;
   uint8_t* mask_ring = smem + S * G::kTileBytes + C::kSBufBytes + 2 * C::kDBytes +
                        2 * C::kStageOutBytes;
@@ -158,10 +160,8 @@ __global__ void __launch_bounds__(320, 1)
                        ch * 16,
                    z);
     }
-    for (int o = threadIdx.x * 16; o < C::kDPadBytes; o += C::kThreads * 16) {
+    for (int o = threadIdx.x * 16; o < C::kDPadBytes; o += C::kThreads * 16)
       st_shared_v4(d_pad + o, z);
-      st_shared_v4(l_pad + o, z);
-    }
     fence_proxy_async_smem();
   }
   if (warp == 0) {
@@ -283,8 +283,6 @@ __global__ void __launch_bounds__(320, 1)
           const uint64_t bl = smem_desc(l_buf + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
                                         G::kGroupBytes, G::kLayout);
           mma_bf16(tmem + C::kAcc3, ad, bl, idesc3, 1u);
-          const uint64_t blz = smem_desc(l_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
-          mma_bf16(tmem + C::kAcc3 + D, ad, blz, idesc3z, 1u);
         }
         mma_commit(qempty(s));
         mma_commit(dfree);
@@ -390,12 +388,11 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       const float dot = (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
       const float dden = valid_tok ? -dot * rden * rden : 0.f;
-      const uint32_t dden_hi = pack_bf16x2(dden, 0.f);
-      const float dden_lo = dden - bf16lo_to_f32(dden_hi);
-      // pad region row: chunk 0 (columns 0..7) sits at chunk slot (row >> 2) & 1
+      const float dden_lo = dden - bf16lo_to_f32(pack_bf16x2(dden, 0.f));
+      // pad region row: chunk 0 (columns 0..7) sits at chunk slot (row >> 2) & 1;
+      // column 0 = dden rounded to bf16, column 1 = the rounding's remainder
       const uint32_t poff = row * 32 + ((row >> 2) & 1) * 16;
-      st_shared_v4(d_pad + poff, make_uint4(dden_hi, 0u, 0u, 0u));
-      st_shared_v4(l_pad + poff, make_uint4(pack_bf16x2(dden_lo, 0.f), 0u, 0u, 0u));
+      st_shared_v4(d_pad + poff, make_uint4(pack_bf16x2(dden, dden_lo), 0u, 0u, 0u));
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -468,10 +465,11 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
         }
-        uint32_t zr;
+        uint32_t zr, zl;  // the normaliser column: hi and lo parts of dden
         tmem_ld_1col(t3 + D, zr);
+        tmem_ld_1col(t3 + D + 1, zl);
         tmem_wait_ld();
-        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr);
+        dst[static_cast<int64_t>(D) * D] = __uint_as_float(zr) + __uint_as_float(zl);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc3_free);
