@@ -85,9 +85,9 @@ KERNEL_DEPS = {
 }
 NCU_TRAFFIC = {
     "720p-5s": {
-        "increment": (1899738368 + 65973760, "adfba699d59f78a6"),
-        "scan": (75846144 + 5643008, "4d675cb7e40bc9d1"),
-        "output": (985641728 + 897636864, "60851f75ff180302"),
+        "increment": (1899750400 + 65932800, "7ba1204ca68b5243"),
+        "scan": (75847168 + 5340416, "a01d1703ef5f48a1"),
+        "output": (985584384 + 895718912, "da79c97d4ca61853"),
     },
 }
 
