@@ -82,3 +82,44 @@ def test_reference_arm_prints_on_rank0_only(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip())
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_of_every_path(capsys, monkeypatch):
+    """The reference arm (the oracle on the host) prints one valid line for
+    the layer, each variant and the backward pass, with that path's metric."""
+    sys.path.insert(0, ROOT)
+    import json
+
+    import bench
+
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    seen = set()
+    for extra in (["--variant", "rope"], ["--variant", "gdn"], ["--variant", "softmax"],
+                  ["--mode", "backward"]):
+        assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0",
+                           "--workload", "tiny"] + extra) == 0
+        line = json.loads(capsys.readouterr().out.strip())
+        assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
+        assert line["metric"] == bench.metric_for(*(("backward", "plain") if "--mode" in extra
+                                                    else ("forward", extra[1])))
+        seen.add(line["metric"])
+    assert len(seen) == 4
+
+
+def test_anchor_pair_count_matches_the_oracle_key_ranges():
+    """The softmax anchor's roofline counts 4 d flops per (query, key) pair;
+    the pair count agrees with the oracle's key ranges summed frame by frame."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle.gla_softmax_oracle import anchor_key_ranges
+    from workloads import WORKLOADS
+
+    for name, window, n_sink in (("720p-5s", 2, 3680), ("tiny", 3, 5), ("480p-5s", 1, 0)):
+        w = WORKLOADS[name]
+        T = w.tokens_per_frame
+        per_bh = 0
+        for f in range(w.frames):
+            (s0, s1), (w0, w1) = anchor_key_ranges(f, T, window, n_sink)
+            per_bh += T * ((s1 - s0) + (w1 - w0))
+        assert bench.anchor_pairs(w, window, n_sink) == per_bh * w.B * w.H
