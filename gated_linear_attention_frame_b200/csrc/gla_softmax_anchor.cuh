@@ -27,6 +27,11 @@
 // (m, l) once per unit, through their own columns of the unit's last S buffer,
 // and the epilogue combines out = sigmoid(z) (O_0 f_0 + O_1 f_1) / (l_0 f_0 +
 // l_1 f_1), f_c = 2^(m_c - max(m_0, m_1)) in the scaled units.
+// The softmax is bound by instruction issue and the MUFU exponential unit:
+// it scales and shifts the scores and sums P on packed fp32 pairs
+// (fma / add .f32x2), takes the tile maximum with a three-input max, and
+// computes one pair of exponentials in four on the FMA pipe (exp2_poly3_x2),
+// the rest with ex2.approx.
 // The MMA issuers run one tile ahead: S of tile j+1 is issued before P V of
 // tile j, so the tensor core computes the next scores while the softmax warps
 // exponentiate.  Ring order of the key/value tiles: K0 K1 V0 K2 V1 ..

@@ -165,6 +165,10 @@ size_t gla_noalloc_scratch_bytes(void);
  * shape or NULL (no gate); window_frames >= 1; n_sink >= 0.  No workspace.
  * Returns the gla_forward codes (GLA_ERR_SHAPE for window_frames < 1 or
  * n_sink < 0).
+ * Precision: scores and row sums in fp32; the softmax weights enter P V
+ * rounded to bf16 (some exponentials by a polynomial of relative error
+ * 7.5e-5); out is rounded once to bf16.  Keys past a frame's end are masked;
+ * a query always sees its own frame, so every row has at least one key.
  */
 int gla_softmax_anchor(const void* q, const void* k, const void* v, const void* gate_z,
                        void* out, int B, int H, int frames, int tokens_per_frame, int d,
