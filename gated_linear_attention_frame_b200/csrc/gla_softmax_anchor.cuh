@@ -13,8 +13,10 @@
 // One work unit = 128 query tokens of one (b, f, h).  Its key tiles (128 keys
 // of one frame, the frame's last tile ragged) are walked once, online:
 //   S = Q K^T into TMEM (two buffers); the softmax warps write
-//   P = 2^((S - m) log2(e) / sqrt(d)) in bf16 to shared memory (two buffers)
-//   and sum l = sum P; O += P V accumulates in TMEM.
+//   P = 2^((S - m) log2(e) / sqrt(d)) in bf16 back into the S buffer they
+//   just read (two bf16 per 32-bit column, each key half into the first half
+//   of its own columns) and sum l = sum P; O += P V accumulates in TMEM with
+//   P as the MMA's A operand straight from TMEM.
 // The reference maximum m of a row moves lazily: only when a tile's maximum
 // exceeds it by more than 2^kRescaleLog2 in P, and then the row of O and l are
 // scaled by the ratio (after the previous P V has completed); otherwise P is
@@ -37,7 +39,7 @@
 // exponentiate.  Ring order of the key/value tiles: K0 K1 V0 K2 V1 ..
 // K(n-1) V(n-2) V(n-1), the order in which they are consumed.
 //   S:  A = Q [M = 128 queries, K = d] K-major,   B = K tile [N = 128 keys] K-major
-//   PV: A = P [M = 128 queries, K = 64 keys] K-major, B = V rows [N = d] MN-major
+//   PV: A = P [M = 128 queries, K = 64 keys] in TMEM, B = V rows [N = d] MN-major
 // Warp roles: 0-7 softmax / epilogue, 8 TMA, 9 and 10 MMA.  A tcgen05.mma
 // issue returns only about when the tensor core takes the instruction, so a
 // lone issuing thread leaves the tensor core idle while it waits on barriers
@@ -146,6 +148,18 @@ __device__ __forceinline__ void exp2_poly3_x2(float a0, float a1, float& x0, flo
   x1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate (A: lane
+// = row, two consecutive K elements per 32-bit column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // A wait on a phase that has most likely completed already: one vote of the
 // warp on a single try_wait, the bounded warp_wait otherwise.
 __device__ __forceinline__ bool warp_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
@@ -158,7 +172,7 @@ template <int D>
 struct AnchorCfg {
   using G = Geo<D>;
   static_assert(D == 128, "the softmax anchor kernel is built for d = 128");
-  static constexpr int kStages = 3;                 // K / V tile ring
+  static constexpr int kStages = 5;                 // K / V tile ring
   static constexpr int kTileBytes = G::kTileBytes;  // 32 KB
   static constexpr int kThreads = 352;
   static constexpr int kSoftmaxWarps = 8;
@@ -168,8 +182,8 @@ struct AnchorCfg {
   static constexpr int kPolyPairs = 1;              // of each 4 pairs of exponentials, on the
                                                     // FMA pipe
   static constexpr int kBarCount = 2 * kStages + 16;
-  // Q, P x 2, gate / output, ring
-  static constexpr int kSmemBytes = 1024 + (4 + kStages) * kTileBytes + kBarCount * 8 + 16;
+  // Q, gate / output, ring
+  static constexpr int kSmemBytes = 1024 + (2 + kStages) * kTileBytes + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -191,10 +205,9 @@ __global__ void __launch_bounds__(352, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t q_buf = sbase;
-  auto p_buf = [&](int i) { return sbase + (1 + i) * C::kTileBytes; };
-  const uint32_t o_buf = sbase + 3 * C::kTileBytes;  // gate in, output out
-  auto ring = [&](int s) { return sbase + (4 + s) * C::kTileBytes; };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (4 + S) * C::kTileBytes);
+  const uint32_t o_buf = sbase + C::kTileBytes;  // gate in, output out
+  auto ring = [&](int s) { return sbase + (2 + s) * C::kTileBytes; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + S) * C::kTileBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto rfull = [&](int s) { return bar0 + 8u * s; };
   auto rempty = [&](int s) { return bar0 + 8u * (S + s); };
@@ -319,7 +332,6 @@ __global__ void __launch_bounds__(352, 1)
       const uint64_t qd = smem_desc(q_buf, 16, G::kGroupBytes, G::kLayout);
       const uint64_t kd = smem_desc(ring(0), 16, G::kGroupBytes, G::kLayout);
       const uint64_t vd = smem_desc(ring(0), G::kAtomTileBytes, G::kGroupBytes, G::kLayout);
-      const uint64_t pd = smem_desc(p_buf(0), 16, G::kGroupBytes, G::kLayout);
       uint32_t rs = 0, rph = 0;  // ring slot and phase of the next tile consumed
       uint32_t ns = 0, np = 0;   // S tiles, P tiles
       auto ring_next = [&]() {
@@ -336,9 +348,11 @@ __global__ void __launch_bounds__(352, 1)
         const uint32_t ph = static_cast<uint32_t>(it & 1);
         if (!mbar_wait(qfull, ph, abort, kCode)) break;
         // issuer 0: S = Q K^T of the next ring tile into S buffer ns % 2
+        // (the buffer also held P of tile ns - 2: wait for that P V too)
         auto issue_s = [&]() {
           const uint32_t sb = ns & 1u;
           if (!mbar_wait(sfree(sb), ((ns >> 1) & 1u) ^ 1u, abort, kCode) ||
+              !mbar_wait(pfree(sb), ((ns >> 1) & 1u) ^ 1u, abort, kCode) ||
               !mbar_wait(rfull(rs), rph, abort, kCode))
             return false;
           tc_fence_after();
@@ -357,7 +371,8 @@ __global__ void __launch_bounds__(352, 1)
           return true;
         };
         // issuer 1: O_c += P[:, 64 c ..] V[64 c .., :] for both key halves c, P
-        // from buffer np % 2 and V the next ring tile
+        // in S buffer np % 2 (key half c at its columns 64 c .. + 31) and V the
+        // next ring tile
         auto issue_pv = [&](bool first) {
           const uint32_t pb = np & 1u;
           if (!mbar_wait(pfull(pb), (np >> 1) & 1u, abort, kCode) ||
@@ -365,15 +380,14 @@ __global__ void __launch_bounds__(352, 1)
             return false;
           if (first && !mbar_wait(ofree, ph ^ 1u, abort, kCode)) return false;
           tc_fence_after();
-          const uint64_t ad0 = pd + pb * kBufStep;
+          const uint32_t pa = tmem + pb * kTileTokens;
           const uint64_t bd0 = vd + rs * kBufStep;
 #pragma unroll
           for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-            const uint64_t aoff =
-                static_cast<uint64_t>(((kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32) >> 4);
+            const uint32_t acol = (kk / KPA) * 64 + (kk % KPA) * 8;  // 16 keys = 8 columns
             const uint64_t boff = static_cast<uint64_t>((kk * 2 * G::kGroupBytes) >> 4);
-            mma_bf16(tmem + C::kAccO + (kk / KPA) * D, ad0 + aoff, bd0 + boff, idesc_o,
-                     (first && kk % KPA == 0) ? 0u : 1u);
+            mma_bf16_ts(tmem + C::kAccO + (kk / KPA) * D, pa + acol, bd0 + boff, idesc_o,
+                        (first && kk % KPA == 0) ? 0u : 1u);
           }
           mma_commit(pfree(pb));
           mma_commit(rempty(rs));
@@ -496,20 +510,16 @@ __global__ void __launch_bounds__(352, 1)
             tmem_wait_st();
           }
         }
-        // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0)
+        // P = 2^((S - m) scale log2 e) in bf16 (masked keys give 0), written
+        // over this half's S columns (S of this buffer landed after the P V
+        // that last read it, so the columns are free)
         const int pb = static_cast<int>(np & 1);
-        if (!warp_wait_fast(pfree(pb), static_cast<uint32_t>(((np >> 1) & 1) ^ 1), abort,
-                            kCode)) {
-          ok = false;
-          break;
-        }
         const float ms = m == -INFINITY ? 0.f : m * sl2;
-        const uint32_t pbase = p_buf(pb) + hc * G::kAtomTileBytes + row * G::kRowBytes;
+        uint32_t pw[32];
         const uint64_t sc2 = f2_pack(sl2, sl2), sh2 = f2_pack(-ms, -ms);
         uint64_t ls2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // pair-wise row sums
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const int e = ch * 8 + 2 * e2;
@@ -524,26 +534,26 @@ __global__ void __launch_bounds__(352, 1)
               x1 = ex2_approx(a1);
             }
             ls2[e2 & 1] = f2_add(ls2[e2 & 1], f2_pack(x0, x1));
-            w[e2] = pack_bf16x2(x0, x1);
+            pw[ch * 4 + e2] = pack_bf16x2(x0, x1);
           }
-          st_shared_v4(pbase + G::swz(row, ch) * 16, make_uint4(w[0], w[1], w[2], w[3]));
         }
+        tmem_st_32cols(tmem + lane_base + sb * kTileTokens + c0, pw);
+        tmem_wait_st();
         {
           float l0, l1, l2, l3;
           f2_unpack(ls2[0], l0, l1);
           f2_unpack(ls2[1], l2, l3);
           l += (l0 + l1) + (l2 + l3);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();  // orders a rescale's TMEM stores before the P V
+        tc_fence_before();  // orders P's (and a rescale's) TMEM stores before the P V
         __syncwarp();
         if (lane == 0) mbar_arrive(pfull(pb));
         ++np;
         if (last) {
           // swap (m, l) with the other key half through this half's own
-          // columns of the S buffer just read, then release it
-          const uint32_t mine = tmem + lane_base + sb * kTileTokens + c0;
-          const uint32_t other = tmem + lane_base + sb * kTileTokens + (c0 ^ 64);
+          // columns of the S buffer just read (past its P), then release it
+          const uint32_t mine = tmem + lane_base + sb * kTileTokens + c0 + 32;
+          const uint32_t other = tmem + lane_base + sb * kTileTokens + (c0 ^ 64) + 32;
           tmem_st_1col(mine, __float_as_uint(m));
           tmem_st_1col(mine + 1, __float_as_uint(l));
           tmem_wait_st();
