@@ -213,10 +213,13 @@ __global__ void __launch_bounds__(352, 1)
   auto rempty = [&](int s) { return bar0 + 8u * (S + s); };
   const uint32_t qfull = bar0 + 8u * (2 * S + 0);
   const uint32_t qempty = bar0 + 8u * (2 * S + 1);
+  // per S buffer b: S landed (sfull), the softmax warps are done with its
+  // scores and, on a unit's last tile, with the (m, l) exchange (sfree), P is
+  // written over it (pfull), the P V that read that P is done (pfree)
   auto sfull = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
   auto sfree = [&](int b) { return bar0 + 8u * (2 * S + 4 + b); };
-  auto pfull = [&](int i) { return bar0 + 8u * (2 * S + 6 + i); };
-  auto pfree = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
+  auto pfull = [&](int b) { return bar0 + 8u * (2 * S + 6 + b); };
+  auto pfree = [&](int b) { return bar0 + 8u * (2 * S + 8 + b); };
   const uint32_t ofull = bar0 + 8u * (2 * S + 10);
   const uint32_t ofree = bar0 + 8u * (2 * S + 11);
   const uint32_t zfull = bar0 + 8u * (2 * S + 12);
