@@ -30,7 +30,9 @@ EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noal
             "gla_forward_rope", "gla_forward_rope_timed", "gla_forward_gdn", "gla_forward_gdn_timed",
             "gla_softmax_anchor", "gla_softmax_anchor_timed",
             "gla_backward", "gla_backward_timed",
-            "gla_trim_workspace", "gla_error_string", "gla_device_fault", "gla_version")
+            "gla_trim_workspace", "gla_set_workspace_retention", "gla_inject_alloc_failure",
+            "gla_set_wait_limit_ns", "gla_inject_stall", "gla_error_string", "gla_device_fault",
+            "gla_version")
 
 
 class RopeConfig(ctypes.Structure):
@@ -99,6 +101,14 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.gla_trim_workspace.argtypes = []
     lib.gla_trim_workspace.restype = i32
+    lib.gla_set_workspace_retention.argtypes = [ctypes.c_ulonglong]
+    lib.gla_set_workspace_retention.restype = i32
+    lib.gla_inject_alloc_failure.argtypes = [i32]
+    lib.gla_inject_alloc_failure.restype = i32
+    lib.gla_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gla_set_wait_limit_ns.restype = i32
+    lib.gla_inject_stall.argtypes = [ctypes.c_longlong]
+    lib.gla_inject_stall.restype = i32
     lib.gla_error_string.argtypes = [i32]
     lib.gla_error_string.restype = ctypes.c_char_p
     lib.gla_device_fault.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -355,6 +365,36 @@ def gla_trim_workspace() -> None:
     st = load_library().gla_trim_workspace()
     if st != GLA_OK:
         raise GLAError(st, "gla_trim_workspace")
+
+
+def gla_set_workspace_retention(nbytes: int) -> None:
+    """Bytes of freed workspace the current device's pool keeps mapped
+    between calls (default: all of it; 0 returns everything at each
+    synchronisation)."""
+    st = load_library().gla_set_workspace_retention(int(nbytes))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_set_workspace_retention")
+
+
+def gla_inject_alloc_failure(count: int) -> None:
+    """Testing hook: the next `count` workspace allocations fail (GLA_ERR_ALLOC)."""
+    load_library().gla_inject_alloc_failure(int(count))
+
+
+def gla_set_wait_limit_ns(ns: int) -> None:
+    """Testing hook: the kernels' barrier-wait limit on the current device
+    (0 restores the default of one second)."""
+    st = load_library().gla_set_wait_limit_ns(int(ns))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_set_wait_limit_ns")
+
+
+def gla_inject_stall(tile: int) -> None:
+    """Testing hook: the next state-increment launch withholds one tile on its
+    first CTA, so that a wait runs out (see include/gla.h)."""
+    st = load_library().gla_inject_stall(int(tile))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_inject_stall")
 
 
 def gla_error_string(status: int) -> str:

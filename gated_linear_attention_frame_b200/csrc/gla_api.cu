@@ -96,6 +96,32 @@ cudaMemPool_t workspace_pool() {
   }
   return g_pool[dev];
 }
+// gla_inject_alloc_failure (testing): workspace allocations still to fail.
+int g_fail_allocs = 0;
+
+// Stream-ordered workspace of `bytes` from the device's pool; GLA_ERR_ALLOC
+// (nothing enqueued) when the pool cannot provide it.
+int take_workspace(int64_t bytes, cudaStream_t stream, uint8_t** ws) {
+  *ws = nullptr;
+  if (bytes <= 0) return GLA_OK;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_fail_allocs > 0) {
+      --g_fail_allocs;
+      return GLA_ERR_ALLOC;
+    }
+  }
+  cudaMemPool_t pool = workspace_pool();
+  if (pool == nullptr || cudaMallocFromPoolAsync(reinterpret_cast<void**>(ws),
+                                                 static_cast<size_t>(bytes), pool,
+                                                 stream) != cudaSuccess) {
+    cudaGetLastError();
+    *ws = nullptr;
+    return GLA_ERR_ALLOC;
+  }
+  return GLA_OK;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 template <int D>
@@ -326,14 +352,9 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   if (fixed != nullptr) {
     if (static_cast<size_t>(ws_bytes) > fixed->bytes) return GLA_ERR_SCRATCH;
     ws = ws_bytes > 0 ? fixed->ptr : nullptr;
-  } else if (ws_bytes > 0) {
-    cudaMemPool_t pool = workspace_pool();
-    if (pool == nullptr ||
-        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
-                                a.stream) != cudaSuccess) {
-      cudaGetLastError();
-      return GLA_ERR_ALLOC;
-    }
+  } else {
+    const int st = take_workspace(ws_bytes, a.stream, &ws);
+    if (st != GLA_OK) return st;
   }
   float* partial = reinterpret_cast<float*>(ws);
   uint8_t* image = ws ? ws + partial_bytes : nullptr;
@@ -439,14 +460,9 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
     if ((st = encode_map(&tm_out, a.out, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
   }
   uint8_t* ws = nullptr;
-  if (ws_bytes > 0) {
-    cudaMemPool_t pool = workspace_pool();
-    if (pool == nullptr ||
-        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
-                                a.stream) != cudaSuccess) {
-      cudaGetLastError();
-      return GLA_ERR_ALLOC;
-    }
+  {
+    const int st = take_workspace(ws_bytes, a.stream, &ws);
+    if (st != GLA_OK) return st;
   }
   float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
   float* mpartial = W > 0 ? reinterpret_cast<float*>(ws + partial_bytes) : nullptr;
@@ -614,8 +630,9 @@ int validate_bwd(const BwdArgs& a) {
 // The six kernels of the backward pass (d = 128).  The workspace holds the
 // partials (the recompute's increments, then the local state gradients L_f:
 // the forward scan has finished reading the first before the query kernel
-// writes the second), the bf16 images (S_f^T, then G_f^T, likewise), the fp32
-// forward states S_f and the per-warp partial sums of da_f.
+// writes the second), the bf16 images (S_f^T, then the hi part of G_f^T,
+// likewise), the fp32 forward states S_f, the per-warp partial sums of da_f,
+// the lo part of the G_f^T images and the fp32 normaliser rows G_f[:, d].
 int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   constexpr int D = 128;
   using G = Geo<D>;
@@ -631,7 +648,8 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
   const int64_t states_bytes = align256(units * static_cast<int64_t>(PF) * 4);
   const int64_t da_bytes = align256(units * static_cast<int64_t>(RS::kGroups) * 8 * 4);
-  const int64_t ws_bytes = partial_bytes + image_bytes + states_bytes + da_bytes;
+  const int64_t gnorm_bytes = W > 0 ? align256(units * static_cast<int64_t>(D) * 4) : 0;
+  const int64_t ws_bytes = partial_bytes + 2 * image_bytes + states_bytes + da_bytes + gnorm_bytes;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_dout, tm_dq, tm_dk, tm_dv;
   if (W > 0) {
@@ -647,20 +665,17 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
 
   uint8_t* ws = nullptr;
-  if (ws_bytes > 0) {
-    cudaMemPool_t pool = workspace_pool();
-    if (pool == nullptr ||
-        cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), static_cast<size_t>(ws_bytes), pool,
-                                a.stream) != cudaSuccess) {
-      cudaGetLastError();
-      return GLA_ERR_ALLOC;
-    }
+  {
+    const int st = take_workspace(ws_bytes, a.stream, &ws);
+    if (st != GLA_OK) return st;
   }
   float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
   uint8_t* image = W > 0 ? ws + partial_bytes : nullptr;
   float* states = ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes) : nullptr;
   float* da_part =
       ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + states_bytes) : nullptr;
+  uint8_t* image_lo = W > 0 ? ws + partial_bytes + image_bytes + states_bytes + da_bytes : nullptr;
+  float* gnorm = W > 0 ? reinterpret_cast<float*>(image_lo + image_bytes) : nullptr;
 
   int status = GLA_OK;
   auto check = [&]() {
@@ -703,8 +718,8 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(3);
   if (status == GLA_OK && (a.F > 0 || a.ds_in != nullptr)) {
-    gla::ScanBwdParams rp{partial, a.g, states, a.s_in, a.ds_out, a.ds_in, image, da_part, wp,
-                          a.H, a.F, tpu};
+    gla::ScanBwdParams rp{partial, a.g,   states,  a.s_in, a.ds_out, a.ds_in, image,
+                          image_lo, gnorm, da_part, wp,    a.H,      a.F,     tpu};
     const unsigned grid = static_cast<unsigned>(RS::kGroups) * static_cast<unsigned>(a.B * a.H);
     if (launch_dependent(gla::gla_scan_bwd_kernel<D>, grid, RS::kThreads, RS::kSmemBytes,
                          a.stream, rp) != cudaSuccess)
@@ -721,7 +736,7 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(5);
   if (W > 0 && status == GLA_OK) {
-    gla::BwdKVParams kp{image, wp, a.H, a.F, a.T};
+    gla::BwdKVParams kp{image, image_lo, gnorm, wp, a.H, a.F, a.T};
     if (launch_dependent(gla::gla_bwd_kv_kernel<D>, G1, gla::BwdKVCfg<D>::kThreads,
                          gla::BwdKVCfg<D>::kSmemBytes, a.stream, tm_k, tm_v, tm_dk, tm_dv,
                          kp) != cudaSuccess)
@@ -908,6 +923,41 @@ int gla_trim_workspace(void) {
   }
   if (pool == nullptr) return GLA_OK;
   return cudaMemPoolTrimTo(pool, 0) == cudaSuccess ? GLA_OK : GLA_ERR_LAUNCH;
+}
+
+int gla_set_workspace_retention(unsigned long long bytes) {
+  cudaMemPool_t pool = workspace_pool();
+  if (pool == nullptr) return GLA_ERR_DEVICE;
+  uint64_t keep = bytes;
+  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+    cudaGetLastError();
+    return GLA_ERR_LAUNCH;
+  }
+  return GLA_OK;
+}
+
+int gla_set_wait_limit_ns(unsigned long long ns) {
+  const uint64_t v = ns == 0 ? gla::kWaitLimitDefaultNs : static_cast<uint64_t>(ns);
+  if (cudaMemcpyToSymbol(gla::g_gla_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return GLA_ERR_LAUNCH;
+  }
+  return GLA_OK;
+}
+
+int gla_inject_stall(long long tile) {
+  const long long v = tile < 0 ? -1 : tile;
+  if (cudaMemcpyToSymbol(gla::g_gla_stall_tile, &v, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return GLA_ERR_LAUNCH;
+  }
+  return GLA_OK;
+}
+
+int gla_inject_alloc_failure(int count) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_fail_allocs = count > 0 ? count : 0;
+  return GLA_OK;
 }
 
 const char* gla_error_string(int status) {

@@ -4,15 +4,18 @@
 // and S_f = a_f S_{f-1} + phi(K_f)^T [V_f | 1], for every token t of frame f:
 //   dk_t = 1[k_t > 0] * ([v_t | 1] G_f^T)      (d outputs)
 //   dv_t = phi(k_t) G_f[:, :d]                 (d outputs)
-// Per 128-token tile, two contractions into TMEM:
-//   dk~ : A = [v | 1]  [M = 128 tokens, K = d + 16]  K-major; the ones column
-//         is a constant 32-byte-swizzled region used by the last K step;
-//         B = G_f^T image read MN-major          [N = d key features]
-//   dv  : A = phi(k)   [M = 128 tokens, K = d]      K-major (ReLU in smem)
-//         B = G_f^T image read K-major           [N = d value columns]
-// One bf16 image of G_f^T (the scan's swizzled K-major layout, d + 1 rows
-// + 15 zero rows in shared memory) serves both.  The ReLU warps also keep a
-// per-row byte mask of phi(k) > 0 in a small ring for the dk epilogue.
+// The reverse scan hands over G_f as two bf16 images of its value rows, G =
+// G_hi + G_lo (the scan's swizzled K-major layout), and its normaliser row
+// G_f[:, d] in fp32.  Per 128-token tile, two contractions into TMEM:
+//   dk~ : A = v        [M = 128 tokens, K = d]  K-major
+//         B = G_hi^T, then G_lo^T, read MN-major [N = d key features]
+//         (the sum cancels strongly on frames of few tokens, where a single
+//         bf16 copy of G would not hold the tolerance); the epilogue adds the
+//         fp32 normaliser row, the "| 1" column of [v | 1]
+//   dv  : A = phi(k)   [M = 128 tokens, K = d]  K-major (ReLU in smem)
+//         B = G_hi^T read K-major                 [N = d value columns]
+// The ReLU warps also keep a per-row byte mask of phi(k) > 0 in a small ring
+// for the dk epilogue.
 // Warp roles as the forward kernels: 0-3 epilogue, 4-7 ReLU/mask, 8 TMA, 9 MMA.
 #pragma once
 
@@ -27,22 +30,24 @@ struct BwdKVCfg {
   using G = Geo<D>;
   static_assert(D == 128, "the backward kernels are built for d = 128");
   static constexpr int kStages = 2;
-  static constexpr int kStageBytes = 2 * G::kTileBytes;                    // v tile + k tile
-  static constexpr int kGBufBytes = G::kAtoms * G::kNPad * G::kRowBytes;  // G^T image
-  static constexpr int kOnesBytes = kTileTokens * 32;                     // [1 | 0 x 15] rows
+  static constexpr int kStageBytes = 2 * G::kTileBytes;                   // v tile + k tile
+  static constexpr int kGAtomBytes = D * G::kRowBytes;                   // value rows of one atom
+  static constexpr int kGBufBytes = G::kAtoms * kGAtomBytes;             // one part of G^T
   static constexpr int kMaskRing = 4;
-  static constexpr int kMaskBytes = kTileTokens * (D / 8);                // one byte per 8 features
-  static constexpr int kStageOutBytes = G::kAtomTileBytes;
-  static constexpr int kTmemCols = 512;                                   // 2 x (dk~ | dv)
+  static constexpr int kMaskBytes = kTileTokens * (D / 8);               // one byte per 8 features
+  static constexpr int kStageOutBytes = G::kAtomTileBytes;               // one store round
+  static constexpr int kTmemCols = 512;                                  // 2 x (dk~ | dv)
   static constexpr int kThreads = 320;
   static constexpr int kBarCount = 3 * kStages + 2 + 4 + 2 * kMaskRing + 1;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kGBufBytes + kOnesBytes +
-                                    kMaskRing * kMaskBytes + 2 * kStageOutBytes + kBarCount * 8 + 16;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kGBufBytes +
+                                    kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 struct BwdKVParams {
-  const uint8_t* gimage;  // [units][kImageBytes] bf16 G_f^T images
+  const uint8_t* gimage;     // [units][kImageBytes] bf16 G_f^T images, hi part (rows 0..d-1)
+  const uint8_t* gimage_lo;  // [units][kImageBytes] bf16 G_f^T images, lo part (rows 0..d-1)
+  const float* gnorm;        // [units][d] G_f[:, d] in fp32
   WorkPlan wp;
   int H, F, T;
 };
@@ -64,13 +69,11 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t sbase = smem_u32(smem);
   auto v_buf = [&](int s) { return sbase + s * C::kStageBytes; };
   auto k_buf = [&](int s) { return sbase + s * C::kStageBytes + G::kTileBytes; };
-  const uint32_t g_buf = sbase + S * C::kStageBytes;
-  const uint32_t ones_buf = g_buf + C::kGBufBytes;
-  uint8_t* mask_ring = smem + S * C::kStageBytes + C::kGBufBytes + C::kOnesBytes;
-  const uint32_t o_base = ones_buf + C::kOnesBytes + R * C::kMaskBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kGBufBytes +
-                                               C::kOnesBytes + R * C::kMaskBytes +
-                                               2 * C::kStageOutBytes);
+  const uint32_t g_hi = sbase + S * C::kStageBytes;
+  const uint32_t g_lo = g_hi + C::kGBufBytes;
+  const uint32_t o_base = g_lo + C::kGBufBytes;  // output staging (1024-byte aligned)
+  uint8_t* mask_ring = smem + S * C::kStageBytes + 2 * C::kGBufBytes + C::kStageOutBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + R * C::kMaskBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
@@ -110,29 +113,6 @@ __global__ void __launch_bounds__(320, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  {
-    // Zero rows d+1 .. d+15 of the G image buffer and build the ones region:
-    // row t holds bf16 1.0 in column 0 (32-byte swizzle: chunk c of row t sits
-    // at chunk slot c ^ ((t >> 2) & 1)), zeros elsewhere.
-    constexpr int kPadRows = G::kNPad - G::kStateRows;
-    constexpr int kPadChunks = G::kAtoms * kPadRows * (G::kRowBytes / 16);
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int idx = threadIdx.x; idx < kPadChunks; idx += C::kThreads) {
-      const int ch = idx % (G::kRowBytes / 16);
-      const int rr = (idx / (G::kRowBytes / 16)) % kPadRows;
-      const int at = idx / ((G::kRowBytes / 16) * kPadRows);
-      st_shared_v4(g_buf + at * (G::kNPad * G::kRowBytes) + (G::kStateRows + rr) * G::kRowBytes +
-                       ch * 16,
-                   z);
-    }
-    for (int t = threadIdx.x; t < kTileTokens; t += C::kThreads) {
-      const uint32_t row = ones_buf + t * 32;
-      const int slot0 = (t >> 2) & 1;
-      st_shared_v4(row + slot0 * 16, make_uint4(0x3F80u, 0, 0, 0));
-      st_shared_v4(row + (slot0 ^ 1) * 16, z);
-    }
-    fence_proxy_async_smem();
-  }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
@@ -154,12 +134,15 @@ __global__ void __launch_bounds__(320, 1)
         if (cur.first) {
           unit_coords(cur.u, p.H, p.F, b, f, h);
           if (!mbar_wait(gempty, static_cast<uint32_t>((seg & 1) ^ 1), abort, kCode)) break;
-          mbar_arrive_expect_tx(gfull, G::kImageBytes);
-          const uint8_t* src = p.gimage + static_cast<int64_t>(cur.u) * G::kImageBytes;
+          mbar_arrive_expect_tx(gfull, 2u * C::kGBufBytes);
+          const int64_t off = static_cast<int64_t>(cur.u) * G::kImageBytes;
 #pragma unroll
-          for (int a = 0; a < G::kAtoms; ++a)
-            bulk_load(g_buf + a * G::kNPad * G::kRowBytes, src + a * G::kImageAtomBytes,
-                      G::kImageAtomBytes, gfull);
+          for (int a = 0; a < G::kAtoms; ++a) {
+            bulk_load(g_hi + a * C::kGAtomBytes, p.gimage + off + a * G::kImageAtomBytes,
+                      C::kGAtomBytes, gfull);
+            bulk_load(g_lo + a * C::kGAtomBytes, p.gimage_lo + off + a * G::kImageAtomBytes,
+                      C::kGAtomBytes, gfull);
+          }
           ++seg;
         }
         const int s = static_cast<int>(issued % S);
@@ -185,7 +168,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_dk = idesc_bf16_f32(128, D, false, true);   // B MN-major
       constexpr uint32_t idesc_dv = idesc_bf16_f32(128, D, false, false);  // B K-major
       constexpr int KPA = G::kAtomElems / 16;
-      constexpr uint32_t kGAtom = G::kNPad * G::kRowBytes;
+      constexpr uint32_t kGAtom = C::kGAtomBytes;
       int64_t i = 0, seg = 0;
       for (; cur.valid(); cur.advance(), ++i) {
         if (cur.first) {
@@ -198,28 +181,27 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const uint32_t acc_dk = tmem + ab * 256;
         const uint32_t acc_dv = acc_dk + 128;
-        // dk~ = [v | 1] . G^T : K over value columns j (d) plus the ones column
+        // dk~ = v . (G_hi + G_lo)^T : K over the value columns j
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc(v_buf(s) + (kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32,
-                                        16, G::kGroupBytes, G::kLayout);
-          const uint64_t bd = smem_desc(g_buf + kk * 2 * G::kGroupBytes, kGAtom, G::kGroupBytes,
-                                        G::kLayout);
-          mma_bf16(acc_dk, ad, bd, idesc_dk, kk > 0 ? 1u : 0u);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t gb = part == 0 ? g_hi : g_lo;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = smem_desc(
+                v_buf(s) + (kk / KPA) * G::kAtomTileBytes + (kk % KPA) * 32, 16, G::kGroupBytes,
+                G::kLayout);
+            const uint64_t bd =
+                smem_desc(gb + kk * 2 * G::kGroupBytes, kGAtom, G::kGroupBytes, G::kLayout);
+            mma_bf16(acc_dk, ad, bd, idesc_dk, (part > 0 || kk > 0) ? 1u : 0u);
+          }
         }
-        {
-          const uint64_t ad = smem_desc(ones_buf, 16, 256, kLayoutSW32);
-          const uint64_t bd = smem_desc(g_buf + (D / 16) * 2 * G::kGroupBytes, kGAtom,
-                                        G::kGroupBytes, G::kLayout);
-          mma_bf16(acc_dk, ad, bd, idesc_dk, 1u);
-        }
-        // dv = phi(k) . G[:, :d] : K over key features i
+        // dv = phi(k) . G_hi[:, :d] : K over the key features i
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int a = kk / KPA, w = kk % KPA;
           const uint64_t ad = smem_desc(k_buf(s) + a * G::kAtomTileBytes + w * 32, 16,
                                         G::kGroupBytes, G::kLayout);
-          const uint64_t bd = smem_desc(g_buf + a * kGAtom + w * 32, 16, G::kGroupBytes, G::kLayout);
+          const uint64_t bd = smem_desc(g_hi + a * kGAtom + w * 32, 16, G::kGroupBytes, G::kLayout);
           mma_bf16(acc_dv, ad, bd, idesc_dv, kk > 0 ? 1u : 0u);
         }
         mma_commit(empty(s));
@@ -278,6 +260,8 @@ __global__ void __launch_bounds__(320, 1)
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // token within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // G_f[:, d] of the reverse scan
+    const uint32_t stg = o_base;  // this warp stores rows q4*32 .. q4*32+31 of it
     int64_t i = 0;
     int b = 0, f = 0, h = 0;
     for (; cur.valid(); cur.advance(), ++i) {
@@ -288,21 +272,21 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
       const int tok0 = cur.t * kTileTokens + q4 * 32;
+      const float4* gn = reinterpret_cast<const float4*>(p.gnorm + static_cast<int64_t>(cur.u) * D);
       // the row's sign mask
       const uint4 mk = *reinterpret_cast<const uint4*>(mask_ring + m * C::kMaskBytes + row * (D / 8));
       __syncwarp();
       if (lane == 0) mbar_arrive(maskfree(m));
       const uint32_t mwords[4] = {mk.x, mk.y, mk.z, mk.w};
 #pragma unroll
-      for (int out = 0; out < 2; ++out) {  // 0: dk (masked), 1: dv
+      for (int out = 0; out < 2; ++out) {  // 0: dk (normaliser row added, masked), 1: dv
         const uint32_t tb = tmem + lane_base + ab * 256 + out * 128;
         const CUtensorMap* tm = out == 0 ? &tm_dk : &tm_dv;
 #pragma unroll
         for (int a = 0; a < G::kAtoms; ++a) {
-          const int buf = static_cast<int>((i * 2 * G::kAtoms + out * G::kAtoms + a) & 1);
-          const uint32_t stg = o_base + buf * C::kStageOutBytes;
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
+          // TMEM -> bf16 in registers first, so that the wait for the previous
+          // store to leave the staging buffer overlaps the load
+          uint32_t pk[G::kAtomElems / 2];
 #pragma unroll
           for (int cc = 0; cc < G::kAtomElems / 32; ++cc) {
             uint32_t r[32];
@@ -314,18 +298,26 @@ __global__ void __launch_bounds__(320, 1)
               const uint32_t mb = (mwords[col8 >> 2] >> (8 * (col8 & 3))) & 0xFFu;
               float x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                x[e] = __uint_as_float(r[8 * ch + e]);
-                if (out == 0 && ((mb >> e) & 1u) == 0u) x[e] = 0.f;
+              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * ch + e]);
+              if (out == 0) {
+                const float4 g0 = __ldg(gn + 2 * col8), g1 = __ldg(gn + 2 * col8 + 1);
+                x[0] += g0.x; x[1] += g0.y; x[2] += g0.z; x[3] += g0.w;
+                x[4] += g1.x; x[5] += g1.y; x[6] += g1.z; x[7] += g1.w;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (((mb >> e) & 1u) == 0u) x[e] = 0.f;
               }
-              uint4 w;
-              w.x = pack_bf16x2(x[0], x[1]);
-              w.y = pack_bf16x2(x[2], x[3]);
-              w.z = pack_bf16x2(x[4], x[5]);
-              w.w = pack_bf16x2(x[6], x[7]);
-              st_shared_v4(stg + row * G::kRowBytes + G::swz(row, cc * 4 + ch) * 16, w);
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2)
+                pk[(cc * 4 + ch) * 4 + e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
             }
           }
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+#pragma unroll
+          for (int ch = 0; ch < G::kAtomElems / 8; ++ch)
+            st_shared_v4(stg + row * G::kRowBytes + G::swz(row, ch) * 16,
+                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {

@@ -161,6 +161,12 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      // gla_inject_stall (testing): CTA 0 withholds one tile, once
+      long long stall = -1;
+      if (blockIdx.x == 0 && g_gla_stall_tile >= 0) {
+        stall = g_gla_stall_tile;
+        g_gla_stall_tile = -1;
+      }
       int64_t issued = 0;
       int b = 0, f = 0, h = 0;
       for (; cur.valid(); cur.advance(), ++issued) {
@@ -168,6 +174,7 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
         const uint32_t ph = static_cast<uint32_t>((issued / S) & 1);
         if (!mbar_wait(empty(s), ph ^ 1u, abort, kCode)) break;
         if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+        if (issued == stall) continue;  // nothing arrives on full(s) for this tile
         const int t = cur.t;
         mbar_arrive_expect_tx(full(s), 2u * G::kTileBytes);
 #pragma unroll

@@ -9,8 +9,12 @@
 // the same slot layout as the forward increments) and G_f is the total
 // gradient reaching S_f.  From it:
 //   da_f = <G_f, S_{f-1}>  (S_{-1} = state_in),   dstate_in = a_0 G_0,
-// and G_f^T rounded to bf16 is written in the same swizzled K-major image
-// layout as the forward prefix states, for the key/value backward kernel.
+// and G_f^T is written for the key/value backward kernel as two bf16 images
+// in the swizzled K-major layout of the forward prefix states, G = G_hi +
+// G_lo with G_hi = bf16(G) and G_lo = bf16(G - G_hi) (value rows 0..d-1), plus
+// the normaliser row G_f[:, d] in fp32: dk = [v | 1] G^T cancels strongly
+// when a frame has few tokens (out_t then stays near v_t and dk carries
+// dout_t . (v_t - out_t)), so a single bf16 copy of G is not accurate enough.
 //
 // Same structure as the forward scan: a producer warp bulk-copies each
 // frame's partials and S_{f-1} rows (the forward states saved by the
@@ -33,7 +37,9 @@ struct ScanBwdParams {
   const float* state_in;    // [B, H, d, d+1] or nullptr
   const float* dstate_out;  // [B, H, d, d+1] or nullptr
   float* dstate_in;         // [B, H, d, d+1] or nullptr
-  uint8_t* image;           // G_f^T images [units][kImageBytes]
+  uint8_t* image;           // G_f^T images (hi part) [units][kImageBytes], rows 0..d-1
+  uint8_t* image_lo;        // G_f^T images (lo part) [units][kImageBytes], rows 0..d-1
+  float* gnorm;             // G_f[:, d] in fp32 [units][d]
   float* da_part;           // [units][kGroups][8] per-warp partial sums of da_f
   WorkPlan wp;
   int H, F, tpu;
@@ -242,13 +248,25 @@ __global__ void __launch_bounds__(288, 2) gla_scan_bwd_kernel(const ScanBwdParam
           G8[e] = fmaf(a_next, G8[e], L[e]);
           da = fmaf(G8[e], Sp[e], da);
         }
-        uint4 w;
-        w.x = pack_bf16x2(G8[0], G8[1]);
-        w.y = pack_bf16x2(G8[2], G8[3]);
-        w.z = pack_bf16x2(G8[4], G8[5]);
-        w.w = pack_bf16x2(G8[6], G8[7]);
-        if (p.image != nullptr)
-          *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) = w;
+        if (p.image != nullptr) {
+          if (j < D) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi[e] = pack_bf16x2(G8[2 * e], G8[2 * e + 1]);
+              lo[e] = pack_bf16x2(G8[2 * e] - bf16lo_to_f32(hi[e]),
+                                  G8[2 * e + 1] - bf16hi_to_f32(hi[e]));
+            }
+            *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(p.image_lo + u * G::kImageBytes + img_off) =
+                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          } else {
+            float4* gn = reinterpret_cast<float4*>(p.gnorm + u * D + c * 8);
+            gn[0] = make_float4(G8[0], G8[1], G8[2], G8[3]);
+            gn[1] = make_float4(G8[4], G8[5], G8[6], G8[7]);
+          }
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) da += __shfl_xor_sync(0xffffffffu, da, o);

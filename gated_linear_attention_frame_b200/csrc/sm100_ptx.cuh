@@ -64,9 +64,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Longest a kernel waits on one barrier phase before it gives up (a correct
-// launch never comes close: every wait here ends within microseconds).
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// Longest a kernel waits on one barrier phase before it gives up, by default
+// (a correct launch never comes close: every wait here ends within
+// microseconds).  gla_set_wait_limit_ns() changes it per device; the tests
+// lower it to make a withheld wait run out quickly.
+constexpr uint64_t kWaitLimitDefaultNs = 1000000000ull;
+__device__ uint64_t g_gla_wait_limit_ns = kWaitLimitDefaultNs;
+
+// Test hook set by gla_inject_stall(): the next launch of the state-increment
+// kernel withholds, on CTA 0, the loads of this tile of its sequence and
+// their barrier arrival, so that the wait for that tile runs out.  -1: none.
+// The kernel clears it when it takes it.
+__device__ long long g_gla_stall_tile = -1;
 
 // Device-wide fault word of this library (read and cleared by the host).  The
 // library is one translation unit, so the definition lives here.
@@ -80,11 +89,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           unsigned int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = g_gla_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit) {
         *abort = 1;
         atomicOr(&g_gla_fault, code);
         return false;
@@ -97,8 +107,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // before a CTA exits).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = g_gla_wait_limit_ns;
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit) return false;
   }
   return true;
 }

@@ -83,7 +83,8 @@ typedef enum {
  * (per-frame fp32 state increments and bf16 prefix states) from the
  * library's stream-ordered memory pool on `stream` and frees it on the same
  * stream.  The pool (one per device, created at the first call) keeps freed
- * memory mapped for later calls; gla_trim_workspace() returns it.
+ * memory mapped for later calls (gla_set_workspace_retention bounds that);
+ * gla_trim_workspace() returns it.
  * Returns GLA_OK or a gla_status code; on error nothing was enqueued, except
  * GLA_ERR_LAUNCH, after which part of the work may have been enqueued.
  */
@@ -324,13 +325,53 @@ int gla_backward_timed(const void* q, const void* k, const void* v,
  */
 int gla_trim_workspace(void);
 
+/*
+ * gla_set_workspace_retention -- how much freed workspace memory the current
+ * device's pool keeps mapped between calls (its release threshold, bytes).
+ * The default keeps all of it (a later call of the same size then maps
+ * nothing; measured at 720p-60s, 4.72 -> 3.79 ms per call), so after a large
+ * call the pool holds up to that call's workspace (about 0.6 GB at 720p-60s)
+ * until gla_trim_workspace().  A caller that runs its own caching allocator
+ * beside this library can pass 0 (return everything at each synchronisation)
+ * or a budget.  Creates the pool if needed.
+ * Returns GLA_OK, GLA_ERR_DEVICE or GLA_ERR_LAUNCH.
+ */
+int gla_set_workspace_retention(unsigned long long bytes);
+
+/*
+ * Testing hooks for the failure paths (no counterpart in the paper).  They
+ * make the library fail on purpose, without a GPU fault:
+ *
+ * gla_inject_alloc_failure -- the next `count` workspace allocations (of any
+ *   entry point that allocates; not gla_forward_noalloc) fail as if the pool
+ *   had no memory left: the call returns GLA_ERR_ALLOC and enqueues nothing.
+ *   count = 0 disarms it.  Host only.  Returns GLA_OK.
+ *
+ * gla_set_wait_limit_ns -- the time after which a kernel gives up a barrier
+ *   wait on the current device (default one second; ns = 0 restores it).
+ *   Returns GLA_OK or GLA_ERR_LAUNCH.
+ *
+ * gla_inject_stall -- the next launch of the state-increment kernel on the
+ *   current device withholds, on its first CTA, the loads of the tile with
+ *   index `tile` in that CTA's sequence (0 = its first tile), once.  The wait
+ *   for that tile runs out after the wait limit; the kernel then sets bit 0
+ *   of the fault word (gla_device_fault), lets its copies in flight land,
+ *   frees its tensor memory and returns, and that call's outputs are invalid.
+ *   The next call runs normally.  tile < 0 disarms it.
+ *   Returns GLA_OK or GLA_ERR_LAUNCH.
+ */
+int gla_inject_alloc_failure(int count);
+int gla_set_wait_limit_ns(unsigned long long ns);
+int gla_inject_stall(long long tile);
+
 /* Static string for a gla_status code (never NULL). Host only, no CUDA call. */
 const char* gla_error_string(int status);
 
 /*
  * gla_device_fault -- synchronises `stream`, then reads and clears the
  * library's device-side fault word of the current device.  Nonzero means a
- * kernel gave up a bounded wait (about one second) and returned early; its
+ * kernel gave up a bounded wait (about one second unless
+ * gla_set_wait_limit_ns changed it) and returned early; its
  * output is then invalid.  Bit 0: state-increment kernel, bit 1: output
  * kernel, bit 2: forward scan, bit 3: reverse scan, bit 4: key/value
  * gradient kernel, bit 5: query gradient kernel, bit 6: delta-rule scan,

@@ -210,3 +210,9 @@ def test_missing_library_fails_loudly(tmp_path):
 
     with pytest.raises(ImportError):
         load_library(str(tmp_path / "libgla.so"))
+
+
+def test_alloc_failure_hook_is_host_only(lib):
+    # arming and disarming the hook makes no CUDA call (this runs without a GPU)
+    assert lib.gla_inject_alloc_failure(3) == 0
+    assert lib.gla_inject_alloc_failure(0) == 0
