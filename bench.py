@@ -75,9 +75,9 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "720p-5s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
-# DRAM bytes (read + write) per launch from one ncu capture of the full
-# workload (profiles/dram_traffic_720p5s.md), valid only while the kernel's
-# sources are unchanged: the hash of its files must match.
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel on
+# the full workload, valid only while the kernel's sources are unchanged: the
+# hash of its files must match.
 KERNEL_DEPS = {
     "output": ["gla_output.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
     "increment": ["gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
@@ -181,7 +181,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.max_mhz = None
         self.ok = False
@@ -585,6 +585,37 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     return res
 
 
+# The other layer workloads timed beside the headline one by the default run
+# (same --steps / --warmup; the streaming workload as its 64 consecutive calls
+# with the state carried).  The tiny workload is launch-bound: parity only.
+OTHER_WORKLOADS = ("480p-5s", "720p-60s", "stream")
+STREAM_CALLS = 64
+
+
+def workload_summary(r: dict) -> dict:
+    lr = r["layer_roofline"]
+    return {"ms_per_call": r["ms_per_step"], "tokens_per_s": r["value"], "calls": r["steps"],
+            "layer_roofline_ms": lr["roofline_ms"], "layer_roofline_frac": lr["frac"],
+            "kernel_ms": lr["kernel_ms"], "dominant_kernel": r["roofline"]["kernel"],
+            "dominant_kernel_frac": r["roofline"]["frac"],
+            "state_in": r["config"]["state_in"], "clocks": r["clocks"],
+            "device_fault": r["device_fault"]}
+
+
+def run_other_workloads(args, head: dict, dist, rank, local_rank, world) -> dict:
+    """Every layer workload's line (the headline's included) for one JSON key."""
+    out = {head["config"]["workload"]: workload_summary(head)}
+    for name in OTHER_WORKLOADS:
+        a = argparse.Namespace(**vars(args))
+        a.no_e2e = True
+        if name == "stream":
+            a.steps = STREAM_CALLS
+        torch.cuda.empty_cache()
+        out[name] = workload_summary(run_gpu(a, WORKLOADS[name], dist, rank, local_rank, world))
+    out["tiny"] = "parity only (launch-bound)"
+    return out
+
+
 def run_gpu_backward(args, w, dist, rank, local_rank, world):
     """One step = one gla_backward call over one batch of the workload
     (recompute of the forward states, then the five gradient kernels)."""
@@ -874,6 +905,9 @@ def main(argv=None):
                     help="override the workload's frame count (small profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (the default run also times the other layer "
+                         "workloads into the line's 'workloads' key)")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle work for cpu_baseline (0 = skip)")
     args = ap.parse_args(argv)
@@ -897,6 +931,9 @@ def main(argv=None):
             res = run_gpu_anchor(args, w, dist, rank, local_rank, world)
         else:
             res = run_gpu(args, w, dist, rank, local_rank, world)
+            if (args.variant == "plain" and args.workload == DEFAULT_WORKLOAD and args.frames == 0
+                    and not args.no_workloads):
+                res["workloads"] = run_other_workloads(args, res, dist, rank, local_rank, world)
         if rank == 0 and world == 1 and args.cpu_budget > 0:
             res["cpu_baseline"] = (time_oracle_backward(w, args.cpu_budget)
                                    if args.mode == "backward"

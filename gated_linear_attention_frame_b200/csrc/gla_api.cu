@@ -212,8 +212,12 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // 5-D view (d, H, T, F, B) of a bf16 [B, F*T, H, d] tensor; box = one swizzle
 // atom of features x `box_rows` tokens of one head of one frame.
-int encode_map(CUtensorMap* m, const void* base, int d, int H, int T, int F, int B, int box_rows) {
-  const int atom = d >= 64 ? 64 : 32;
+// Tensor map of a bf16 [B, F*T, H, d] tensor with boxes of `box_rows` tokens
+// x `box_cols` features (0: one swizzle atom, 64 features at d >= 64, else
+// 32); 32-feature boxes use the 64-byte swizzle, 64-feature boxes 128-byte.
+int encode_map(CUtensorMap* m, const void* base, int d, int H, int T, int F, int B, int box_rows,
+               int box_cols = 0) {
+  const int atom = box_cols > 0 ? box_cols : (d >= 64 ? 64 : 32);
   const cuuint64_t e = 2;
   cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(F),
@@ -225,7 +229,7 @@ int encode_map(CUtensorMap* m, const void* base, int d, int H, int T, int F, int
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        atom == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GLA_OK : GLA_ERR_LAUNCH;
 }
@@ -632,7 +636,8 @@ int validate_bwd(const BwdArgs& a) {
 // the forward scan has finished reading the first before the query kernel
 // writes the second), the bf16 images (S_f^T, then the hi part of G_f^T,
 // likewise), the fp32 forward states S_f, the per-warp partial sums of da_f,
-// the lo part of the G_f^T images and the fp32 normaliser rows G_f[:, d].
+// the lo parts of the images (S_f^T, then G_f^T) and the fp32 normaliser rows
+// G_f[:, d].
 int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   constexpr int D = 128;
   using G = Geo<D>;
@@ -659,9 +664,10 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
     if ((st = encode_map(&tm_q, a.q, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
     if ((st = encode_map(&tm_k, a.k, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
     if ((st = encode_map(&tm_v, a.v, D, a.H, a.T, a.F, a.B, gla::kTileTokens)) != GLA_OK) return st;
-    if ((st = encode_map(&tm_dq, a.dq, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
-    if ((st = encode_map(&tm_dk, a.dk, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
-    if ((st = encode_map(&tm_dv, a.dv, D, a.H, a.T, a.F, a.B, 32)) != GLA_OK) return st;
+    // gradient stores: 32 tokens x 32 features per warp and round (64-byte swizzle)
+    if ((st = encode_map(&tm_dq, a.dq, D, a.H, a.T, a.F, a.B, 32, 32)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_dk, a.dk, D, a.H, a.T, a.F, a.B, 32, 32)) != GLA_OK) return st;
+    if ((st = encode_map(&tm_dv, a.dv, D, a.H, a.T, a.F, a.B, 32, 32)) != GLA_OK) return st;
   }
 
   uint8_t* ws = nullptr;
@@ -695,7 +701,8 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(1);
   if (status == GLA_OK && a.F > 0) {
-    gla::ScanParams sp{partial, a.g, a.s_in, nullptr, image, states, wp, a.H, a.F, tpu};
+    gla::ScanParams sp{partial, a.g, a.s_in, nullptr, image, states, wp, a.H, a.F, tpu,
+                       nullptr, image_lo};
     using SC1 = gla::ScanCfg<D, 1>;
     using SC3 = gla::ScanCfg<D, 3>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
@@ -709,7 +716,7 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(2);
   if (W > 0 && status == GLA_OK) {
-    gla::BwdQParams qp{image, partial, a.eps, wp, a.H, a.F, a.T};
+    gla::BwdQParams qp{image, image_lo, states, partial, a.eps, wp, a.H, a.F, a.T};
     if (launch_dependent(gla::gla_bwd_q_kernel<D>, G1, gla::BwdQCfg<D>::kThreads,
                          gla::BwdQCfg<D>::kSmemBytes, a.stream, tm_q, tm_dout, tm_dq,
                          qp) != cudaSuccess)

@@ -35,7 +35,11 @@ struct BwdKVCfg {
   static constexpr int kGBufBytes = G::kAtoms * kGAtomBytes;             // one part of G^T
   static constexpr int kMaskRing = 4;
   static constexpr int kMaskBytes = kTileTokens * (D / 8);               // one byte per 8 features
-  static constexpr int kStageOutBytes = G::kAtomTileBytes;               // one store round
+  // dk / dv stores: rounds of 32 tokens x 32 features per warp (64-byte
+  // swizzle, 2 KB), two buffers per warp
+  static constexpr int kRoundCols = 32;
+  static constexpr int kRoundBytes = 32 * kRoundCols * 2;
+  static constexpr int kStageOutBytes = 4 * 2 * kRoundBytes;
   static constexpr int kTmemCols = 512;                                  // 2 x (dk~ | dv)
   static constexpr int kThreads = 320;
   static constexpr int kBarCount = 3 * kStages + 2 + 4 + 2 * kMaskRing + 1;
@@ -71,7 +75,7 @@ __global__ void __launch_bounds__(320, 1)
   auto k_buf = [&](int s) { return sbase + s * C::kStageBytes + G::kTileBytes; };
   const uint32_t g_hi = sbase + S * C::kStageBytes;
   const uint32_t g_lo = g_hi + C::kGBufBytes;
-  const uint32_t o_base = g_lo + C::kGBufBytes;  // output staging (1024-byte aligned)
+  const uint32_t o_base = g_lo + C::kGBufBytes;  // output staging: 2 rounds per epilogue warp
   uint8_t* mask_ring = smem + S * C::kStageBytes + 2 * C::kGBufBytes + C::kStageOutBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + R * C::kMaskBytes);
   const uint32_t bar0 = smem_u32(bars);
@@ -261,7 +265,6 @@ __global__ void __launch_bounds__(320, 1)
     const int row = q4 * 32 + lane;  // token within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     asm volatile("griddepcontrol.wait;" ::: "memory");  // G_f[:, d] of the reverse scan
-    const uint32_t stg = o_base;  // this warp stores rows q4*32 .. q4*32+31 of it
     int64_t i = 0;
     int b = 0, f = 0, h = 0;
     for (; cur.valid(); cur.advance(), ++i) {
@@ -283,46 +286,41 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t tb = tmem + lane_base + ab * 256 + out * 128;
         const CUtensorMap* tm = out == 0 ? &tm_dk : &tm_dv;
 #pragma unroll
-        for (int a = 0; a < G::kAtoms; ++a) {
-          // TMEM -> bf16 in registers first, so that the wait for the previous
-          // store to leave the staging buffer overlaps the load
-          uint32_t pk[G::kAtomElems / 2];
+        for (int cc = 0; cc < D / C::kRoundCols; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(tb + cc * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-          for (int cc = 0; cc < G::kAtomElems / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld_32cols(tb + a * G::kAtomElems + cc * 32, r);
-            tmem_wait_ld();
+          for (int ch = 0; ch < 4; ++ch) {
+            const int col8 = cc * 4 + ch;  // 8-feature chunk index
+            const uint32_t mb = (mwords[col8 >> 2] >> (8 * (col8 & 3))) & 0xFFu;
+            float x[8];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              const int col8 = (a * G::kAtomElems + cc * 32) / 8 + ch;  // 8-feature chunk index
-              const uint32_t mb = (mwords[col8 >> 2] >> (8 * (col8 & 3))) & 0xFFu;
-              float x[8];
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * ch + e]);
+            if (out == 0) {
+              const float4 g0 = __ldg(gn + 2 * col8), g1 = __ldg(gn + 2 * col8 + 1);
+              x[0] += g0.x; x[1] += g0.y; x[2] += g0.z; x[3] += g0.w;
+              x[4] += g1.x; x[5] += g1.y; x[6] += g1.z; x[7] += g1.w;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * ch + e]);
-              if (out == 0) {
-                const float4 g0 = __ldg(gn + 2 * col8), g1 = __ldg(gn + 2 * col8 + 1);
-                x[0] += g0.x; x[1] += g0.y; x[2] += g0.z; x[3] += g0.w;
-                x[4] += g1.x; x[5] += g1.y; x[6] += g1.z; x[7] += g1.w;
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  if (((mb >> e) & 1u) == 0u) x[e] = 0.f;
-              }
-#pragma unroll
-              for (int e2 = 0; e2 < 4; ++e2)
-                pk[(cc * 4 + ch) * 4 + e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
+              for (int e = 0; e < 8; ++e)
+                if (((mb >> e) & 1u) == 0u) x[e] = 0.f;
             }
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) pk[ch * 4 + e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
           }
-          if (lane == 0) bulk_wait_group_read<0>();
+          const int rnd = out * (D / C::kRoundCols) + cc;
+          const uint32_t stg = o_base + q4 * 2 * C::kRoundBytes + (rnd & 1) * C::kRoundBytes;
+          if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
 #pragma unroll
-          for (int ch = 0; ch < G::kAtomElems / 8; ++ch)
-            st_shared_v4(stg + row * G::kRowBytes + G::swz(row, ch) * 16,
+          for (int ch = 0; ch < 4; ++ch)  // 64-byte swizzle: chunk ch of row lane
+            st_shared_v4(stg + lane * 64 + ((ch ^ ((lane >> 1) & 3)) * 16),
                          make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (tok0 < p.T)
-              tma_store_5d(tm, stg + q4 * 32 * G::kRowBytes, a * G::kAtomElems, h, tok0, f, b);
+            if (tok0 < p.T) tma_store_5d(tm, stg, cc * C::kRoundCols, h, tok0, f, b);
             bulk_commit_group();
           }
         }

@@ -11,7 +11,8 @@
 //     (one per CTA that owned some of the unit's tiles),
 //   * updates S in registers,
 //   * writes S_f^T rounded to bf16 into the swizzled K-major image that the
-//     output kernel bulk-copies into shared memory as its B operand.
+//     output kernel bulk-copies into shared memory as its B operand (and, for
+//     the backward pass, the bf16 rounding of the remainder in a second image).
 // After the last frame it writes state_out in the caller's [d][d+1] layout.
 // A producer warp streams each frame's partial increments into a ring of
 // shared-memory stages with plain bulk copies (one copy per partial: the
@@ -39,6 +40,8 @@ struct ScanParams {
   WorkPlan wp;             // increment kernel's tile assignment (valid if tpu > 0)
   int H, F, tpu;
   float* zvec;             // [units][d] fp32 S_f[:, d] per frame, or nullptr (rotary variant)
+  uint8_t* image_lo;       // [units][kImageBytes] bf16(S_f - bf16(S_f))^T, value rows 0..d-1,
+                           // or nullptr (backward: the query kernel's dq contraction)
 };
 
 template <int D, int kStagesT = 3>
@@ -219,6 +222,14 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
           w.z = pack_bf16x2(S8[4], S8[5]);
           w.w = pack_bf16x2(S8[6], S8[7]);
           *reinterpret_cast<uint4*>(p.image + u * G::kImageBytes + img_off) = w;
+          if (p.image_lo != nullptr && j < D) {
+            uint4 l;
+            l.x = pack_bf16x2(S8[0] - bf16lo_to_f32(w.x), S8[1] - bf16hi_to_f32(w.x));
+            l.y = pack_bf16x2(S8[2] - bf16lo_to_f32(w.y), S8[3] - bf16hi_to_f32(w.y));
+            l.z = pack_bf16x2(S8[4] - bf16lo_to_f32(w.z), S8[5] - bf16hi_to_f32(w.z));
+            l.w = pack_bf16x2(S8[6] - bf16lo_to_f32(w.w), S8[7] - bf16hi_to_f32(w.w));
+            *reinterpret_cast<uint4*>(p.image_lo + u * G::kImageBytes + img_off) = l;
+          }
         }
         if (p.zvec != nullptr && j == D) {
           float4* dst = reinterpret_cast<float4*>(p.zvec + u * D + c * 8);

@@ -106,6 +106,13 @@ SMALL = [
     # most there (out_t stays near v_t), the case that needs G_f in hi/lo parts
     (1, 1, 3, 1, True, True),
     (1, 2, 6, 3, True, False),
+    # from a zero state dq cancels exactly in the first frame of one-token
+    # frames (out = v there, whatever q): the case that needs dq from dout
+    # against S_f in hi/lo parts
+    (1, 2, 3, 1, False, True),
+    (1, 1, 5, 1, False, False),
+    (1, 3, 3, 2, False, True),
+    (1, 4, 2, 2, False, False),
     (1, 2, 5, 300, False, True),
     (1, 1, 2, 700, True, False),
     (1, 3, 4, 64, True, True),

@@ -103,10 +103,10 @@ def test_alloc_failure_returns_status_and_enqueues_nothing(gla):
 
 @pytest.mark.parametrize("tile", [0, 1])
 def test_wait_that_runs_out_is_reported_and_recovered(gla, tile):
-    # 2 heads x 3 frames x 300 tokens = 18 tiles on 18 CTAs (one each); with
-    # 4 heads x 3 frames x 700 tokens CTA 0 holds several tiles, so tile 1 is
-    # a later one of its sequence
-    w, host_in, dev_in = _case(H=2 if tile == 0 else 4, T=300 if tile == 0 else 700)
+    # 2 heads x 3 frames x 300 tokens: 18 tiles on 18 CTAs, one each; 24 heads
+    # x 3 frames x 700 tokens: 432 tiles on (at most) 148 CTAs, so CTA 0 holds
+    # two or more and tile 1 is a later one of its sequence
+    w, host_in, dev_in = _case(H=2 if tile == 0 else 24, T=300 if tile == 0 else 700)
     try:
         gla.gla_set_wait_limit_ns(5_000_000)  # 5 ms
         gla.gla_inject_stall(tile)
