@@ -794,6 +794,40 @@ def run_gpu_anchor(args, w, dist, rank, local_rank, world):
 
         e2e = e2e_pipelined(dev, stream, dist, world, host_in, [out], call,
                             max(2, min(K, args.e2e_steps)), w.total_tokens)
+    # One rollout step (gla_softmax_anchor_step): the last frame from its sink
+    # and window caches, the same K step / warm-up counts, events around them.
+    fl = w.frames - 1
+    lo = max(0, fl - W + 1)
+    rows = slice(fl * T, (fl + 1) * T)
+    qs, ks, vs, zs = (x[:, rows].contiguous() for x in (q, k, v, z))
+    sk, sv = k[:, :T].contiguous(), v[:, :T].contiguous()
+    wk = k[:, lo * T:fl * T].contiguous() if fl > lo else None
+    wv = v[:, lo * T:fl * T].contiguous() if fl > lo else None
+    os_ = torch.empty_like(qs)
+
+    def rstep():
+        gla.gla_softmax_anchor_step(qs, ks, vs, zs, sk, sv, wk, wv, os_, w.B, w.H, T, w.d, fl, W, T,
+                                    stream)
+
+    for _ in range(warm):
+        rstep()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    t0.record(stream)
+    for _ in range(K):
+        rstep()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_r = reduce_max(t0.elapsed_time(t1), dist, dev) / K
+    keys_r = min(T, lo * T) + (fl + 1 - lo) * T
+    flops_r = 4 * w.d * w.B * w.H * T * keys_r
+    rollout = {"call": "gla_softmax_anchor_step", "frame": fl, "keys_per_query": keys_r,
+               "ms_per_step": round(ms_r, 5),
+               "tokens_per_s": round(world * w.B * T / (ms_r * 1e-3), 1),
+               "achieved_tflops": round(flops_r / (ms_r * 1e-3) / 1e12, 1),
+               "frac": round(flops_r / (ms_r * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+               "device_fault": gla.gla_device_fault(stream)}
     return {
         "metric": metric_for("forward", "softmax"), "value": round(world * w.total_tokens /
                                                                  (ms_step * 1e-3), 1),
@@ -806,7 +840,7 @@ def run_gpu_anchor(args, w, dist, rank, local_rank, world):
                    "l2": "inputs larger than L2; no flush",
                    "parallelism": "dp%d (independent sequences per GPU)" % world},
         "roofline": roof, "layer_roofline": layer, "gpu_launches": K, "e2e": e2e,
-        "clocks": clocks.summary(), "device_fault": fault,
+        "clocks": clocks.summary(), "device_fault": fault, "rollout_step": rollout,
         "gpu": torch.cuda.get_device_name(dev),
     }
 

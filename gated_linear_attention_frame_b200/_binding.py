@@ -28,7 +28,7 @@ GLA_ERR_ROPE = 9
 
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
             "gla_forward_rope", "gla_forward_rope_timed", "gla_forward_gdn", "gla_forward_gdn_timed",
-            "gla_softmax_anchor", "gla_softmax_anchor_timed",
+            "gla_softmax_anchor", "gla_softmax_anchor_timed", "gla_softmax_anchor_step",
             "gla_backward", "gla_backward_timed",
             "gla_trim_workspace", "gla_set_workspace_retention", "gla_inject_alloc_failure",
             "gla_set_wait_limit_ns", "gla_inject_stall", "gla_error_string", "gla_device_fault",
@@ -82,6 +82,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_softmax_anchor.restype = i32
     lib.gla_softmax_anchor_timed.argtypes = anc + [ctypes.POINTER(vp)]
     lib.gla_softmax_anchor_timed.restype = i32
+    lib.gla_softmax_anchor_step.argtypes = [vp] * 9 + [i32] * 7 + [vp]
+    lib.gla_softmax_anchor_step.restype = i32
     gdn = fwd[:4] + [vp] + fwd[4:]
     lib.gla_forward_gdn.argtypes = gdn
     lib.gla_forward_gdn.restype = i32
@@ -241,6 +243,35 @@ def softmax_anchor(q, k, v, frames, window_frames, n_sink=0, gate_z=None, out=No
     if out is None:
         out = torch.empty_like(q)
     gla_softmax_anchor(q, k, v, gate_z, out, B, H, frames, T, d, window_frames, n_sink, stream)
+    return out
+
+
+def gla_softmax_anchor_step(q, k, v, gate_z, sink_k, sink_v, win_k, win_v, out, B, H,
+                            tokens_per_frame, d, frame, window_frames, n_sink,
+                            stream=None) -> None:
+    """The softmax anchor layer for one new frame of a rollout, from the sink
+    and window caches (see include/gla.h; d = 128)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("gate_z", gate_z), ("sink_k", sink_k),
+                    ("sink_v", sink_v), ("win_k", win_k), ("win_v", win_v), ("out", out)):
+        if isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+            raise TypeError("gla: %s must be torch.bfloat16, got %s" % (name, t.dtype))
+    st = load_library().gla_softmax_anchor_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(sink_k), _ptr(sink_v), _ptr(win_k),
+        _ptr(win_v), _ptr(out), int(B), int(H), int(tokens_per_frame), int(d), int(frame),
+        int(window_frames), int(n_sink), _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_softmax_anchor_step")
+
+
+def softmax_anchor_step(q, k, v, frame, window_frames, n_sink=0, sink_k=None, sink_v=None,
+                        win_k=None, win_v=None, gate_z=None, out=None, stream=None):
+    """Convenience wrapper of gla_softmax_anchor_step: q, k, v [B, T, H, d] of
+    frame `frame`; returns out."""
+    B, T, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    gla_softmax_anchor_step(q, k, v, gate_z, sink_k, sink_v, win_k, win_v, out, B, H, T, d,
+                            frame, window_frames, n_sink, stream)
     return out
 
 

@@ -341,6 +341,9 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   }
   const int64_t table_bytes = align256(table_pairs * 8);
   const int64_t zvec_bytes = (kRope && W > 0) ? align256(units * static_cast<int64_t>(D) * 4) : 0;
+  // single frame, plain layer: the increment kernel folds the scan step for
+  // the units it owns whole; the scan runs over the split units alone
+  const bool fold = !kRope && a.F == 1 && W > 0;
   const int64_t ws_bytes = partial_bytes + image_bytes + table_bytes + zvec_bytes;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_out;
@@ -367,6 +370,7 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   float* zvec = zvec_bytes > 0
                     ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + table_bytes)
                     : nullptr;
+
   rg.table = reinterpret_cast<const float4*>(table);
 
   int status = GLA_OK;
@@ -388,17 +392,28 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   }
   if (W > 0 && status == GLA_OK) {
     gla::IncParams ip{partial, wp, a.H, a.F, a.T, rg};
+    if (fold) {
+      ip.fold = 1;
+      ip.gate = a.g;
+      ip.state_in = a.s_in;
+      ip.state_out = a.s_out;
+      ip.image = image;
+    }
     gla::gla_increment_kernel<D, kRope>
         <<<G1, gla::IncCfg<D, kRope>::kThreads, gla::IncCfg<D, kRope>::kSmemBytes, a.stream>>>(
             tm_k, tm_v, ip);
     check();
   }
   record(1);
-  if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
+  // (b, h) pairs the scan covers: all, or with the fold the split units only
+  const int32_t bh0 = fold ? wp.full_units() : 0;
+  const int64_t nbh = static_cast<int64_t>(a.B) * a.H - bh0;
+  if (status == GLA_OK && nbh > 0 && (a.F > 0 || a.s_out != nullptr)) {
     gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu, zvec};
+    sp.bh0 = bh0;
     using SC1 = gla::ScanCfg<D, 1>;
     using SC3 = gla::ScanCfg<D, 3>;
-    const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
+    const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(nbh);
     const cudaError_t e =
         a.F <= 1 ? launch_dependent(gla::gla_scan_kernel<D, 1>, grid, SC1::kThreads,
                                     SC1::kSmemBytes, a.stream, sp)
@@ -768,9 +783,16 @@ int backward_impl(const BwdArgs& a, cudaEvent_t* ev) {
 }
 
 // The softmax anchor layer (d = 128).
+// A rollout step of the anchor layer: the sink and window caches (see
+// gla_softmax_anchor_step).  nullptr: a call over the whole sequence.
+struct AnchorStep {
+  const void *sink_k, *sink_v, *win_k, *win_v;
+  int frame;
+};
+
 int anchor_impl(const void* q, const void* k, const void* v, const void* z, void* out, int B,
                 int H, int F, int T, int d, int window, int n_sink, cudaStream_t stream,
-                cudaEvent_t* ev) {
+                cudaEvent_t* ev, const AnchorStep* step = nullptr) {
   if (d != 128) return GLA_ERR_UNSUPPORTED_D;
   Args chk{q, k, v, nullptr, nullptr, nullptr, out, B, H, F, T, d, 0.f, stream};
   const int64_t units0 = static_cast<int64_t>(B) * F * H;
@@ -780,6 +802,23 @@ int anchor_impl(const void* q, const void* k, const void* v, const void* z, void
   if (st != GLA_OK) return st;
   if (window < 1 || n_sink < 0) return GLA_ERR_SHAPE;
   if (z != nullptr && !aligned(z, 16)) return GLA_ERR_ALIGN;
+  // rollout step: the frames of the window before this one come from the
+  // window cache, the sink tokens that precede the window from the sink cache
+  int win_frames = 0, sinks = 0;
+  if (step != nullptr) {
+    if (step->frame < 0) return GLA_ERR_SHAPE;
+    win_frames = step->frame < window - 1 ? step->frame : window - 1;
+    const int64_t w_lo = static_cast<int64_t>(step->frame - win_frames) * T;
+    sinks = static_cast<int>(n_sink < w_lo ? n_sink : w_lo);
+    if (static_cast<int64_t>(B) * H * T > 0) {
+      if (win_frames > 0 && (step->win_k == nullptr || step->win_v == nullptr))
+        return GLA_ERR_NULL;
+      if (sinks > 0 && (step->sink_k == nullptr || step->sink_v == nullptr)) return GLA_ERR_NULL;
+      if ((win_frames > 0 && (!aligned(step->win_k, 16) || !aligned(step->win_v, 16))) ||
+          (sinks > 0 && (!aligned(step->sink_k, 16) || !aligned(step->sink_v, 16))))
+        return GLA_ERR_ALIGN;
+    }
+  }
   const int tpf = (T + gla::kTileTokens - 1) / gla::kTileTokens;
   const int64_t units = units0 * tpf;
   if (units > INT32_MAX) return GLA_ERR_SHAPE;
@@ -793,14 +832,38 @@ int anchor_impl(const void* q, const void* k, const void* v, const void* z, void
   if ((st = encode_map(&tm_z, z != nullptr ? z : q, d, H, T, F, B, gla::kTileTokens)) != GLA_OK)
     return st;
   if ((st = encode_map(&tm_out, out, d, H, T, F, B, 32)) != GLA_OK) return st;
-  gla::AnchorParams ap{H, F, T, window, n_sink, static_cast<int>(units),
-                       static_cast<float>(1.4426950408889634 / std::sqrt(128.0)), z != nullptr};
+  gla::AnchorCaches caches;  // a whole-sequence call never reads them
+  caches.ks = caches.vs = caches.kw = caches.vw = tm_k;
+  if (step != nullptr) {
+    if (sinks > 0 &&
+        ((st = encode_map(&caches.ks, step->sink_k, d, H, n_sink, 1, B, gla::kTileTokens)) !=
+             GLA_OK ||
+         (st = encode_map(&caches.vs, step->sink_v, d, H, n_sink, 1, B, gla::kTileTokens)) !=
+             GLA_OK))
+      return st;
+    if (win_frames > 0 &&
+        ((st = encode_map(&caches.kw, step->win_k, d, H, T, win_frames, B, gla::kTileTokens)) !=
+             GLA_OK ||
+         (st = encode_map(&caches.vw, step->win_v, d, H, T, win_frames, B, gla::kTileTokens)) !=
+             GLA_OK))
+      return st;
+  }
+  gla::AnchorParams ap{H,
+                       F,
+                       T,
+                       window,
+                       n_sink,
+                       static_cast<int>(units),
+                       static_cast<float>(1.4426950408889634 / std::sqrt(128.0)),
+                       z != nullptr,
+                       step != nullptr,
+                       step != nullptr ? step->frame : 0};
   const int grid = static_cast<int>(units < di.sms ? units : di.sms);
   int status = GLA_OK;
   if (ev != nullptr && cudaEventRecord(ev[0], stream) != cudaSuccess) return GLA_ERR_LAUNCH;
   gla::gla_softmax_anchor_kernel<128>
       <<<grid, gla::AnchorCfg<128>::kThreads, gla::AnchorCfg<128>::kSmemBytes, stream>>>(
-          tm_q, tm_k, tm_v, tm_z, tm_out, ap);
+          tm_q, tm_k, tm_v, tm_z, tm_out, caches, ap);
   if (cudaGetLastError() != cudaSuccess) status = GLA_ERR_LAUNCH;
   if (ev != nullptr && status == GLA_OK && cudaEventRecord(ev[1], stream) != cudaSuccess)
     status = GLA_ERR_LAUNCH;
@@ -853,6 +916,16 @@ int gla_softmax_anchor_timed(const void* q, const void* k, const void* v, const 
   if (events == nullptr) return GLA_ERR_NULL;
   return anchor_impl(q, k, v, gate_z, out, B, H, frames, tokens_per_frame, d, window_frames,
                      n_sink, stream, events);
+}
+
+int gla_softmax_anchor_step(const void* q, const void* k, const void* v, const void* gate_z,
+                            const void* sink_k, const void* sink_v, const void* win_k,
+                            const void* win_v, void* out, int B, int H, int tokens_per_frame,
+                            int d, int frame, int window_frames, int n_sink,
+                            cudaStream_t stream) {
+  const AnchorStep st{sink_k, sink_v, win_k, win_v, frame};
+  return anchor_impl(q, k, v, gate_z, out, B, H, 1, tokens_per_frame, d, window_frames, n_sink,
+                     stream, nullptr, &st);
 }
 
 int gla_forward_gdn(const void* q, const void* k, const void* v, const float* gate_logits,

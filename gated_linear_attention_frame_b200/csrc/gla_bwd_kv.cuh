@@ -43,8 +43,10 @@ struct BwdKVCfg {
   static constexpr int kTmemCols = 512;                                  // 2 x (dk~ | dv)
   static constexpr int kThreads = 320;
   static constexpr int kBarCount = 3 * kStages + 2 + 4 + 2 * kMaskRing + 1;
+  static constexpr int kGNormBytes = 4 * D * 4;  // a private copy of G_f[:, d] per epilogue warp
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kGBufBytes +
-                                    kStageOutBytes + kMaskRing * kMaskBytes + kBarCount * 8 + 16;
+                                    kStageOutBytes + kMaskRing * kMaskBytes + kGNormBytes +
+                                    kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -77,7 +79,8 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t g_lo = g_hi + C::kGBufBytes;
   const uint32_t o_base = g_lo + C::kGBufBytes;  // output staging: 2 rounds per epilogue warp
   uint8_t* mask_ring = smem + S * C::kStageBytes + 2 * C::kGBufBytes + C::kStageOutBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + R * C::kMaskBytes);
+  float* gnorm_s = reinterpret_cast<float*>(mask_ring + R * C::kMaskBytes);  // [4][D]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mask_ring + R * C::kMaskBytes + C::kGNormBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
@@ -273,9 +276,17 @@ __global__ void __launch_bounds__(320, 1)
       if (!warp_wait(accf(ab), static_cast<uint32_t>((i >> 1) & 1), abort, kCode)) break;
       if (!warp_wait(maskfull(m), static_cast<uint32_t>((i / R) & 1), abort, kCode)) break;
       tc_fence_after();
-      if (cur.first) unit_coords(cur.u, p.H, p.F, b, f, h);
+      float* gw = gnorm_s + q4 * D;  // this warp's copy of the unit's G_f[:, d]
+      if (cur.first) {
+        unit_coords(cur.u, p.H, p.F, b, f, h);
+        __syncwarp();  // the previous unit's reads of the copy are done
+        for (int c = lane; c < D / 4; c += 32)
+          reinterpret_cast<float4*>(gw)[c] =
+              __ldg(reinterpret_cast<const float4*>(p.gnorm + static_cast<int64_t>(cur.u) * D) + c);
+        __syncwarp();
+      }
       const int tok0 = cur.t * kTileTokens + q4 * 32;
-      const float4* gn = reinterpret_cast<const float4*>(p.gnorm + static_cast<int64_t>(cur.u) * D);
+      const float4* gn = reinterpret_cast<const float4*>(gw);
       // the row's sign mask
       const uint4 mk = *reinterpret_cast<const uint4*>(mask_ring + m * C::kMaskBytes + row * (D / 8));
       __syncwarp();
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * ch + e]);
             if (out == 0) {
-              const float4 g0 = __ldg(gn + 2 * col8), g1 = __ldg(gn + 2 * col8 + 1);
+              const float4 g0 = gn[2 * col8], g1 = gn[2 * col8 + 1];
               x[0] += g0.x; x[1] += g0.y; x[2] += g0.z; x[3] += g0.w;
               x[4] += g1.x; x[5] += g1.y; x[6] += g1.z; x[7] += g1.w;
 #pragma unroll

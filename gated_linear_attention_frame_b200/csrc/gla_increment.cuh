@@ -47,7 +47,10 @@ struct IncCfg {
   static constexpr int kThreads = (kReluWarps + 6) * 32;        // + epilogue, TMA, MMA warps
   static constexpr int kBarBytes = (3 * kStages + 7) * 8;
   static constexpr int kZBytes = kReluWarps * D * 4;  // per-ReLU-warp normaliser sums
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kZBytes + kBarBytes + 16;
+  // single-frame fold (plain layer): a 32 x 33 fp32 transpose tile per epilogue warp
+  static constexpr int kFoldBytes = (!kRope && !kGram) ? 4 * 32 * 33 * 4 : 0;
+  static constexpr int kSmemBytes =
+      1024 + kStages * kStageBytes + kZBytes + kFoldBytes + kBarBytes + 16;
 };
 
 struct IncParams {
@@ -58,6 +61,16 @@ struct IncParams {
   RopeGeo rope;     // rotary variant only
   float* mpartial;  // Gram variant: [(units + gridDim.x) slots][d][d] fp32 partials of
                     // M_f = phi(K_f)^T phi(K_f), rows as the increment partials
+  // Single-frame calls of the plain layer (fold = 1): for a unit owned whole
+  // by one CTA the scan's step S = a S_in + dS is done here, from TMEM, at the
+  // unit's end (overlapping the CTA's next tiles); a unit whose tiles are
+  // split over several CTAs writes its partials as usual, and the scan runs
+  // over those units alone.
+  int fold;
+  const float* gate;        // [B, 1, H] gate logits
+  const float* state_in;    // [B, H, d, d+1] or nullptr (zero state)
+  float* state_out;         // [B, H, d, d+1] or nullptr (not written; may alias state_in)
+  uint8_t* image;           // [units][kImageBytes] bf16 S^T images for the output kernel
 };
 
 // (b, f, h) of unit u = (b * F + f) * H + h.
@@ -102,7 +115,9 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   float* zpart = reinterpret_cast<float*>(smem + S * C::kStageBytes);  // [RW][D]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kZBytes);
+  float* fold_t = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kZBytes);  // [4][32][33]
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kZBytes + C::kFoldBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto relu_done = [&](int s) { return bar0 + 8u * (S + s); };
@@ -111,7 +126,7 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
   auto acce = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (3 * S + 4);
   const uint32_t zfull = bar0 + 8u * (3 * S + 5);  // the ReLU warps wrote zpart
-  const uint32_t zfree = bar0 + 8u * (3 * S + 6);  // warp 4 consumed zpart
+  const uint32_t zfree = bar0 + 8u * (3 * S + 6);  // warp 4 and the epilogue consumed zpart
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 7);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto a_buf = [&](int s) { return sbase + s * C::kStageBytes; };
@@ -134,7 +149,7 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
     }
     mbar_init(done_bar, 1);
     mbar_init(zfull, RW);
-    mbar_init(zfree, 1);
+    mbar_init(zfree, 5);
     *abort = 0;
     fence_mbar_init();
   }
@@ -299,13 +314,15 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
         if (lane == 0) mbar_arrive(zfull);
         if (warp == 4) {
           if (!warp_wait(zfull, zround & 1u, abort, kCode)) break;
-          float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) +
-                       static_cast<int64_t>(D) * D;
-          for (int col = lane; col < D; col += 32) {
-            float zs = zpart[col];
+          if (!p.fold) {  // (a folding epilogue takes the sums itself)
+            float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) +
+                         static_cast<int64_t>(D) * D;
+            for (int col = lane; col < D; col += 32) {
+              float zs = zpart[col];
 #pragma unroll
-            for (int w = 1; w < RW; ++w) zs += zpart[w * D + col];
-            dst[col] = zs;
+              for (int w = 1; w < RW; ++w) zs += zpart[w * D + col];
+              dst[col] = zs;
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(zfree);
@@ -319,18 +336,132 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
     // ------------------------------------------------------------- epilogue
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // key feature i
+    const bool has_row = q4 * 32 < D;
     int64_t seg = 0;
     for (; cur.valid(); cur.advance()) {
+      if (!kRope && !kGram && p.fold && cur.first && cur.u < cur.U_full && has_row &&
+          p.state_in != nullptr) {
+        // a unit folded here: bring this warp's 32 state rows (16.5 KB) into
+        // L2 while the unit's tiles stream, so that the fold reads them there
+        int b, f, h;
+        unit_coords(cur.u, p.H, p.F, b, f, h);
+        const char* rows = reinterpret_cast<const char*>(
+            p.state_in + (static_cast<int64_t>(b) * p.H + h) * D * (D + 1) +
+            static_cast<int64_t>(q4 * 32) * (D + 1));
+        for (int l = lane; l * 128 < 32 * (D + 1) * 4; l += 32)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rows + l * 128));
+      }
       if (!cur.last) continue;
       const int ab = static_cast<int>(seg & 1);
       if (!warp_wait(accf(ab), static_cast<uint32_t>((seg >> 1) & 1), abort, kCode)) break;
       tc_fence_after();
-      if (q4 * 32 < D) {
-        float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) + row;
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * AC;
+      float* dst = p.partial + cur.slot() * static_cast<int64_t>(C::kPartialFloats) + row;
+      if (!kRope && !kGram && p.fold) {
+        // ---- single frame: S = a S_in + dS for this CTA's units
+        if (!warp_wait(zfull, static_cast<uint32_t>(seg & 1), abort, kCode)) break;
+        float zs = 0.f;  // the normaliser column's entry of this key feature
+        if (has_row) {
+          zs = zpart[row];
+#pragma unroll
+          for (int w = 1; w < RW; ++w) zs += zpart[w * D + row];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zfree);
+        const int32_t u = cur.u;
+        int b, f, h;
+        unit_coords(u, p.H, p.F, b, f, h);
+        const float a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));  // frame 0: gate index u
+        // this warp's 32 key features i0 .. i0 + 31 of state (b, h), [d][d+1]
+        const int64_t sbase = (static_cast<int64_t>(b) * p.H + h) * D * (D + 1) +
+                              static_cast<int64_t>(q4 * 32) * (D + 1);
+        uint8_t* img = p.image + static_cast<int64_t>(u) * G::kImageBytes +
+                       (row / G::kAtomElems) * G::kImageAtomBytes + (row % 8) * 2;
+        const int cin = (row % G::kAtomElems) / 8;
+        float* tt = fold_t + q4 * 32 * 33;  // [32][33]: a 32 x 32 block, padded
+        // one block of 32 value columns j0 ..: this thread holds dS[i0 + lane][j0 + c]
+        // in dv[c]; S = a S_in + dS through the transpose tile so that state_in
+        // and state_out move along their rows (lane = column) and the image
+        // along its rows (lane = key feature)
+        auto fold_block = [&](int j0, const float (&dv)[32]) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) tt[lane * 33 + c] = dv[c];
+          __syncwarp();
+          // the 32 state_in loads of the block in flight together
+          float si[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r)
+            si[r] = p.state_in != nullptr
+                        ? p.state_in[sbase + static_cast<int64_t>(r) * (D + 1) + j0 + lane]
+                        : 0.f;
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            const int64_t off = sbase + static_cast<int64_t>(r) * (D + 1) + j0 + lane;
+            const float sv = fmaf(a, si[r], tt[r * 33 + lane]);
+            if (p.state_out != nullptr) p.state_out[off] = sv;
+            tt[r * 33 + lane] = sv;
+          }
+          __syncwarp();
+#pragma unroll 8
+          for (int c = 0; c < 32; ++c) {
+            const int j = j0 + c;
+            *reinterpret_cast<__nv_bfloat16*>(img + j * G::kRowBytes + G::swz(j, cin) * 16) =
+                __float2bfloat16_rn(tt[lane * 33 + c]);
+          }
+          __syncwarp();
+        };
+        // the normaliser column j = d, one entry per thread
+        auto fold_norm = [&](float dS) {
+          const int64_t off = sbase + static_cast<int64_t>(lane) * (D + 1) + D;
+          const float si = p.state_in != nullptr ? p.state_in[off] : 0.f;
+          const float sv = fmaf(a, si, dS);
+          if (p.state_out != nullptr) p.state_out[off] = sv;
+          *reinterpret_cast<__nv_bfloat16*>(img + D * G::kRowBytes + G::swz(D, cin) * 16) =
+              __float2bfloat16_rn(sv);
+        };
+        if (u < cur.U_full) {
+          // the whole unit is this CTA's: fold from TMEM
+          if (has_row) {
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(tacc + cc * 32, r);
+              tmem_wait_ld();
+              float dv[32];
+#pragma unroll
+              for (int jj = 0; jj < 32; ++jj) dv[jj] = __uint_as_float(r[jj]);
+              fold_block(cc * 32, dv);
+            }
+            fold_norm(zs);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acce(ab));
+        } else {
+          // a unit split over CTAs: this CTA's partial (the scan adds them up)
+          if (has_row) {
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(tacc + cc * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+            }
+            dst[static_cast<int64_t>(D) * D] = zs;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acce(ab));
+        }
+        ++seg;
+        continue;
+      }
+      if (has_row) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
-          tmem_ld_32cols(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * AC + cc * 32, r);
+          tmem_ld_32cols(tacc + cc * 32, r);
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
@@ -340,8 +471,7 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t r[32];
-            tmem_ld_32cols(
-                tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * AC + D + cc * 32, r);
+            tmem_ld_32cols(tacc + D + cc * 32, r);
             tmem_wait_ld();
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) mdst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
@@ -350,7 +480,10 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce(ab));
+      if (lane == 0) {
+        mbar_arrive(acce(ab));
+        mbar_arrive(zfree);  // (the normaliser sums are warp 4's here)
+      }
       ++seg;
     }
   }

@@ -42,6 +42,8 @@ struct ScanParams {
   float* zvec;             // [units][d] fp32 S_f[:, d] per frame, or nullptr (rotary variant)
   uint8_t* image_lo;       // [units][kImageBytes] bf16(S_f - bf16(S_f))^T, value rows 0..d-1,
                            // or nullptr (backward: the query kernel's dq contraction)
+  int bh0;                 // first (b, h) of the grid (single-frame calls whose whole
+                           // units the increment kernel folds: the split ones only)
 };
 
 template <int D, int kStagesT = 3>
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(288, (kStagesT == 1) ? 4 : 3)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / C::kGroups;
+  const int bh = p.bh0 + static_cast<int>(blockIdx.x / C::kGroups);
   const int j0 = (blockIdx.x % C::kGroups) * C::kRows;
   const int nrows = (D + 1 - j0 < C::kRows) ? D + 1 - j0 : C::kRows;
   const int r = threadIdx.x / C::kOcts;  // consumer: row within the block

@@ -61,6 +61,14 @@ struct AnchorParams {
   int units;         // B * F * H * tiles per frame
   float scale_log2;  // log2(e) / sqrt(d)
   int has_gate;
+  // Rollout step (step != 0): q, k, v, z and out hold one frame (F == 1), the
+  // frame `frame` of the sequence; the earlier frames of its window come from
+  // a window cache (win_frames frames, oldest first) and the sink tokens
+  // from a sink cache (the first n_sink tokens of the sequence).  The key
+  // tiles are the same, in the same order, as for that frame in a call over
+  // the whole sequence.
+  int step;
+  int frame;
 };
 
 // The key tiles of the queries of frame f, in order: the sink tokens that
@@ -187,13 +195,20 @@ struct AnchorCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
+// Key / value sources of a rollout step (unused by a whole-sequence call):
+// the sink cache [B, n_sink, H, d] and the window cache [B, frames * T, H, d].
+struct AnchorCaches {
+  CUtensorMap ks, vs, kw, vw;
+};
+
 template <int D>
 __global__ void __launch_bounds__(352, 1)
     gla_softmax_anchor_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v,
                               const __grid_constant__ CUtensorMap tm_z,
-                              const __grid_constant__ CUtensorMap tm_out, const AnchorParams p) {
+                              const __grid_constant__ CUtensorMap tm_out,
+                              const __grid_constant__ AnchorCaches caches, const AnchorParams p) {
   using G = Geo<D>;
   using C = AnchorCfg<D>;
   constexpr int S = C::kStages;
@@ -296,8 +311,23 @@ __global__ void __launch_bounds__(352, 1)
             tma_load_5d(o_buf + a * G::kAtomTileBytes, &tm_z, zfull, a * G::kAtomElems, h,
                         qt * kTileTokens, f, b);
         }
-        // one ring tile: K or V rows [t0, t0 + 128) of frame fr
-        auto load = [&](const CUtensorMap* tm, int fr, int t0) {
+        // one ring tile: K or V rows [t0, t0 + 128) of frame fr (of the
+        // sequence; a rollout step reads the caches for earlier frames)
+        auto load = [&](bool is_v, const KeyTiles& t) {
+          const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+          int fr = t.fr, t0 = t.t0;
+          if (p.step) {
+            if (t.in_sink) {  // sink tokens fr * T + t0 .. of the sink cache
+              tm = is_v ? &caches.vs : &caches.ks;
+              t0 += fr * p.T;
+              fr = 0;
+            } else if (t.fr < t.f) {  // an earlier frame of the window
+              tm = is_v ? &caches.vw : &caches.kw;
+              fr = t.fr - t.w_lo_frame;
+            } else {
+              fr = 0;
+            }
+          }
           const int s = static_cast<int>(n % S);
           if (!mbar_wait(rempty(s), static_cast<uint32_t>(((n / S) & 1) ^ 1), abort, kCode))
             return false;
@@ -308,15 +338,16 @@ __global__ void __launch_bounds__(352, 1)
           ++n;
           return true;
         };
-        KeyTiles kt;
-        int pfr = -1, pt0 = 0;  // the previous tile, whose V follows this tile's K
-        for (kt.init(p.T, f, p.window, p.n_sink); ok && !kt.done; kt.advance()) {
-          ok = load(&tm_k, kt.fr, kt.t0);
-          if (ok && pfr >= 0) ok = load(&tm_v, pfr, pt0);
-          pfr = kt.fr;
-          pt0 = kt.t0;
+        KeyTiles kt, prev;
+        bool has_prev = false;  // the previous tile, whose V follows this tile's K
+        for (kt.init(p.T, p.step ? p.frame : f, p.window, p.n_sink); ok && !kt.done;
+             kt.advance()) {
+          ok = load(false, kt);
+          if (ok && has_prev) ok = load(true, prev);
+          prev = kt;
+          has_prev = true;
         }
-        if (ok && pfr >= 0) ok = load(&tm_v, pfr, pt0);
+        if (ok && has_prev) ok = load(true, prev);
       }
       for (int64_t i = (n > S ? n - S : 0); i < n; ++i)
         mbar_wait_drain(rfull(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1));
@@ -410,7 +441,7 @@ __global__ void __launch_bounds__(352, 1)
           return true;
         };
         KeyTiles kt;
-        kt.init(p.T, f, p.window, p.n_sink);
+        kt.init(p.T, p.step ? p.frame : f, p.window, p.n_sink);
         if (!kt.done) {
           ok = me == 0 ? issue_s() : skip_s();
           for (bool first = true; ok; first = false) {
@@ -445,7 +476,7 @@ __global__ void __launch_bounds__(352, 1)
       float mo = -INFINITY, lo = 0.f;  // the other half's, after the exchange
       bool ok = true;
       KeyTiles kt;
-      kt.init(p.T, f, p.window, p.n_sink);
+      kt.init(p.T, p.step ? p.frame : f, p.window, p.n_sink);
       for (bool first = true; !kt.done; first = false) {
         const int sb = static_cast<int>(ns & 1);
         KeyTiles nx = kt;

@@ -182,6 +182,37 @@ int gla_softmax_anchor_timed(const void* q, const void* k, const void* v, const 
                              cudaEvent_t* events);
 
 /*
+ * gla_softmax_anchor_step -- the softmax anchor layer for one new frame of a
+ * rollout, from cached keys and values.
+ *
+ * The SANA-WM pages (method components) give the softmax layers attention
+ * sinks and a local window of frames so that memory and per-chunk latency
+ * stay constant over a long rollout: a new frame needs only the sink tokens
+ * and the window's earlier frames, not the whole sequence.  This call computes
+ * the output of frame `frame` of the sequence exactly as gla_softmax_anchor
+ * over the whole sequence would (the same key tiles in the same order, so the
+ * result is the same bit for bit):
+ *   q, k, v, gate_z, out   bf16 [B, T, H, d], the new frame (gate_z may be NULL)
+ *   sink_k, sink_v         bf16 [B, n_sink, H, d]: the first n_sink tokens of the
+ *                          sequence.  Only the min(n_sink, w_lo * T) of them
+ *                          that precede the window are read, w_lo =
+ *                          max(0, frame - window_frames + 1); NULL allowed when
+ *                          that is 0.
+ *   win_k, win_v           bf16 [B, nw * T, H, d]: the window's earlier frames
+ *                          w_lo .. frame - 1, oldest first, nw = min(frame,
+ *                          window_frames - 1); NULL allowed when nw = 0.
+ *   frame >= 0, window_frames >= 1, n_sink >= 0, d = 128; T = tokens_per_frame.
+ * The caller keeps the caches (a copy of the first n_sink keys and values and
+ * of the last window_frames - 1 frames).  All pointers 16-byte aligned device
+ * pointers.  Returns the gla_softmax_anchor codes.
+ */
+int gla_softmax_anchor_step(const void* q, const void* k, const void* v, const void* gate_z,
+                            const void* sink_k, const void* sink_v, const void* win_k,
+                            const void* win_v, void* out, int B, int H, int tokens_per_frame,
+                            int d, int frame, int window_frames, int n_sink,
+                            cudaStream_t stream);
+
+/*
  * gla_forward_gdn -- the frame-wise gated delta-rule variant (Gated DeltaNet).
  *
  * The SANA-WM pages (paper analysis: abstract, method components) describe

@@ -216,3 +216,14 @@ def test_alloc_failure_hook_is_host_only(lib):
     # arming and disarming the hook makes no CUDA call (this runs without a GPU)
     assert lib.gla_inject_alloc_failure(3) == 0
     assert lib.gla_inject_alloc_failure(0) == 0
+
+
+def test_anchor_step_validation_before_any_cuda_call(lib):
+    # d != 128, negative frame, missing caches: rejected without touching CUDA
+    vp = FAKE
+    assert lib.gla_softmax_anchor_step(vp, vp, vp, None, vp, vp, vp, vp, vp, 1, 1, 64, 64, 1, 2,
+                                       64, None) == 4
+    assert lib.gla_softmax_anchor_step(vp, vp, vp, None, vp, vp, vp, vp, vp, 1, 1, 64, 128, -1,
+                                       2, 64, None) == 3
+    assert lib.gla_softmax_anchor_step(vp, vp, vp, None, vp, vp, None, None, vp, 1, 1, 64, 128, 3,
+                                       2, 64, None) == 1
