@@ -311,10 +311,10 @@ __global__ void __launch_bounds__(320, 1)
             !mbar_wait(acc3_free, static_cast<uint32_t>((seg & 1) ^ 1), abort, kCode))
           break;
         tc_fence_after();
-        // MMA3: L_f += phi(Q)^T . D  (K over the tile's tokens; N = d value
-        // columns from D_hi's main atoms, N = 16 from the pad region, then
-        // D_lo): the D_hi buffer, where the next dout lands, is released
-        // before the D_lo half runs
+        // MMA3: L_f += phi(Q)^T . D  (K over the tile's tokens): N = d value
+        // columns from D_hi's main atoms first, then the release of that
+        // buffer (the next dout lands there), then N = 16 from the pad region
+        // and D_lo (both written again only after lfree)
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
           const uint32_t acc = (cur.first && kk == 0) ? 0u : 1u;
@@ -323,14 +323,15 @@ __global__ void __launch_bounds__(320, 1)
           const uint64_t bd = smem_desc(d_buf + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
                                         G::kGroupBytes, G::kLayout);
           mma_bf16(tmem + C::kAcc3, ad, bd, idesc3, acc);
-          const uint64_t bz = smem_desc(d_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
-          mma_bf16(tmem + C::kAcc3 + D, ad, bz, idesc3z, acc);
         }
         mma_commit(dfree);
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+          const uint32_t acc = (cur.first && kk == 0) ? 0u : 1u;
           const uint64_t ad = smem_desc(q_buf(s) + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
                                         G::kGroupBytes, G::kLayout);
+          const uint64_t bz = smem_desc(d_pad + kk * 512, C::kDPadBytes, 256, kLayoutSW32);
+          mma_bf16(tmem + C::kAcc3 + D, ad, bz, idesc3z, acc);
           const uint64_t bl = smem_desc(l_buf + kk * 2 * G::kGroupBytes, G::kAtomTileBytes,
                                         G::kGroupBytes, G::kLayout);
           mma_bf16(tmem + C::kAcc3, ad, bl, idesc3, 1u);
