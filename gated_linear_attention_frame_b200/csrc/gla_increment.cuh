@@ -91,6 +91,14 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return ok != 0;
 }
 
+// A wait on a phase that has most likely completed already: one vote of the
+// warp on a non-blocking test, the bounded warp_wait otherwise.
+__device__ __forceinline__ bool warp_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               unsigned int code) {
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+  return warp_wait(bar, parity, abort, code);
+}
+
 // kRope: the rotary variant (gla_rope.cuh): phi(K) is rotated in shared
 // memory after its normaliser sums are taken, so the contraction forms
 // (R phi(K))^T V while row d keeps sum phi(k).

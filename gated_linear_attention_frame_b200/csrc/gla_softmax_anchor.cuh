@@ -156,26 +156,6 @@ __device__ __forceinline__ void exp2_poly3_x2(float a0, float a1, float& x0, flo
   x1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate (A: lane
-// = row, two consecutive K elements per 32-bit column).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// A wait on a phase that has most likely completed already: one vote of the
-// warp on a single try_wait, the bounded warp_wait otherwise.
-__device__ __forceinline__ bool warp_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
-                                               unsigned int code) {
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return warp_wait(bar, parity, abort, code);
-}
-
 template <int D>
 struct AnchorCfg {
   using G = Geo<D>;
