@@ -44,6 +44,11 @@
 
 namespace {
 
+// Partial slices in flight per scan block over a sequence of frames (three
+// blocks of 74 KB share an SM at 4).
+constexpr int kScanStages = 4;
+
+
 using gla::Geo;
 
 constexpr int kMaxDevices = 64;
@@ -137,8 +142,8 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gla::ScanCfg<D, 1>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           gla::ScanCfg<D, 3>::kSmemBytes);
+  e = cudaFuncSetAttribute(gla::gla_scan_kernel<D, kScanStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gla::ScanCfg<D, kScanStages>::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla::gla_increment_kernel<D, false, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -412,12 +417,12 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
     gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu, zvec};
     sp.bh0 = bh0;
     using SC1 = gla::ScanCfg<D, 1>;
-    using SC3 = gla::ScanCfg<D, 3>;
+    using SC3 = gla::ScanCfg<D, kScanStages>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(nbh);
     const cudaError_t e =
         a.F <= 1 ? launch_dependent(gla::gla_scan_kernel<D, 1>, grid, SC1::kThreads,
                                     SC1::kSmemBytes, a.stream, sp)
-                 : launch_dependent(gla::gla_scan_kernel<D, 3>, grid, SC3::kThreads,
+                 : launch_dependent(gla::gla_scan_kernel<D, kScanStages>, grid, SC3::kThreads,
                                     SC3::kSmemBytes, a.stream, sp);
     if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
@@ -719,12 +724,12 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
     gla::ScanParams sp{partial, a.g, a.s_in, nullptr, image, states, wp, a.H, a.F, tpu,
                        nullptr, image_lo};
     using SC1 = gla::ScanCfg<D, 1>;
-    using SC3 = gla::ScanCfg<D, 3>;
+    using SC3 = gla::ScanCfg<D, kScanStages>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(a.B * a.H);
     const cudaError_t e =
         a.F <= 1 ? launch_dependent(gla::gla_scan_kernel<D, 1>, grid, SC1::kThreads,
                                     SC1::kSmemBytes, a.stream, sp)
-                 : launch_dependent(gla::gla_scan_kernel<D, 3>, grid, SC3::kThreads,
+                 : launch_dependent(gla::gla_scan_kernel<D, kScanStages>, grid, SC3::kThreads,
                                     SC3::kSmemBytes, a.stream, sp);
     if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
