@@ -621,8 +621,8 @@ def run_other_workloads(args, head: dict, dist, rank, local_rank, world) -> dict
 
 # The library's other paths at the headline workload, timed by the default run
 # as well (fewer steps: each is one call of its entry point per step).
-OTHER_PATHS = (("backward", "plain"), ("forward", "rope"), ("forward", "gdn"),
-               ("forward", "softmax"))
+OTHER_PATHS = (("backward", "plain"), ("backward", "saved"), ("forward", "rope"),
+               ("forward", "gdn"), ("forward", "softmax"))
 PATH_STEPS = 10
 
 
@@ -636,6 +636,8 @@ def path_summary(r: dict) -> dict:
         out["kernel_ms"] = r["layer_roofline"]["kernel_ms"]
     if "rollout_step" in r:
         out["rollout_step"] = r["rollout_step"]
+    if "saved_context" in r:
+        out["saved_context"] = r["saved_context"]
     return out
 
 
@@ -644,7 +646,8 @@ def run_other_paths(args, w, dist, rank, local_rank, world) -> dict:
     for mode, variant in OTHER_PATHS:
         a = argparse.Namespace(**vars(args))
         a.no_e2e = True
-        a.mode, a.variant = mode, variant
+        a.mode, a.variant = mode, "plain" if variant == "saved" else variant
+        a.saved = variant == "saved"
         a.steps = min(args.steps, PATH_STEPS)
         torch.cuda.empty_cache()
         if mode == "backward":
@@ -653,15 +656,20 @@ def run_other_paths(args, w, dist, rank, local_rank, world) -> dict:
             r = run_gpu_anchor(a, w, dist, rank, local_rank, world)
         else:
             r = run_gpu(a, w, dist, rank, local_rank, world)
-        out[mode if mode == "backward" else variant] = path_summary(r)
+        key = ("backward_saved" if variant == "saved" else "backward") if mode == "backward" \
+            else variant
+        out[key] = path_summary(r)
     return out
 
 
 def run_gpu_backward(args, w, dist, rank, local_rank, world):
     """One step = one gla_backward call over one batch of the workload
-    (recompute of the forward states, then the five gradient kernels)."""
+    (recompute of the forward states, then the five gradient kernels), or with
+    --saved one gla_backward_saved call from the context a gla_forward_train
+    call of the same inputs wrote before the timed region (four kernels)."""
     import gated_linear_attention_frame_b200 as gla
 
+    saved_mode = bool(getattr(args, "saved", False))
     if w.d != 128:
         raise SystemExit("the backward pass is built for d = 128")
     dev = torch.device("cuda", local_rank)
@@ -675,11 +683,45 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
     dg = torch.empty_like(g)
     ds_in = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev) if s_in is not None else None
     work = algorithmic_work_backward(w, s_in is not None, ds_out is not None, ds_in is not None)
+    saved = None
+    fwd_train = None
+    if saved_mode:
+        saved = torch.empty(max(1, gla.gla_saved_bytes(w.B, w.H, w.frames, w.tokens_per_frame,
+                                                       w.d)), device=dev, dtype=torch.uint8)
+        f_out = torch.empty_like(q)
+        f_state = torch.empty(w.B, w.H, w.d, w.d + 1, device=dev)
+        fa = (q, k, v, g, s_in, f_state, f_out)
+        dims = (w.B, w.H, w.frames, w.tokens_per_frame, w.d, w.eps, stream)
+        # the training forward's cost over the plain forward (context writes)
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for _ in range(3):
+            gla.gla_forward(*fa, *dims)
+            gla.gla_forward_train(*fa, saved, *dims)
+        fe[0].record(stream)
+        for _ in range(5):
+            gla.gla_forward(*fa, *dims)
+        fe[1].record(stream)
+        fe[2].record(stream)
+        for _ in range(5):
+            gla.gla_forward_train(*fa, saved, *dims)
+        fe[3].record(stream)
+        torch.cuda.synchronize(dev)
+        fwd_train = {"forward_ms": round(fe[0].elapsed_time(fe[1]) / 5, 5),
+                     "forward_train_ms": round(fe[2].elapsed_time(fe[3]) / 5, 5),
+                     "saved_bytes": int(saved.numel()),
+                     "note": "the context is written by gla_forward_train before the timed "
+                             "region; the timed calls are gla_backward_saved"}
 
     def step(events=None):
         a = (q, k, v, g, s_in, dout, ds_out, dq, dk, dv, dg, ds_in, w.B, w.H, w.frames,
              w.tokens_per_frame, w.d, w.eps, stream)
-        if events is None:
+        if saved_mode:
+            b = a[:5] + (saved,) + a[5:]
+            if events is None:
+                gla.gla_backward_saved(*b)
+            else:
+                gla.gla_backward_saved_timed(*b, events)
+        elif events is None:
             gla.gla_backward(*a)
         else:
             gla.gla_backward_timed(*a, events)
@@ -720,6 +762,9 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
     fault = gla.gla_device_fault(stream)
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs])
     avg = per.mean(axis=0)
+    if saved_mode:
+        names = names[2:]
+        avg = avg[2:]
     dom = int(np.argmax(avg))
     achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
     roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
@@ -744,15 +789,19 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
 
         def call(bi, bo):
             q_, k_, v_, g_, do_, s_, dso_ = bi
-            gla.gla_backward(q_, k_, v_, g_, s_, do_, dso_, bo[0], bo[1], bo[2], bo[3],
-                             bo[4] if len(bo) > 4 else None, w.B, w.H, w.frames,
-                             w.tokens_per_frame, w.d, w.eps, stream)
+            tail = (bo[0], bo[1], bo[2], bo[3], bo[4] if len(bo) > 4 else None, w.B, w.H,
+                    w.frames, w.tokens_per_frame, w.d, w.eps, stream)
+            if saved_mode:  # the context stays on the device, as in training
+                gla.gla_backward_saved(q_, k_, v_, g_, s_, saved, do_, dso_, *tail)
+            else:
+                gla.gla_backward(q_, k_, v_, g_, s_, do_, dso_, *tail)
 
         e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
                             max(2, min(K, args.e2e_steps)), w.total_tokens)
 
-    return {
-        "metric": METRIC_BWD, "mode": "backward", "value": round(value, 1), "unit": UNIT,
+    res = {
+        "metric": METRIC_BWD, "mode": "backward_saved" if saved_mode else "backward",
+        "value": round(value, 1), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": warm, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -762,10 +811,13 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
                    "l2": "inputs larger than L2 (%.2f GB read+written per step); no flush"
                          % (work["bytes"] / 1e9),
                    "parallelism": "dp%d (independent sequences per GPU)" % world},
-        "roofline": roof, "layer_roofline": layer, "gpu_launches": 6 * K, "e2e": e2e,
-        "clocks": clocks.summary(), "device_fault": fault,
+        "roofline": roof, "layer_roofline": layer, "gpu_launches": (4 if saved_mode else 6) * K,
+        "e2e": e2e, "clocks": clocks.summary(), "device_fault": fault,
         "gpu": torch.cuda.get_device_name(dev),
     }
+    if fwd_train is not None:
+        res["saved_context"] = fwd_train
+    return res
 
 
 def run_gpu_anchor(args, w, dist, rank, local_rank, world):
@@ -976,6 +1028,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
                     help="time gla_forward (the layer metric) or gla_backward")
+    ap.add_argument("--saved", action="store_true",
+                    help="--mode backward: time gla_backward_saved from a gla_forward_train "
+                         "context instead of gla_backward (no recompute)")
     ap.add_argument("--variant", choices=["plain", "rope", "gdn", "softmax"], default="plain",
                     help="forward only: the plain layer, gla_forward_rope (3D RoPE), "
                          "gla_forward_gdn (frame-wise gated delta rule) or gla_softmax_anchor")

@@ -29,7 +29,8 @@ GLA_ERR_ROPE = 9
 EXPORTED = ("gla_forward", "gla_forward_timed", "gla_forward_noalloc", "gla_noalloc_scratch_bytes",
             "gla_forward_rope", "gla_forward_rope_timed", "gla_forward_gdn", "gla_forward_gdn_timed",
             "gla_softmax_anchor", "gla_softmax_anchor_timed", "gla_softmax_anchor_step",
-            "gla_backward", "gla_backward_timed",
+            "gla_backward", "gla_backward_timed", "gla_saved_bytes", "gla_forward_train",
+            "gla_backward_saved", "gla_backward_saved_timed",
             "gla_trim_workspace", "gla_set_workspace_retention", "gla_inject_alloc_failure",
             "gla_set_wait_limit_ns", "gla_inject_stall", "gla_error_string", "gla_device_fault",
             "gla_version")
@@ -99,6 +100,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gla_backward.restype = i32
     lib.gla_backward_timed.argtypes = bwd + [ctypes.POINTER(vp)]
     lib.gla_backward_timed.restype = i32
+    lib.gla_saved_bytes.argtypes = [i32] * 5
+    lib.gla_saved_bytes.restype = ctypes.c_size_t
+    lib.gla_forward_train.argtypes = [vp] * 8 + [i32] * 5 + [f32, vp]
+    lib.gla_forward_train.restype = i32
+    bwds = [vp] * 13 + [i32, i32, i32, i32, i32, f32, vp]  # gla_backward's + saved
+    lib.gla_backward_saved.argtypes = bwds
+    lib.gla_backward_saved.restype = i32
+    lib.gla_backward_saved_timed.argtypes = bwds + [ctypes.POINTER(vp)]
+    lib.gla_backward_saved_timed.restype = i32
     lib.gla_noalloc_scratch_bytes.argtypes = []
     lib.gla_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.gla_trim_workspace.argtypes = []
@@ -386,6 +396,56 @@ def gla_backward_timed(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk,
         raise GLAError(st, "gla_backward_timed")
 
 
+def gla_saved_bytes(B, H, frames, tokens_per_frame, d) -> int:
+    """Bytes of the context gla_forward_train saves (0 if d != 128)."""
+    return int(load_library().gla_saved_bytes(int(B), int(H), int(frames), int(tokens_per_frame),
+                                              int(d)))
+
+
+def gla_forward_train(q, k, v, gate_logits, state_in, state_out, out, saved, B, H, frames,
+                      tokens_per_frame, d, eps, stream=None) -> None:
+    """gla_forward that also writes the backward's context into `saved`
+    (gla_saved_bytes bytes, 256-byte aligned; see include/gla.h)."""
+    st = load_library().gla_forward_train(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits), _ptr(state_in), _ptr(state_out), _ptr(out),
+        _ptr(saved), int(B), int(H), int(frames), int(tokens_per_frame), int(d), float(eps),
+        _stream(stream))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_forward_train")
+
+
+def _saved_args(args, saved):
+    return args[:5] + (_ptr(saved),) + args[5:]
+
+
+def gla_backward_saved(q, k, v, gate_logits, state_in, saved, dout, dstate_out, dq, dk, dv,
+                       dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps,
+                       stream=None) -> None:
+    """gla_backward from a context of gla_forward_train (no recompute)."""
+    args = _bwd_args(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+                     dstate_in, B, H, frames, tokens_per_frame, d, eps, stream)
+    st = load_library().gla_backward_saved(*_saved_args(args, saved))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_backward_saved")
+
+
+def gla_backward_saved_timed(q, k, v, gate_logits, state_in, saved, dout, dstate_out, dq, dk, dv,
+                             dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps,
+                             stream, events) -> None:
+    """gla_backward_saved that records 7 CUDA events (as gla_backward_timed)."""
+    args = _bwd_args(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dgate_logits,
+                     dstate_in, B, H, frames, tokens_per_frame, d, eps, stream)
+    lib = load_library()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 7)(*[e.cuda_event for e in events])
+    st = lib.gla_backward_saved_timed(*_saved_args(args, saved),
+                                      ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    if st != GLA_OK:
+        raise GLAError(st, "gla_backward_saved_timed")
+
+
 def gla_noalloc_scratch_bytes() -> int:
     return int(load_library().gla_noalloc_scratch_bytes())
 
@@ -500,10 +560,33 @@ def forward_rope(q, k, v, gate_logits, rope: RopeConfig, state_in=None, eps: flo
     return out, state_out
 
 
+def forward_train(q, k, v, gate_logits, state_in=None, eps: float = 1e-6, out=None,
+                  state_out=None, saved=None, stream=None):
+    """forward() that also returns the context for backward(..., saved=):
+    (out, state_out, saved), `saved` a uint8 device tensor (allocated if not
+    given)."""
+    B, N, H, d = q.shape
+    frames = gate_logits.shape[1]
+    T = 0 if frames == 0 else N // frames
+    if frames and N % frames:
+        raise ValueError("token axis %d is not a multiple of frames %d" % (N, frames))
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None:
+        state_out = torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
+    if saved is None:
+        n = gla_saved_bytes(B, H, frames, T, d)
+        saved = torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
+    gla_forward_train(q, k, v, gate_logits, state_in, state_out, out, saved, B, H, frames, T, d,
+                      eps, stream)
+    return out, state_out, saved
+
+
 def backward(q, k, v, gate_logits, dout, state_in=None, dstate_out=None, eps: float = 1e-6,
-             stream=None, want_dstate_in: bool = True):
-    """Convenience wrapper of gla_backward: allocates the gradients and
-    returns (dq, dk, dv, dgate_logits, dstate_in or None)."""
+             stream=None, want_dstate_in: bool = True, saved=None):
+    """Convenience wrapper of gla_backward (gla_backward_saved when `saved`,
+    the context of forward_train for the same inputs, is given): allocates the
+    gradients and returns (dq, dk, dv, dgate_logits, dstate_in or None)."""
     B, N, H, d = q.shape
     frames = gate_logits.shape[1]
     if frames == 0:
@@ -516,6 +599,10 @@ def backward(q, k, v, gate_logits, dout, state_in=None, dstate_out=None, eps: fl
     dg = torch.empty_like(gate_logits)
     ds_in = (torch.empty(B, H, d, d + 1, device=q.device, dtype=torch.float32)
              if want_dstate_in else None)
-    gla_backward(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dg, ds_in, B, H,
-                 frames, T, d, eps, stream)
+    if saved is None:
+        gla_backward(q, k, v, gate_logits, state_in, dout, dstate_out, dq, dk, dv, dg, ds_in, B,
+                     H, frames, T, d, eps, stream)
+    else:
+        gla_backward_saved(q, k, v, gate_logits, state_in, saved, dout, dstate_out, dq, dk, dv,
+                           dg, ds_in, B, H, frames, T, d, eps, stream)
     return dq, dk, dv, dg, ds_in

@@ -250,7 +250,9 @@ struct Args {
   cudaStream_t stream;
   const gla_rope_config* rope = nullptr;  // rotary variant when set
   const float* beta = nullptr;            // delta-rule variant: [B, F, H] write-strength logits
+  uint8_t* saved = nullptr;               // training forward: the context for the backward
 };
+
 
 // Host-only checks of a rotary configuration; no CUDA call.
 int validate_rope(const gla_rope_config* r, int d) {
@@ -309,6 +311,24 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned b
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// The context a training forward saves for gla_backward_saved (d = 128):
+// per unit the bf16 image of S_f^T (as the output kernel reads it), its bf16
+// remainder (value rows 0..d-1) and S_f in fp32 ([d+1][d], as the scan writes
+// them for the backward's query kernel), each region 256-byte aligned.
+struct SavedLayout {
+  int64_t image, image_lo, states, total;  // byte offsets, size
+};
+SavedLayout saved_layout(int64_t units) {
+  constexpr int D = 128;
+  SavedLayout l;
+  const int64_t img = align256(units * static_cast<int64_t>(Geo<D>::kImageBytes));
+  l.image = 0;
+  l.image_lo = img;
+  l.states = 2 * img;
+  l.total = 2 * img + align256(units * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4);
+  return l;
+}
+
 template <int D, bool kRope = false>
 int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
         const FixedScratch* fixed = nullptr) {
@@ -348,8 +368,11 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   const int64_t zvec_bytes = (kRope && W > 0) ? align256(units * static_cast<int64_t>(D) * 4) : 0;
   // single frame, plain layer: the increment kernel folds the scan step for
   // the units it owns whole; the scan runs over the split units alone
-  const bool fold = !kRope && a.F == 1 && W > 0;
-  const int64_t ws_bytes = partial_bytes + image_bytes + table_bytes + zvec_bytes;
+  // (a training forward writes every unit's state through the scan)
+  const bool fold = !kRope && a.F == 1 && W > 0 && a.saved == nullptr;
+  const SavedLayout sl = saved_layout(units);
+  const int64_t ws_image_bytes = a.saved != nullptr ? 0 : image_bytes;
+  const int64_t ws_bytes = partial_bytes + ws_image_bytes + table_bytes + zvec_bytes;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_out;
   if (W > 0) {
@@ -369,11 +392,11 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
     if (st != GLA_OK) return st;
   }
   float* partial = reinterpret_cast<float*>(ws);
-  uint8_t* image = ws ? ws + partial_bytes : nullptr;
-  float2* table = table_pairs > 0 ? reinterpret_cast<float2*>(ws + partial_bytes + image_bytes)
+  uint8_t* image = a.saved != nullptr ? a.saved + sl.image : (ws ? ws + partial_bytes : nullptr);
+  float2* table = table_pairs > 0 ? reinterpret_cast<float2*>(ws + partial_bytes + ws_image_bytes)
                                   : nullptr;
   float* zvec = zvec_bytes > 0
-                    ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + table_bytes)
+                    ? reinterpret_cast<float*>(ws + partial_bytes + ws_image_bytes + table_bytes)
                     : nullptr;
 
   rg.table = reinterpret_cast<const float4*>(table);
@@ -416,6 +439,10 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
   if (status == GLA_OK && nbh > 0 && (a.F > 0 || a.s_out != nullptr)) {
     gla::ScanParams sp{partial, a.g, a.s_in, a.s_out, image, nullptr, wp, a.H, a.F, tpu, zvec};
     sp.bh0 = bh0;
+    if (a.saved != nullptr) {  // the backward's inputs as well
+      sp.states = reinterpret_cast<float*>(a.saved + sl.states);
+      sp.image_lo = a.saved + sl.image_lo;
+    }
     using SC1 = gla::ScanCfg<D, 1>;
     using SC3 = gla::ScanCfg<D, kScanStages>;
     const unsigned grid = static_cast<unsigned>(SC3::kGroups) * static_cast<unsigned>(nbh);
@@ -631,6 +658,7 @@ struct BwdArgs {
   int B, H, F, T, d;
   float eps;
   cudaStream_t stream;
+  const uint8_t* saved = nullptr;  // a training forward's context: no recompute
 };
 
 // Host-only checks of gla_backward's arguments; no CUDA call.
@@ -674,7 +702,11 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   const int64_t states_bytes = align256(units * static_cast<int64_t>(PF) * 4);
   const int64_t da_bytes = align256(units * static_cast<int64_t>(RS::kGroups) * 8 * 4);
   const int64_t gnorm_bytes = W > 0 ? align256(units * static_cast<int64_t>(D) * 4) : 0;
-  const int64_t ws_bytes = partial_bytes + 2 * image_bytes + states_bytes + da_bytes + gnorm_bytes;
+  const bool saved = a.saved != nullptr;
+  // with a saved context the S_f images and states are read from it and the
+  // G_f^T images go to the workspace (the caller's context is not written)
+  const int64_t ws_bytes =
+      partial_bytes + 2 * image_bytes + (saved ? 0 : states_bytes) + da_bytes + gnorm_bytes;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_dout, tm_dq, tm_dk, tm_dv;
   if (W > 0) {
@@ -695,13 +727,25 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
     const int st = take_workspace(ws_bytes, a.stream, &ws);
     if (st != GLA_OK) return st;
   }
+  const int64_t ws_states = saved ? 0 : states_bytes;
   float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
-  uint8_t* image = W > 0 ? ws + partial_bytes : nullptr;
+  uint8_t* image = W > 0 ? ws + partial_bytes : nullptr;  // S_f^T (recompute), then G_f^T
   float* states = ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes) : nullptr;
   float* da_part =
-      ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + states_bytes) : nullptr;
-  uint8_t* image_lo = W > 0 ? ws + partial_bytes + image_bytes + states_bytes + da_bytes : nullptr;
+      ws ? reinterpret_cast<float*>(ws + partial_bytes + image_bytes + ws_states) : nullptr;
+  uint8_t* image_lo = W > 0 ? ws + partial_bytes + image_bytes + ws_states + da_bytes : nullptr;
   float* gnorm = W > 0 ? reinterpret_cast<float*>(image_lo + image_bytes) : nullptr;
+  // the query kernel's S_f inputs: the recompute's, or the saved context's
+  const uint8_t* s_image = image;
+  const uint8_t* s_image_lo = image_lo;
+  const float* s_states = states;
+  if (saved) {
+    const SavedLayout sl = saved_layout(units);
+    s_image = a.saved + sl.image;
+    s_image_lo = a.saved + sl.image_lo;
+    s_states = reinterpret_cast<const float*>(a.saved + sl.states);
+    states = nullptr;
+  }
 
   int status = GLA_OK;
   auto check = [&]() {
@@ -713,14 +757,14 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   };
 
   record(0);
-  if (W > 0 && status == GLA_OK) {
+  if (!saved && W > 0 && status == GLA_OK) {
     gla::IncParams ip{partial, wp, a.H, a.F};
     gla::gla_increment_kernel<D>
         <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
     check();
   }
   record(1);
-  if (status == GLA_OK && a.F > 0) {
+  if (!saved && status == GLA_OK && a.F > 0) {
     gla::ScanParams sp{partial, a.g, a.s_in, nullptr, image, states, wp, a.H, a.F, tpu,
                        nullptr, image_lo};
     using SC1 = gla::ScanCfg<D, 1>;
@@ -736,7 +780,7 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(2);
   if (W > 0 && status == GLA_OK) {
-    gla::BwdQParams qp{image, image_lo, states, partial, a.eps, wp, a.H, a.F, a.T};
+    gla::BwdQParams qp{s_image, s_image_lo, s_states, partial, a.eps, wp, a.H, a.F, a.T};
     if (launch_dependent(gla::gla_bwd_q_kernel<D>, G1, gla::BwdQCfg<D>::kThreads,
                          gla::BwdQCfg<D>::kSmemBytes, a.stream, tm_q, tm_dout, tm_dq,
                          qp) != cudaSuccess)
@@ -745,8 +789,8 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   }
   record(3);
   if (status == GLA_OK && (a.F > 0 || a.ds_in != nullptr)) {
-    gla::ScanBwdParams rp{partial, a.g,   states,  a.s_in, a.ds_out, a.ds_in, image,
-                          image_lo, gnorm, da_part, wp,    a.H,      a.F,     tpu};
+    gla::ScanBwdParams rp{partial, a.g,   s_states, a.s_in, a.ds_out, a.ds_in, image,
+                          image_lo, gnorm, da_part, wp,     a.H,    a.F,      tpu};
     const unsigned grid = static_cast<unsigned>(RS::kGroups) * static_cast<unsigned>(a.B * a.H);
     if (launch_dependent(gla::gla_scan_bwd_kernel<D>, grid, RS::kThreads, RS::kSmemBytes,
                          a.stream, rp) != cudaSuccess)
@@ -996,6 +1040,60 @@ int gla_backward_timed(const void* q, const void* k, const void* v, const float*
   BwdArgs a{q,  k,  v,  gate_logits, state_in, dout, dstate_out, dq, dk,     dv,
             dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream};
   return backward_impl(a, events);
+}
+
+size_t gla_saved_bytes(int B, int H, int frames, int tokens_per_frame, int d) {
+  if (d != 128 || B < 0 || H < 0 || frames < 0 || tokens_per_frame < 0) return 0;
+  return static_cast<size_t>(saved_layout(static_cast<int64_t>(B) * frames * H).total);
+}
+
+int gla_forward_train(const void* q, const void* k, const void* v, const float* gate_logits,
+                      const float* state_in, float* state_out, void* out, void* saved, int B,
+                      int H, int frames, int tokens_per_frame, int d, float eps,
+                      cudaStream_t stream) {
+  Args a{q, k, v, gate_logits, state_in, state_out, out, B, H, frames, tokens_per_frame, d, eps,
+         stream};
+  int st = validate(a);
+  if (st != GLA_OK) return st;
+  if (d != 128) return GLA_ERR_UNSUPPORTED_D;
+  if (static_cast<int64_t>(B) * frames * H > 0 && saved == nullptr) return GLA_ERR_NULL;
+  if (!aligned(saved, 256)) return GLA_ERR_ALIGN;
+  a.saved = static_cast<uint8_t*>(saved);
+  return forward_impl(a, nullptr);
+}
+
+namespace {
+int backward_saved(const BwdArgs& a, cudaEvent_t* ev) {
+  int st = validate_bwd(a);
+  if (st != GLA_OK) return st;
+  if (static_cast<int64_t>(a.B) * a.F * a.H > 0 && a.saved == nullptr) return GLA_ERR_NULL;
+  if (!aligned(a.saved, 256)) return GLA_ERR_ALIGN;
+  return backward_impl(a, ev);
+}
+}  // namespace
+
+int gla_backward_saved(const void* q, const void* k, const void* v, const float* gate_logits,
+                       const float* state_in, const void* saved, const void* dout,
+                       const float* dstate_out, void* dq, void* dk, void* dv, float* dgate_logits,
+                       float* dstate_in, int B, int H, int frames, int tokens_per_frame, int d,
+                       float eps, cudaStream_t stream) {
+  BwdArgs a{q,  k,  v,  gate_logits, state_in, dout, dstate_out, dq, dk,     dv,
+            dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream,
+            static_cast<const uint8_t*>(saved)};
+  return backward_saved(a, nullptr);
+}
+
+int gla_backward_saved_timed(const void* q, const void* k, const void* v,
+                             const float* gate_logits, const float* state_in, const void* saved,
+                             const void* dout, const float* dstate_out, void* dq, void* dk,
+                             void* dv, float* dgate_logits, float* dstate_in, int B, int H,
+                             int frames, int tokens_per_frame, int d, float eps,
+                             cudaStream_t stream, cudaEvent_t* events) {
+  if (events == nullptr) return GLA_ERR_NULL;
+  BwdArgs a{q,  k,  v,  gate_logits, state_in, dout, dstate_out, dq, dk,     dv,
+            dgate_logits, dstate_in, B, H, frames, tokens_per_frame, d, eps, stream,
+            static_cast<const uint8_t*>(saved)};
+  return backward_saved(a, events);
 }
 
 int gla_trim_workspace(void) {

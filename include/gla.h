@@ -308,7 +308,8 @@ int gla_forward_rope_timed(const void* q, const void* k, const void* v,
  *            G_{frames-1} adds dstate_out       (G_f = dL/dS_f, d x (d+1))
  *   dk_t   = 1[k_t > 0] * ([v_t | 1] G_f^T),   dv_t = phi(k_t) G_f[:, :d]
  *   dgate_logits[b, f, h] = a_f (1 - a_f) <G_f, S_{f-1}>,  dstate_in = a_0 G_0
- * The forward states are recomputed (nothing is saved between the calls).
+ * The forward states are recomputed (nothing is saved between the calls;
+ * gla_forward_train and gla_backward_saved keep them instead).
  *
  * Arguments (device pointers):
  *   q, k, v, gate_logits, state_in, B, H, frames, tokens_per_frame, eps
@@ -348,6 +349,65 @@ int gla_backward_timed(const void* q, const void* k, const void* v,
                        float* dgate_logits, float* dstate_in,
                        int B, int H, int frames, int tokens_per_frame, int d,
                        float eps, cudaStream_t stream, cudaEvent_t* events);
+
+/*
+ * gla_saved_bytes -- size in bytes of the context gla_forward_train saves for
+ * gla_backward_saved: per (b, f, h) the frame's state S_f as the bf16 image
+ * the output kernel reads, its bf16 remainder and S_f in fp32, i.e. about
+ * B*H*frames*4*(d+1)*d bytes (133 MB for B=2, H=24, 21 frames, d=128).
+ * 0 when d != 128 or a size is negative.  Host-only; no CUDA call.
+ */
+size_t gla_saved_bytes(int B, int H, int frames, int tokens_per_frame, int d);
+
+/*
+ * gla_forward_train -- gla_forward (head dim d = 128, plain layer) that also
+ * writes the per-frame states into `saved`, so that the backward pass of the
+ * same call does not recompute them (gla_backward_saved).  out and state_out
+ * are the same as gla_forward's, bit for bit.
+ *   saved   device buffer of gla_saved_bytes(B, H, frames, tokens_per_frame,
+ *           d) bytes, 256-byte aligned, owned by the caller; its contents are
+ *           opaque and valid for the backward of this call's inputs (q, k, v,
+ *           gate_logits, state_in) only.  Must not be NULL when
+ *           B * H * frames > 0 (GLA_ERR_NULL), nor overlap any argument.
+ * Other arguments, memory and return codes as gla_forward; d != 128 gives
+ * GLA_ERR_UNSUPPORTED_D.  Single-frame calls write every unit's state
+ * through the scan kernel (the increment kernel's fold is not used).
+ */
+int gla_forward_train(const void* q, const void* k, const void* v,
+                      const float* gate_logits, const float* state_in, float* state_out,
+                      void* out, void* saved, int B, int H, int frames, int tokens_per_frame,
+                      int d, float eps, cudaStream_t stream);
+
+/*
+ * gla_backward_saved -- gla_backward from the context `saved` that
+ * gla_forward_train wrote for the same inputs: the state increments and the
+ * forward scan are not run again (four kernels instead of six), and the
+ * gradients are the same as gla_backward's, bit for bit.  `saved` is read
+ * only.  The arguments are gla_backward's plus `saved` (NULL: GLA_ERR_NULL
+ * when B * H * frames > 0; 256-byte aligned: GLA_ERR_ALIGN otherwise).  A
+ * context from other inputs gives wrong gradients and is not detected.
+ * Memory: a workspace of about (B*H*frames*8 + #SMs*4) * (d+1)*d bytes.
+ */
+int gla_backward_saved(const void* q, const void* k, const void* v,
+                       const float* gate_logits, const float* state_in, const void* saved,
+                       const void* dout, const float* dstate_out,
+                       void* dq, void* dk, void* dv,
+                       float* dgate_logits, float* dstate_in,
+                       int B, int H, int frames, int tokens_per_frame, int d,
+                       float eps, cudaStream_t stream);
+
+/*
+ * gla_backward_saved_timed -- gla_backward_saved that records seven
+ * caller-created CUDA events on `stream` in gla_backward_timed's places (the
+ * first three are back to back: no increment or forward-scan kernel runs).
+ */
+int gla_backward_saved_timed(const void* q, const void* k, const void* v,
+                             const float* gate_logits, const float* state_in,
+                             const void* saved, const void* dout, const float* dstate_out,
+                             void* dq, void* dk, void* dv,
+                             float* dgate_logits, float* dstate_in,
+                             int B, int H, int frames, int tokens_per_frame, int d,
+                             float eps, cudaStream_t stream, cudaEvent_t* events);
 
 /*
  * gla_trim_workspace -- release the current device's unused workspace memory

@@ -227,3 +227,27 @@ def test_anchor_step_validation_before_any_cuda_call(lib):
                                        2, 64, None) == 3
     assert lib.gla_softmax_anchor_step(vp, vp, vp, None, vp, vp, None, None, vp, 1, 1, 64, 128, 3,
                                        2, 64, None) == 1
+
+
+def test_saved_context_calls_validate_before_any_cuda_call(lib):
+    # gla_forward_train / gla_backward_saved: d != 128, a missing or
+    # misaligned context are rejected without touching CUDA
+    vp = FAKE
+    odd = FAKE + 16  # 16-byte but not 256-byte aligned
+    assert lib.gla_saved_bytes(2, 24, 21, 3680, 128) == 133152768
+    assert lib.gla_saved_bytes(2, 24, 21, 3680, 64) == 0
+    assert lib.gla_saved_bytes(-1, 24, 21, 3680, 128) == 0
+    # forward_train: q, k, v, g, state_in, state_out, out, saved, B, H, F, T, d, eps, stream
+    assert lib.gla_forward_train(vp, vp, vp, vp, None, None, vp, vp, 1, 1, 1, 64, 64, 1e-6,
+                                 None) == 4
+    assert lib.gla_forward_train(vp, vp, vp, vp, None, None, vp, None, 1, 1, 1, 64, 128, 1e-6,
+                                 None) == 1
+    assert lib.gla_forward_train(vp, vp, vp, vp, None, None, vp, odd, 1, 1, 1, 64, 128, 1e-6,
+                                 None) == 2
+    # backward_saved: q, k, v, g, state_in, saved, dout, dstate_out, dq, dk, dv, dg, dstate_in, ...
+    assert lib.gla_backward_saved(vp, vp, vp, vp, None, vp, vp, None, vp, vp, vp, vp, None, 1, 1,
+                                  1, 64, 64, 1e-6, None) == 4
+    assert lib.gla_backward_saved(vp, vp, vp, vp, None, None, vp, None, vp, vp, vp, vp, None, 1,
+                                  1, 1, 64, 128, 1e-6, None) == 1
+    assert lib.gla_backward_saved(vp, vp, vp, vp, None, odd, vp, None, vp, vp, vp, vp, None, 1, 1,
+                                  1, 64, 128, 1e-6, None) == 2
