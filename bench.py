@@ -85,12 +85,16 @@ KERNEL_DEPS = {
     "output": ["gla_output.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
     "increment": ["gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
     "scan": ["gla_scan.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "bwd_q": ["gla_bwd_q.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "bwd_kv": ["gla_bwd_kv.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
 }
 NCU_TRAFFIC = {
-    "720p-5s": {
-        "increment": (1899750400 + 65932800, "7ba1204ca68b5243"),
-        "scan": (75847168 + 5340416, "a01d1703ef5f48a1"),
-        "output": (985584384 + 895718912, "da79c97d4ca61853"),
+    "720p-5s": {  # one full-size launch per kernel (profiles/dram_traffic_720p5s.md)
+        "increment": (1899741952 + 66090240, "7ec6315c7f5f901f"),
+        "scan": (76416768 + 9223424, "5b994b5cab5c7b37"),
+        "output": (985622016 + 899729664, "85ca97577127ee68"),
+        "bwd_q": (1972424960 + 993002752, "d8374f4021c3a391"),
+        "bwd_kv": (1972606720 + 1851400960, "9c0a7b912011f98f"),
     },
 }
 
@@ -767,9 +771,10 @@ def run_gpu_backward(args, w, dist, rank, local_rank, world):
         avg = avg[2:]
     dom = int(np.argmax(avg))
     achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
+    traffic = ncu_traffic(w.name, names[dom]) if names[dom] in KERNEL_DEPS else None
     roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": None, "traffic_unit": "bytes per launch (ncu dram read + write)",
+            "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read + write)",
             "algorithmic_bytes_per_launch": work[names[dom]],
             "peak_source": peaks["source"] + " (hbm_gbs)"}
     t_roof = max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
