@@ -487,7 +487,11 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
       W > 0 ? align256(slots * static_cast<int64_t>(gla::IncCfg<D>::kPartialFloats) * 4) : 0;
   const int64_t mpartial_bytes = W > 0 ? align256(slots * static_cast<int64_t>(D) * D * 4) : 0;
   const int64_t image_bytes = W > 0 ? align256(units * static_cast<int64_t>(G::kImageBytes)) : 0;
-  const int64_t ws_bytes = partial_bytes + mpartial_bytes + image_bytes;
+  // d = 128: the tail units' Gram images (the tensor-core scan's A operands)
+  const int32_t tail_units = W > 0 ? wp.units - wp.full_units() : 0;
+  const int64_t mtail_bytes =
+      D == 128 ? align256(static_cast<int64_t>(tail_units) * 2 * gla::GramImage<D>::kBytes) : 0;
+  const int64_t ws_bytes = partial_bytes + mpartial_bytes + image_bytes + mtail_bytes;
 
   // state columns per scan block: as many blocks per (b, h) as fill the SMs
   // once, at least ceil((D + 1) / kMaxCols) and at most one per 8 columns
@@ -518,6 +522,7 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   float* partial = W > 0 ? reinterpret_cast<float*>(ws) : nullptr;
   float* mpartial = W > 0 ? reinterpret_cast<float*>(ws + partial_bytes) : nullptr;
   uint8_t* image = W > 0 ? ws + partial_bytes + mpartial_bytes : nullptr;
+  uint8_t* mtail = mtail_bytes > 0 ? ws + partial_bytes + mpartial_bytes + image_bytes : nullptr;
 
   int status = GLA_OK;
   auto check = [&]() {
@@ -536,7 +541,6 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
     check();
   }
   // the tail units' Gram partials -> one per unit
-  const int32_t tail_units = W > 0 ? wp.units - wp.full_units() : 0;
   if (tail_units > 0 && status == GLA_OK) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tail_units), 4);
@@ -547,13 +551,21 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gla::gla_gram_reduce_kernel<D>, mpartial, wp) != cudaSuccess)
-      status = GLA_ERR_LAUNCH;
+    cudaError_t e;
+    if constexpr (D == 128) {
+      // the tensor-core scan reads one Gram image and one dS partial per unit
+      cfg.gridDim = dim3(static_cast<unsigned>(tail_units), gla::kGramParts + gla::kDsParts);
+      e = cudaLaunchKernelEx(&cfg, gla::gla_gdn_tail_reduce_kernel<D>, partial,
+                             static_cast<const float*>(mpartial), mtail, wp);
+    } else {
+      e = cudaLaunchKernelEx(&cfg, gla::gla_gram_reduce_kernel<D>, mpartial, wp);
+    }
+    if (e != cudaSuccess) status = GLA_ERR_LAUNCH;
     check();
   }
   record(1);
   if (status == GLA_OK && (a.F > 0 || a.s_out != nullptr)) {
-    gla::GdnScanParams sp{partial, mpartial, a.g, a.beta, a.s_in, a.s_out, image, wp,
+    gla::GdnScanParams sp{partial, mpartial, mtail, a.g, a.beta, a.s_in, a.s_out, image, wp,
                           a.H, a.F, tpu, groups, cols};
     const unsigned grid = static_cast<unsigned>(groups) * static_cast<unsigned>(bh);
     cudaError_t e;

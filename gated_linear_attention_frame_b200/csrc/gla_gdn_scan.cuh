@@ -38,7 +38,8 @@ namespace gla {
 
 struct GdnScanParams {
   const float* partial;   // dS_f partials [slots][d + 1][d] (transposed, row d = normaliser)
-  const float* mpartial;  // M_f partials [slots][d][d]
+  const float* mpartial;  // M_f partials [slots][d][d] (d = 128: a whole unit's GramImage pair)
+  const uint8_t* mtail;   // d = 128: GramImage pairs of the tail units [tail units][d * d * 4 B]
   const float* gate;      // [B, F, H] decay logits
   const float* beta;      // [B, F, H] write-strength logits
   const float* state_in;  // [B, H, d, d + 1] or nullptr
@@ -336,35 +337,98 @@ __global__ void __launch_bounds__(256) gla_gram_reduce_kernel(float* mpartial, W
 
 namespace gla {
 
+// The tail units at d = 128 (tensor-core scan): the Gram partials of slots
+// u + c0 .. u + c1 are summed in fp32 (in slot order) and written as the
+// unit's GramImage pair into mtail, and the dS partials of those slots are
+// summed into slot u + c0, so that the scan streams one M_f image and one
+// dS_f per frame.  Grid: (tail units, kGramParts + kDsParts); y < kGramParts
+// takes 2 of the 16 K chunks of M_f (one 8-element chunk of one row per
+// thread), the rest interleaved float4s of the dS rows.
+constexpr int kGramParts = 8;
+constexpr int kDsParts = 8;
+
+template <int D>
+__global__ void __launch_bounds__(256) gla_gdn_tail_reduce_kernel(float* partial,
+                                                                  const float* mpartial,
+                                                                  uint8_t* mtail, WorkPlan wp) {
+  static_assert(D == 128 && D / 8 == 2 * kGramParts, "two K chunks of 128 rows per block");
+  constexpr int PF = IncCfg<D>::kPartialFloats;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t t = blockIdx.x;
+  const int64_t u = static_cast<int64_t>(wp.full_units()) + t;
+  int32_t c0, c1;
+  wp.slot_range(u, c0, c1);
+  if (blockIdx.y < kGramParts) {
+    const int i = threadIdx.x & 127;                        // row of M_f
+    const int ch = 2 * blockIdx.y + (threadIdx.x >> 7);     // elements 8 ch .. 8 ch + 7
+    float x[8];
+    const float* src = mpartial + (u + c0) * static_cast<int64_t>(D) * D + ch * 8 * D + i;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = src[e * D];
+    for (int cc = c0 + 1; cc <= c1; ++cc) {
+      src += static_cast<int64_t>(D) * D;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] += src[e * D];
+    }
+    uint4 hi, lo;
+    split_bf16x8(x, hi, lo);
+    uint8_t* img = mtail + t * (2 * GramImage<D>::kBytes);
+    const int off = GramImage<D>::offset(i, ch);
+    *reinterpret_cast<uint4*>(img + off) = hi;
+    *reinterpret_cast<uint4*>(img + GramImage<D>::kBytes + off) = lo;
+  } else if (c1 > c0) {
+    float4* dst = reinterpret_cast<float4*>(partial + (u + c0) * PF);
+    for (int x = (blockIdx.y - kGramParts) * blockDim.x + threadIdx.x; x < PF / 4;
+         x += kDsParts * blockDim.x) {
+      float4 acc = dst[x];
+      for (int cc = c0 + 1; cc <= c1; ++cc) {
+        const float4 v = reinterpret_cast<const float4*>(partial + (u + cc) * PF)[x];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      dst[x] = acc;
+    }
+  }
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core delta scan (d = 128).  Same recurrence as gla_gdn_scan_kernel;
 // the per-frame product M_f S_{f-1}[:, J] of a block's column group J runs on
 // tcgen05 with a bf16 hi/lo split of both factors (Mh Sh + Mh Sl + Ml Sh into
 // an fp32 TMEM accumulator, the dropped Ml Sl term is ~2^-16 relative):
-//   A = M_f hi / lo   [M = 128 rows i, K = 128]  K-major, 128-byte swizzle
-//                     (built in shared memory from the fp32 Gram matrix)
+//   A = M_f hi / lo   [M = 128 rows i, K = 128]  K-major, no swizzle: the
+//                     GramImage pair that the increment kernel (whole units)
+//                     or the tail reduction wrote, bulk-copied as it is
 //   B = S_{f-1} hi / lo [N = group columns padded to 16, K = 128 rows k]
 //                     MN-major, 32-byte swizzle atoms of 16 columns
-// Thread i of the four consumer warps owns row i of the group's state (TMEM
-// lane i): it converts row i of M_f (M is symmetric, so the row is read as a
-// column, conflict-free), reads back row i of the product, updates its fp32
-// state row and writes the bf16 image and the next frame's B operand.  A
-// producer warp streams M_f; one thread issues the MMAs.
+// A producer warp streams each frame's A images and the group's dS_f rows
+// into a two-stage ring; one thread issues the MMAs once the frame's stage has
+// landed and the consumers have written B.  Thread i of the four consumer
+// warps owns row i of the group's state (TMEM lane i): it reads back row i of
+// the product, updates its fp32 state row, writes the next frame's B operand
+// (the only step between two products) and then, while the next product
+// runs, the bf16 image of S_f^T that the output kernel reads.
 template <int D>
 struct GdnTcCfg {
   static_assert(D == 128, "tensor-core delta scan is built for d = 128");
   static constexpr int kMaxCols = 48;              // three blocks cover d + 1 columns
   static constexpr int kConsumers = 128;
   static constexpr int kThreads = kConsumers + 64; // + producer warp + MMA warp
-  static constexpr int kMBytes = D * D * 4;        // fp32 Gram matrix
-  static constexpr int kStages = 2;                // M_{f+1} streams in during frame f
-  static constexpr int kAImgBytes = D * D * 2;     // one bf16 copy (hi or lo)
+  static constexpr int kAImgBytes = GramImage<D>::kBytes;  // one bf16 image (hi or lo)
+  static constexpr int kDsBytes = kMaxCols * D * 4;        // the group's dS_f rows, fp32
+  static constexpr int kHdrOff = 2 * kAImgBytes + kDsBytes;
+  static constexpr int kStageBytes = kHdrOff + 1024;       // + header; stages 1024-aligned
+  static constexpr int kStages = 2;                // frame f+1 streams in during frame f
   static constexpr int kBAtomBytes = D * 32;       // 16 columns x 128 rows
   static constexpr int kBImgBytes = (kMaxCols / 16) * kBAtomBytes;
   static constexpr int kTmemCols = 64;
   static constexpr int kBarCount = 2 * kStages + 3;
-  static constexpr int kSmemBytes = 1024 + 2 * kAImgBytes + 2 * kBImgBytes +
-                                    kStages * (kMBytes + 16) + kBarCount * 8 + 16;
+  static constexpr int kSmemBytes =
+      1024 + kStages * kStageBytes + 2 * kBImgBytes + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
 };
 
@@ -374,28 +438,25 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   using C = GdnTcCfg<D>;
   constexpr int PF = IncCfg<D>::kPartialFloats;
   constexpr unsigned kCode = 64u;
-  constexpr int CPA = G::kAtomElems / 8;
   constexpr int S = C::kStages;
   constexpr int MC = C::kMaxCols;
+  constexpr int CPA = G::kAtomElems / 8;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t a_hi = sbase;                                  // 1024-aligned
-  const uint32_t a_lo = a_hi + C::kAImgBytes;
-  const uint32_t b_hi = a_lo + C::kAImgBytes;
+  // stage s: [A hi | A lo | dS rows | header]
+  auto stage = [&](int s) { return smem + s * C::kStageBytes; };
+  auto dsst = [&](int s) { return reinterpret_cast<const float*>(stage(s) + 2 * C::kAImgBytes); };
+  auto hdr = [&](int s) { return reinterpret_cast<GdnStageHeader*>(stage(s) + C::kHdrOff); };
+  const uint32_t b_hi = sbase + S * C::kStageBytes;
   const uint32_t b_lo = b_hi + C::kBImgBytes;
-  uint8_t* mbase = smem + 2 * C::kAImgBytes + 2 * C::kBImgBytes;
-  auto mst = [&](int s) { return reinterpret_cast<float*>(mbase + s * (C::kMBytes + 16)); };
-  auto hdr = [&](int s) {
-    return reinterpret_cast<GdnStageHeader*>(mbase + s * (C::kMBytes + 16) + C::kMBytes);
-  };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(mbase + S * (C::kMBytes + 16));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + 2 * C::kBImgBytes);
   const uint32_t bar0 = smem_u32(bars);
-  auto mfull = [&](int s) { return bar0 + 8u * s; };        // M_f landed (producer)
-  auto mempty = [&](int s) { return bar0 + 8u * (S + s); }; // M_f converted (4 warps)
-  const uint32_t opready = bar0 + 8u * (2 * S);     // A and B operands of a frame written
+  auto mfull = [&](int s) { return bar0 + 8u * s; };        // frame's stage landed (producer)
+  auto mempty = [&](int s) { return bar0 + 8u * (S + s); }; // stage used up (4 consumer warps)
+  const uint32_t bready = bar0 + 8u * (2 * S);      // B operand of a frame written (4 warps)
   const uint32_t accfull = bar0 + 8u * (2 * S + 1); // product in TMEM (MMA commit)
   const uint32_t done_bar = bar0 + 8u * (2 * S + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBarCount);
@@ -419,7 +480,7 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
       mbar_init(mfull(s), 1);
       mbar_init(mempty(s), 4);
     }
-    mbar_init(opready, 4);
+    mbar_init(bready, 4);
     mbar_init(accfull, 1);
     mbar_init(done_bar, 1);
     *abort = 0;
@@ -443,9 +504,10 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
     // The whole warp loads the gate and write-strength logits of 32 frames at
-    // a time (one lane per frame); lane 0 streams M_f.
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // Gram partials
+    // a time (one lane per frame); lane 0 streams the stages.
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // Gram images and dS partials
     if (stream) {
+      const uint32_t ds_bytes = static_cast<uint32_t>(ncols) * D * 4;
       float gl = 0.f, bl = 0.f;
       int f = 0;
       for (; f < p.F; ++f) {
@@ -469,9 +531,15 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
             hd->c1 = c1;
             hd->a = 1.0f / (1.0f + expf(-g));
             hd->beta = 1.0f / (1.0f + expf(-bb));
-            mbar_arrive_expect_tx(mfull(s), C::kMBytes);
-            bulk_load(smem_u32(mst(s)), p.mpartial + (u + c0) * static_cast<int64_t>(D) * D,
-                      C::kMBytes, mfull(s));
+            const int32_t uf = p.wp.full_units();
+            const void* aimg =
+                u < uf ? static_cast<const void*>(p.mpartial + u * static_cast<int64_t>(D) * D)
+                       : static_cast<const void*>(p.mtail + (u - uf) * (2 * C::kAImgBytes));
+            mbar_arrive_expect_tx(mfull(s), 2 * C::kAImgBytes + ds_bytes);
+            bulk_load(smem_u32(stage(s)), aimg, 2 * C::kAImgBytes, mfull(s));
+            bulk_load(smem_u32(stage(s)) + 2 * C::kAImgBytes,
+                      p.partial + (u + c0) * PF + static_cast<int64_t>(j0) * D, ds_bytes,
+                      mfull(s));
           }
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -486,8 +554,12 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
       const uint32_t idesc = idesc_bf16_f32(128, np, false, true);
       int f = 0;
       for (; f < p.F; ++f) {
-        if (!mbar_wait(opready, static_cast<uint32_t>(f & 1), abort, kCode)) break;
+        const int s = f % S;
+        if (!mbar_wait(mfull(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
+        if (!mbar_wait(bready, static_cast<uint32_t>(f & 1), abort, kCode)) break;
         tc_fence_after();
+        const uint32_t a_hi = smem_u32(stage(s));
+        const uint32_t a_lo = a_hi + C::kAImgBytes;
         // Mh Sh + Mh Sl + Ml Sh over K = 128 (8 steps of 16)
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass) {
@@ -495,9 +567,9 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
           const uint32_t bbase = pass == 1 ? b_lo : b_hi;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const int at = kk / 4, w = kk % 4;
-            const uint64_t ad = smem_desc(abase + at * (128 * G::kRowBytes) + w * 32, 16,
-                                          G::kGroupBytes, kLayoutSW128);
+            using GI = GramImage<D>;
+            const uint64_t ad = smem_desc(abase + kk * 2 * GI::kChunkStride, GI::kChunkStride,
+                                          GI::kGroupStride, kLayoutNone);
             const uint64_t bd = smem_desc(bbase + kk * 512, C::kBAtomBytes, 256, kLayoutSW32);
             mma_bf16(tmem, ad, bd, idesc, (pass > 0 || kk > 0) ? 1u : 0u);
           }
@@ -517,22 +589,23 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
     auto b_off = [&](int jl) {
       return (jl >> 4) * C::kBAtomBytes + i * 32 + ((((jl >> 3) & 1) ^ ((i >> 2) & 1)) << 4);
     };
-    auto write_b = [&]() {  // the group's columns of row i, hi and lo
+    auto write_b = [&]() {  // the group's columns of row i, hi and lo, then hand B over
 #pragma unroll
       for (int jc = 0; jc < MC; jc += 8) {
         if (jc < np) {
-          uint32_t hw[4], lw[4];
+          float x[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float x0 = (jc + 2 * e2 < ncols) ? sr[jc + 2 * e2] : 0.f;
-            const float x1 = (jc + 2 * e2 + 1 < ncols) ? sr[jc + 2 * e2 + 1] : 0.f;
-            hw[e2] = pack_bf16x2(x0, x1);
-            lw[e2] = pack_bf16x2(x0 - bf16lo_to_f32(hw[e2]), x1 - bf16hi_to_f32(hw[e2]));
-          }
-          st_shared_v4(b_hi + b_off(jc), make_uint4(hw[0], hw[1], hw[2], hw[3]));
-          st_shared_v4(b_lo + b_off(jc), make_uint4(lw[0], lw[1], lw[2], lw[3]));
+          for (int e = 0; e < 8; ++e) x[e] = (jc + e < ncols) ? sr[jc + e] : 0.f;
+          uint4 hi, lo;
+          split_bf16x8(x, hi, lo);
+          st_shared_v4(b_hi + b_off(jc), hi);
+          st_shared_v4(b_lo + b_off(jc), lo);
         }
       }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bready);
     };
     // S_{-1}: row i of the group's columns
 #pragma unroll
@@ -544,59 +617,31 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
     asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int f = 0; f < p.F; ++f) {
       const int64_t u = u0 + static_cast<int64_t>(f) * p.H;
-      float a, beta;
+      float a;
       if (stream) {
         const int s = f % S;
         if (!warp_wait(mfull(s), static_cast<uint32_t>((f / S) & 1), abort, kCode)) break;
         const GdnStageHeader hd = *hdr(s);
         a = hd.a;
-        beta = hd.beta;
-        // A operands: row i of M_f (= column i, M symmetric), hi and lo
-        const float* m = mst(s);
-#pragma unroll 2
-        for (int ch = 0; ch < D / 8; ++ch) {
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = m[(ch * 8 + e) * D + i];
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            hw[e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
-            lw[e2] = pack_bf16x2(x[2 * e2] - bf16lo_to_f32(hw[e2]),
-                                 x[2 * e2 + 1] - bf16hi_to_f32(hw[e2]));
-          }
-          const uint32_t off = (ch / CPA) * (128 * G::kRowBytes) + i * G::kRowBytes +
-                               G::swz(i, ch % CPA) * 16;
-          st_shared_v4(a_hi + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-          st_shared_v4(a_lo + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(mempty(s));  // the producer may load M_{f+2} into this stage
-          mbar_arrive(opready);    // A of this frame and B (written last frame) ready
-        }
-        // this frame's dS rows, loaded while the product runs
+        const float beta = hd.beta;
+        // this frame's dS rows, read while the product runs
+        const float* dss = dsst(s);
         float ds[MC];
 #pragma unroll
-        for (int jl = 0; jl < MC; ++jl) ds[jl] = 0.f;
-        for (int cc = hd.c0; cc <= hd.c1; ++cc) {
-          const float* src = p.partial + (u + cc) * PF + static_cast<int64_t>(j0) * D + i;
-#pragma unroll
-          for (int jl = 0; jl < MC; ++jl)
-            if (jl < ncols) ds[jl] += __ldg(src + static_cast<int64_t>(jl) * D);
-        }
+        for (int jl = 0; jl < MC; ++jl) ds[jl] = jl < ncols ? dss[jl * D + i] : 0.f;
         if (!warp_wait(accfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
         tc_fence_after();
         uint32_t r[2][32];
         tmem_ld_32cols(tmem + lane_base, r[0]);
         tmem_ld_32cols(tmem + lane_base + 32, r[1]);
         tmem_wait_ld();
-        tc_fence_before();
 #pragma unroll
         for (int jl = 0; jl < MC; ++jl)
           if (jl < ncols)
             sr[jl] = a * fmaf(-beta, __uint_as_float(r[jl >> 5][jl & 31]), sr[jl]) + beta * ds[jl];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mempty(s));  // A consumed (product done), dS read
+        if (f + 1 < p.F) write_b();             // next frame's B: the product may start
       } else {
         a = 1.0f / (1.0f + expf(-__ldg(p.gate + u)));  // no tokens: the state only decays
 #pragma unroll
@@ -616,7 +661,6 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
           }
         }
       }
-      if (stream && f + 1 < p.F) write_b();  // next frame's B
     }
     if (p.state_out != nullptr) {
 #pragma unroll

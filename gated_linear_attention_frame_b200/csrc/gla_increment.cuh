@@ -53,6 +53,33 @@ struct IncCfg {
       1024 + kStages * kStageBytes + kZBytes + kFoldBytes + kBarBytes + 16;
 };
 
+// The delta-rule variant at d = 128 hands M_f to the tensor-core scan as
+// that scan's A operand: two bf16 images of [D rows i][D elements k] (hi,
+// then lo = bf16(M - hi), so that hi + lo carries ~16 bits of M), K-major
+// without swizzle: 8-row x 16-byte core matrices, the 16 bytes holding
+// elements 8 ch .. 8 ch + 7 of row i at ch * 16 D + 16 i.  Core matrices are
+// 128 bytes apart along M and 16 D bytes apart along K, and a warp that owns
+// 32 consecutive rows writes one chunk of each as 512 contiguous bytes.
+template <int D>
+struct GramImage {
+  static constexpr int kBytes = D * D * 2;  // one image
+  static constexpr int kChunkStride = 16 * D;  // between K chunks (core matrices along K)
+  static constexpr int kGroupStride = 128;     // between 8-row groups (along M)
+  __host__ __device__ static constexpr int offset(int i, int ch) { return ch * kChunkStride + i * 16; }
+};
+
+// hi / lo bf16 split of 8 consecutive fp32 values (x = hi + lo + O(2^-16 |x|))
+__device__ __forceinline__ void split_bf16x8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e2 = 0; e2 < 4; ++e2) {
+    h[e2] = pack_bf16x2(x[2 * e2], x[2 * e2 + 1]);
+    l[e2] = pack_bf16x2(x[2 * e2] - bf16lo_to_f32(h[e2]), x[2 * e2 + 1] - bf16hi_to_f32(h[e2]));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 struct IncParams {
   float* partial;   // [(units + gridDim.x) slots][d + 1][d] fp32
   WorkPlan wp;      // tile assignment (gridDim.x == wp.G)
@@ -60,7 +87,9 @@ struct IncParams {
   int T;            // tokens per frame (rotary variant)
   RopeGeo rope;     // rotary variant only
   float* mpartial;  // Gram variant: [(units + gridDim.x) slots][d][d] fp32 partials of
-                    // M_f = phi(K_f)^T phi(K_f), rows as the increment partials
+                    // M_f = phi(K_f)^T phi(K_f), rows as the increment partials; at
+                    // d = 128 a unit owned whole by one CTA gets the GramImage pair
+                    // (hi | lo, d * d * 4 bytes) in its slot instead
   // Single-frame calls of the plain layer (fold = 1): for a unit owned whole
   // by one CTA the scan's step S = a S_in + dS is done here, from TMEM, at the
   // unit's end (overlapping the CTA's next tiles); a unit whose tiles are
@@ -475,14 +504,37 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
           for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
         }
         if constexpr (kGram) {
-          float* mdst = p.mpartial + cur.slot() * static_cast<int64_t>(D) * D + row;
+          if (D == 128 && cur.u < cur.U_full) {
+            // the whole unit: row i = row of M_f as the scan's A images
+            uint8_t* img = reinterpret_cast<uint8_t*>(
+                p.mpartial + cur.slot() * static_cast<int64_t>(D) * D);
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld_32cols(tacc + D + cc * 32, r);
-            tmem_wait_ld();
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(tacc + D + cc * 32, r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) mdst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+              for (int q = 0; q < 4; ++q) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[q * 8 + e]);
+                uint4 hi, lo;
+                split_bf16x8(x, hi, lo);
+                const int off = GramImage<D>::offset(row, cc * 4 + q);
+                *reinterpret_cast<uint4*>(img + off) = hi;
+                *reinterpret_cast<uint4*>(img + GramImage<D>::kBytes + off) = lo;
+              }
+            }
+          } else {
+            float* mdst = p.mpartial + cur.slot() * static_cast<int64_t>(D) * D + row;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32cols(tacc + D + cc * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int jj = 0; jj < 32; ++jj) mdst[(cc * 32 + jj) * D] = __uint_as_float(r[jj]);
+            }
           }
         }
       }

@@ -312,7 +312,7 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // ------------------------------------------------------------ descriptors
 
 // Shared-memory layouts of tcgen05 matrix operands (descriptor bits 61..63).
-enum : uint32_t { kLayoutSW128 = 2u, kLayoutSW64 = 4u, kLayoutSW32 = 6u };
+enum : uint32_t { kLayoutNone = 0u, kLayoutSW128 = 2u, kLayoutSW64 = 4u, kLayoutSW32 = 6u };
 
 // Shared-memory matrix descriptor: start address, leading-dimension byte
 // offset, stride-dimension byte offset (all >> 4), version 1 (bit 46), base
