@@ -398,8 +398,11 @@ __global__ void __launch_bounds__(256) gla_gdn_tail_reduce_kernel(float* partial
 // ---------------------------------------------------------------------------
 // Tensor-core delta scan (d = 128).  Same recurrence as gla_gdn_scan_kernel;
 // the per-frame product M_f S_{f-1}[:, J] of a block's column group J runs on
-// tcgen05 with a bf16 hi/lo split of both factors (Mh Sh + Mh Sl + Ml Sh into
-// an fp32 TMEM accumulator, the dropped Ml Sl term is ~2^-16 relative):
+// tcgen05 with a bf16 hi/lo split of both factors, Mh Sh + Mh Sl + Ml Sh in
+// fp32 (the dropped Ml Sl term is ~2^-16 relative): one product of Mh with
+// [Sh | Sl] (N = 48 + the group's padded width) into TMEM columns
+// [0, 48 + N) and Ml Sh accumulated onto columns [0, N), 16 MMAs per frame;
+// the consumers add columns j and 48 + j:
 //   A = M_f hi / lo   [M = 128 rows i, K = 128]  K-major, no swizzle: the
 //                     GramImage pair that the increment kernel (whole units)
 //                     or the tail reduction wrote, bulk-copied as it is
@@ -425,7 +428,7 @@ struct GdnTcCfg {
   static constexpr int kStages = 2;                // frame f+1 streams in during frame f
   static constexpr int kBAtomBytes = D * 32;       // 16 columns x 128 rows
   static constexpr int kBImgBytes = (kMaxCols / 16) * kBAtomBytes;
-  static constexpr int kTmemCols = 64;
+  static constexpr int kTmemCols = 128;            // [Mh Sh + Ml Sh | Mh Sl], 48 + 48 columns
   static constexpr int kBarCount = 2 * kStages + 3;
   static constexpr int kSmemBytes =
       1024 + kStages * kStageBytes + 2 * kBImgBytes + kBarCount * 8 + 16;
@@ -551,6 +554,9 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
   } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && stream) {
+      // [Sh | Sl] is one MN-major operand: Sl's atoms follow Sh's 48 columns
+      static_assert(C::kBImgBytes == (MC / 16) * C::kBAtomBytes, "B hi / lo adjacent");
+      const uint32_t idesc_w = idesc_bf16_f32(128, MC + np, false, true);
       const uint32_t idesc = idesc_bf16_f32(128, np, false, true);
       int f = 0;
       for (; f < p.F; ++f) {
@@ -560,18 +566,17 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
         tc_fence_after();
         const uint32_t a_hi = smem_u32(stage(s));
         const uint32_t a_lo = a_hi + C::kAImgBytes;
-        // Mh Sh + Mh Sl + Ml Sh over K = 128 (8 steps of 16)
+        // Mh [Sh | Sl], then Ml Sh onto the first columns, K = 128 (8 steps of 16)
 #pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t abase = pass == 2 ? a_lo : a_hi;
-          const uint32_t bbase = pass == 1 ? b_lo : b_hi;
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint32_t abase = pass == 1 ? a_lo : a_hi;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             using GI = GramImage<D>;
             const uint64_t ad = smem_desc(abase + kk * 2 * GI::kChunkStride, GI::kChunkStride,
                                           GI::kGroupStride, kLayoutNone);
-            const uint64_t bd = smem_desc(bbase + kk * 512, C::kBAtomBytes, 256, kLayoutSW32);
-            mma_bf16(tmem, ad, bd, idesc, (pass > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bd = smem_desc(b_hi + kk * 512, C::kBAtomBytes, 256, kLayoutSW32);
+            mma_bf16(tmem, ad, bd, pass == 0 ? idesc_w : idesc, (pass > 0 || kk > 0) ? 1u : 0u);
           }
         }
         mma_commit(accfull);
@@ -631,14 +636,31 @@ __global__ void __launch_bounds__(192, 1) gla_gdn_scan_tc_kernel(const GdnScanPa
         for (int jl = 0; jl < MC; ++jl) ds[jl] = jl < ncols ? dss[jl * D + i] : 0.f;
         if (!warp_wait(accfull, static_cast<uint32_t>(f & 1), abort, kCode)) break;
         tc_fence_after();
-        uint32_t r[2][32];
-        tmem_ld_32cols(tmem + lane_base, r[0]);
-        tmem_ld_32cols(tmem + lane_base + 32, r[1]);
-        tmem_wait_ld();
+        {
+          // (M S)[i, jl] = (Mh Sh + Ml Sh)[i, jl] + (Mh Sl)[i, jl], columns jl and MC + jl
+          uint32_t r0[32], r1[32];
+          tmem_ld_32cols(tmem + lane_base, r0);
+          tmem_ld_32cols(tmem + lane_base + MC, r1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int jl = 0; jl < MC; ++jl)
-          if (jl < ncols)
-            sr[jl] = a * fmaf(-beta, __uint_as_float(r[jl >> 5][jl & 31]), sr[jl]) + beta * ds[jl];
+          for (int jl = 0; jl < 32; ++jl)
+            if (jl < ncols) {
+              const float ms = __uint_as_float(r0[jl]) + __uint_as_float(r1[jl]);
+              sr[jl] = a * fmaf(-beta, ms, sr[jl]) + beta * ds[jl];
+            }
+        }
+        {
+          uint32_t r0[16], r1[16];
+          tmem_ld_16cols(tmem + lane_base + 32, r0);
+          tmem_ld_16cols(tmem + lane_base + MC + 32, r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jl = 32; jl < MC; ++jl)
+            if (jl < ncols) {
+              const float ms = __uint_as_float(r0[jl - 32]) + __uint_as_float(r1[jl - 32]);
+              sr[jl] = a * fmaf(-beta, ms, sr[jl]) + beta * ds[jl];
+            }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(mempty(s));  // A consumed (product done), dS read
         if (f + 1 < p.F) write_b();             // next frame's B: the product may start
