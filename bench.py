@@ -90,11 +90,11 @@ KERNEL_DEPS = {
 }
 NCU_TRAFFIC = {
     "720p-5s": {  # one full-size launch per kernel (profiles/dram_traffic_720p5s.md)
-        "increment": (1899741952 + 66090240, "7ec6315c7f5f901f"),
-        "scan": (76416768 + 9223424, "5b994b5cab5c7b37"),
-        "output": (985622016 + 899729664, "85ca97577127ee68"),
-        "bwd_q": (1972424960 + 993002752, "d8374f4021c3a391"),
-        "bwd_kv": (1972606720 + 1851400960, "9c0a7b912011f98f"),
+        "increment": (1899704832 + 66586880, "153cc2e58d51e778"),
+        "scan": (76400640 + 9127936, "aa02fdd8aea19246"),
+        "output": (985666048 + 899841024, "2775a5fbd5bf8547"),
+        "bwd_q": (1972508928 + 991425024, "1059a3a5c0663151"),
+        "bwd_kv": (1972515072 + 1851898624, "4d37c2a8e3dc0690"),
     },
 }
 
