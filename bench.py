@@ -89,7 +89,7 @@ KERNEL_DEPS = {
     "bwd_kv": ["gla_bwd_kv.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
 }
 NCU_TRAFFIC = {
-    "720p-5s": {  # one full-size launch per kernel (profiles/dram_traffic_720p5s.md)
+    "720p-5s": {  # ncu, one kernel and one full-size launch per capture
         "increment": (1899704832 + 66586880, "153cc2e58d51e778"),
         "scan": (76400640 + 9127936, "aa02fdd8aea19246"),
         "output": (985666048 + 899841024, "2775a5fbd5bf8547"),
