@@ -87,6 +87,14 @@ KERNEL_DEPS = {
     "scan": ["gla_scan.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
     "bwd_q": ["gla_bwd_q.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
     "bwd_kv": ["gla_bwd_kv.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    # the variants' kernels, keyed "<variant>:<kernel>"
+    "gdn:increment": ["gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "gdn:output": ["gla_output.cuh", "gla_increment.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "rope:increment": ["gla_increment.cuh", "gla_rope.cuh", "gla_common.cuh", "sm100_ptx.cuh"],
+    "rope:output": ["gla_output.cuh", "gla_rope.cuh", "gla_increment.cuh", "gla_common.cuh",
+                    "sm100_ptx.cuh"],
+    "softmax:anchor": ["gla_softmax_anchor.cuh", "gla_increment.cuh", "gla_common.cuh",
+                       "sm100_ptx.cuh"],
 }
 NCU_TRAFFIC = {
     "720p-5s": {  # ncu, one kernel and one full-size launch per capture
@@ -95,6 +103,11 @@ NCU_TRAFFIC = {
         "output": (985666048 + 899841024, "2775a5fbd5bf8547"),
         "bwd_q": (1972508928 + 991425024, "1059a3a5c0663151"),
         "bwd_kv": (1972515072 + 1851898624, "4d37c2a8e3dc0690"),
+        "gdn:increment": (1899706368 + 131211776, "153cc2e58d51e778"),
+        "gdn:output": (985741056 + 898391808, "2775a5fbd5bf8547"),
+        "rope:increment": (1900125952 + 66200064, "00f70ec8c9dba5a9"),
+        "rope:output": (986217472 + 899981312, "cb6a0252b8370d15"),
+        "softmax:anchor": (9571651328 + 945963008, "3530e0ff9f7818e9"),
     },
 }
 
@@ -114,7 +127,7 @@ def ncu_traffic(workload: str, kernel: str):
     """DRAM bytes per launch measured by ncu for this workload and kernel, or
     None when there is no capture or the kernel changed since."""
     entry = NCU_TRAFFIC.get(workload, {}).get(kernel)
-    if entry is None or entry[1] != kernel_source_hash(kernel):
+    if entry is None or kernel not in KERNEL_DEPS or entry[1] != kernel_source_hash(kernel):
         return None
     return entry[0]
 
@@ -521,7 +534,8 @@ def run_gpu(args, w, dist, rank, local_rank, world):
     avg = per.mean(axis=0)
     dom = int(np.argmax(avg))
     achieved = work[names[dom]] / (avg[dom] * 1e-3) / 1e9
-    traffic = ncu_traffic(w.name, names[dom])
+    traffic = ncu_traffic(w.name, names[dom] if args.variant == "plain"
+                          else "%s:%s" % (args.variant, names[dom]))
     roof = {"bound": "hbm", "kernel": "gla_%s_kernel" % names[dom], "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read + write)",
@@ -560,8 +574,6 @@ def run_gpu(args, w, dist, rank, local_rank, world):
         e2e = e2e_pipelined(dev, stream, dist, world, host_in, dev_out, call,
                             max(2, min(K, args.e2e_steps)), w.total_tokens)
 
-    if rope or gdn:
-        roof["traffic"] = None  # the counters were taken on the plain kernels
     # kernels per call: increment, scan, output; + the rotary table kernel; +
     # the Gram reduction when the tile schedule has tail units (delta rule)
     units = w.B * w.frames * w.H
@@ -878,7 +890,9 @@ def run_gpu_anchor(args, w, dist, rank, local_rank, world):
     peak = peaks["bf16_tflops_sustained"]
     roof = {"bound": "tensor", "kernel": "gla_softmax_anchor_kernel", "achieved": round(achieved, 1),
             "peak": peak, "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4),
+            "traffic": ncu_traffic(w.name, "softmax:anchor"),
+            "traffic_unit": "bytes per launch (ncu dram read + write)",
             "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
             "algorithmic_flops_per_launch": flops,
             "flops_note": "4 d per (query, key) pair (Q K^T and P V, one online pass)",
