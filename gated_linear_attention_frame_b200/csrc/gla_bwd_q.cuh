@@ -424,7 +424,10 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = !cr.valid() || relu();
     int64_t i = 0, useg = -1;
     int b = 0, f = 0, h = 0;
-    float nacc = 0.f;  // sum over this warp's tokens of phi(q_t)[row] dden_t, per unit
+    // sums over this warp's tokens of phi(q_t)[j] dden_t, per unit, for the
+    // key features j = 32 q4 + 16 lb + 8 fh + lane / 4 (index 2 lb + fh), each
+    // over this thread's token pairs
+    float nq[4] = {0.f, 0.f, 0.f, 0.f};
     for (; ok && cur.valid(); cur.advance(), ++i) {
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const int s = static_cast<int>(i % S);
@@ -497,52 +500,56 @@ __global__ void __launch_bounds__(320, 1)
       if (!warp_wait_fast(afree, ph ^ 1u, abort, kCode)) break;
       tc_fence_after();
       {
-        const int cin = (row % G::kAtomElems) / 8;
-        const uint16_t* qcol = reinterpret_cast<const uint16_t*>(
-            smem + (q_buf(s) - sbase) + (row / G::kAtomElems) * G::kAtomTileBytes +
-            hc * 64 * G::kRowBytes + (row % 8) * 2);
-        const uint16_t* b8[8];  // row base of each swizzle phase (token % 8)
-#pragma unroll
-        for (int r = 0; r < 8; ++r) b8[r] = qcol + ((cin ^ r) << 3);
+        // 8 x 8 blocks of phi(Q) (token rows) read transposed: thread t gets,
+        // per block, one key feature (t / 4 of the block's 8) at the token
+        // pair 2 (t % 4), 2 (t % 4) + 1, which is the 16-lane TMEM store's
+        // layout (lanes = key features, columns = token pairs)
         const float* rdn = rd_p + (i & 1) * 2 * kTileTokens + hc * 64;
         const float* ddn = rdn + kTileTokens;
-        uint64_t na2 = f2_pack(0.f, 0.f);
+        const int mi = lane >> 3;                       // this lane's ldmatrix block
+        const int tp = 2 * (lane & 3);                  // first token of this thread's pairs
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int lb = 0; lb < 2; ++lb) {                // key features 32 q4 + 16 lb ..
+          const int fc = q4 * 4 + lb * 2 + (mi & 1);    // 16-byte feature chunk of the row
+          const uint32_t fbase = q_buf(s) + (fc / CPA) * G::kAtomTileBytes;
           uint32_t hi[16], lo[16];
+          uint64_t na2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-          for (int qd = 0; qd < 8; ++qd) {  // 4 tokens
-            const int t0 = half * 32 + qd * 4;  // token within this warp's 64
-            const float4 r4 = *reinterpret_cast<const float4*>(rdn + t0);
-            const float4 g4 = *reinterpret_cast<const float4*>(ddn + t0);
-            const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
-            const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+          for (int tg = 0; tg < 4; ++tg) {              // tokens 64 hc + 16 tg ..
+            const int tr = hc * 64 + tg * 16 + (mi >> 1) * 8 + (lane & 7);
+            uint32_t m4[4];
+            ldmatrix_x4_trans(fbase + tr * G::kRowBytes + G::swz(tr, fc % CPA) * 16, m4);
 #pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-              const int t = t0 + 2 * pr;
-              constexpr int RE = G::kRowBytes / 2;  // elements per swizzled row
-              const float p0 = __uint_as_float(static_cast<uint32_t>(b8[t & 7][t * RE]) << 16);
-              const float p1 =
-                  __uint_as_float(static_cast<uint32_t>(b8[(t + 1) & 7][(t + 1) * RE]) << 16);
-              const uint64_t p2 = f2_pack(p0, p1);
-              float x0, x1;
-              f2_unpack(f2_mul(f2_pack(rr[2 * pr], rr[2 * pr + 1]), p2), x0, x1);
-              const uint32_t w = pack_bf16x2(x0, x1);
-              hi[qd * 2 + pr] = w;
-              float l0, l1;
-              f2_unpack(f2_sub(f2_pack(x0, x1), f2_pack(bf16lo_to_f32(w), bf16hi_to_f32(w))), l0,
-                        l1);
-              lo[qd * 2 + pr] = pack_bf16x2(l0, l1);
-              na2 = f2_fma(p2, f2_pack(gg[2 * pr], gg[2 * pr + 1]), na2);
+            for (int tt = 0; tt < 2; ++tt) {           // token pair tg * 16 + tp + 8 tt
+              const int t = tg * 16 + tp + 8 * tt;
+              const float2 r2 = *reinterpret_cast<const float2*>(rdn + t);
+              const float2 g2 = *reinterpret_cast<const float2*>(ddn + t);
+              const uint64_t rr2 = f2_pack(r2.x, r2.y), gg2 = f2_pack(g2.x, g2.y);
+#pragma unroll
+              for (int fh = 0; fh < 2; ++fh) {         // key feature 16 lb + 8 fh + lane / 4
+                const uint32_t pw = m4[2 * tt + fh];
+                const uint64_t p2 = f2_pack(bf16lo_to_f32(pw), bf16hi_to_f32(pw));
+                float x0, x1;
+                f2_unpack(f2_mul(rr2, p2), x0, x1);
+                const uint32_t w = pack_bf16x2(x0, x1);
+                float l0, l1;
+                f2_unpack(f2_sub(f2_pack(x0, x1), f2_pack(bf16lo_to_f32(w), bf16hi_to_f32(w))),
+                          l0, l1);
+                hi[2 * (2 * tg + tt) + fh] = w;
+                lo[2 * (2 * tg + tt) + fh] = pack_bf16x2(l0, l1);
+                na2[fh] = f2_fma(p2, gg2, na2[fh]);
+              }
             }
           }
-          tmem_st_16cols(tmem + lane_base + C::kAHi + hc * 32 + half * 16, hi);
-          tmem_st_16cols(tmem + lane_base + C::kALo + hc * 32 + half * 16, lo);
-        }
-        {
-          float na0, na1;
-          f2_unpack(na2, na0, na1);
-          nacc += na0 + na1;
+          const uint32_t ta = tmem + lane_base + (static_cast<uint32_t>(lb * 16) << 16) + hc * 32;
+          tmem_st_16x128b_x8(ta + C::kAHi, hi);
+          tmem_st_16x128b_x8(ta + C::kALo, lo);
+#pragma unroll
+          for (int fh = 0; fh < 2; ++fh) {
+            float na0, na1;
+            f2_unpack(na2[fh], na0, na1);
+            nq[2 * lb + fh] += na0 + na1;
+          }
         }
         tmem_wait_st();
       }
@@ -634,7 +641,22 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc3_free);
-        // row d: the two token halves' sums of phi(q_t) dden_t
+        // row d: the two token halves' sums of phi(q_t) dden_t; this warp's
+        // share of lane `row`: the four token-pair partials of its quad
+        float nacc;
+        {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            nq[k] += __shfl_xor_sync(0xffffffffu, nq[k], 1);
+            nq[k] += __shfl_xor_sync(0xffffffffu, nq[k], 2);
+          }
+          const int src = 4 * (lane & 7);               // a thread of feature lane's quad
+          const int kk = 2 * (lane >> 4) + ((lane >> 3) & 1);
+          float v[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) v[k] = __shfl_sync(0xffffffffu, nq[k], src);
+          nacc = kk == 0 ? v[0] : kk == 1 ? v[1] : kk == 2 ? v[2] : v[3];
+        }
         if (hc == 1) {
           nx_p[row] = nacc;
           __syncwarp();
@@ -643,7 +665,8 @@ __global__ void __launch_bounds__(320, 1)
           if (!warp_wait_fast(nbar(q4), static_cast<uint32_t>(useg & 1), abort, kCode)) break;
           dst[static_cast<int64_t>(D) * D] = nacc + nx_p[row];
         }
-        nacc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) nq[k] = 0.f;
       }
     }
     if (lane == 0) bulk_wait_group<0>();

@@ -264,6 +264,31 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
       : "memory");
 }
 
+// 16 lanes x 128 bit, 8 repetitions along the columns: thread t writes, for
+// repetition k, r[2k] to lane l + t / 4 and r[2k + 1] to lane l + 8 + t / 4,
+// both at column c + 4k + t % 4 (l, c: the address's lane and column; l is
+// 0 or 16 within the warp's lane quarter).
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// Four 8 x 8 bf16 matrices from shared memory, transposed: lanes 8m .. 8m + 7
+// give the addresses of matrix m's 8 rows (16 bytes each); thread t gets in
+// r[m] elements (row 2 (t % 4), column t / 4) and (row 2 (t % 4) + 1, column
+// t / 4) of matrix m, the first in the low half.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
 // 32 lanes x 32 bit, 16 consecutive columns (as tmem_ld_32cols).
 __device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
