@@ -98,16 +98,16 @@ KERNEL_DEPS = {
 }
 NCU_TRAFFIC = {
     "720p-5s": {  # ncu, one kernel and one full-size launch per capture
-        "increment": (1899704832 + 66586880, "153cc2e58d51e778"),
-        "scan": (76400640 + 9127936, "aa02fdd8aea19246"),
-        "output": (985666048 + 899841024, "2775a5fbd5bf8547"),
-        "bwd_q": (1972508928 + 991425024, "1059a3a5c0663151"),
-        "bwd_kv": (1972515072 + 1851898624, "4d37c2a8e3dc0690"),
-        "gdn:increment": (1899706368 + 131211776, "153cc2e58d51e778"),
-        "gdn:output": (985741056 + 898391808, "2775a5fbd5bf8547"),
-        "rope:increment": (1900125952 + 66200064, "00f70ec8c9dba5a9"),
-        "rope:output": (986217472 + 899981312, "cb6a0252b8370d15"),
-        "softmax:anchor": (9571651328 + 945963008, "3530e0ff9f7818e9"),
+        "increment": (1899706880 + 66030592, "2dfd12f7c336bb5c"),
+        "scan": (76411136 + 8676608, "d1a81844eb801248"),
+        "output": (985627136 + 899218688, "a46f6cfd4c0fd9a9"),
+        "bwd_q": (1972530176 + 989206016, "6c473591c6b5c7d5"),
+        "bwd_kv": (1972743424 + 1851086336, "b368553cf092d91e"),
+        "gdn:increment": (1899702272 + 128526080, "2dfd12f7c336bb5c"),
+        "gdn:output": (985812992 + 898795520, "a46f6cfd4c0fd9a9"),
+        "rope:increment": (1899828736 + 65959680, "6b6f6cd52f009922"),
+        "rope:output": (986262016 + 900409600, "dd48f0563db5f644"),
+        "softmax:anchor": (8763404800 + 944289024, "09718e6ccbfd6386"),
     },
 }
 
