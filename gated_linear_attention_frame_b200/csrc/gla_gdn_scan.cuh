@@ -10,6 +10,9 @@
 // only the difference.  Unlike the plain gated scan, the update couples the
 // d rows of S through M_f, but every state column j is still independent:
 //   S_f[:, j] = a_f (S_{f-1}[:, j] - beta_f M_f S_{f-1}[:, j]) + beta_f dS_f[:, j].
+// Two kernels run this recurrence: gla_gdn_scan_tc_kernel (d = 128, the
+// product on tcgen05, described with it below) and gla_gdn_scan_kernel
+// (d = 32, 64, CUDA cores), described here.
 // One block owns a group of columns of one (b, h) and loops over the frames:
 // a producer warp bulk-copies M_f (fp32, d x d, the increment kernel's Gram
 // partial) into a two-stage shared-memory ring; eight consumer warps each own
