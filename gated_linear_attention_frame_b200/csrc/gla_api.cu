@@ -15,11 +15,16 @@
 //   5. gla_dgate_kernel      dg = a (1 - a) da
 //   6. gla_bwd_kv_kernel     dk, dv                                   (tcgen05)
 // gla_forward_gdn (the frame-wise delta-rule variant) enqueues
-//   1. gla_increment_kernel  dS_f and M_f = phi(K_f)^T phi(K_f) partials (tcgen05)
-//   2. gla_gdn_scan_kernel   S_f = a_f (S_{f-1} - beta_f M_f S_{f-1}) + beta_f dS_f
+//   1. gla_increment_kernel  dS_f partials and M_f = phi(K_f)^T phi(K_f)    (tcgen05;
+//                            at d = 128 a whole unit's M_f as bf16 hi/lo MMA operand images)
+//   1b. for units split over several CTAs: gla_gdn_tail_reduce_kernel (d = 128) or
+//       gla_gram_reduce_kernel (d = 32, 64)
+//   2. gla_gdn_scan_tc_kernel (d = 128, the product M_f S_{f-1} on tcgen05) or
+//      gla_gdn_scan_kernel (d = 32, 64): S_f = a_f (S_{f-1} - beta_f M_f S_{f-1}) + beta_f dS_f
 //   3. gla_output_kernel     as gla_forward
-// gla_softmax_anchor (d = 128) runs gla_softmax_anchor_kernel: two passes of
-// tcgen05 Q K^T over the key tiles of sinks + window, P V into TMEM.
+// gla_softmax_anchor (d = 128) runs gla_softmax_anchor_kernel: one online pass
+// over the key tiles of sinks + window, S = Q K^T and O += P V on tcgen05
+// with the running maxima and sums in the softmax warps.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
