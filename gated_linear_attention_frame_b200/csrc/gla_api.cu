@@ -432,9 +432,10 @@ int run(const Args& a, const DeviceInfo& di, cudaEvent_t* ev,
       ip.state_out = a.s_out;
       ip.image = image;
     }
-    gla::gla_increment_kernel<D, kRope>
-        <<<G1, gla::IncCfg<D, kRope>::kThreads, gla::IncCfg<D, kRope>::kSmemBytes, a.stream>>>(
-            tm_k, tm_v, ip);
+    if (launch_dependent(gla::gla_increment_kernel<D, kRope>, G1, gla::IncCfg<D, kRope>::kThreads,
+                         gla::IncCfg<D, kRope>::kSmemBytes, a.stream, tm_k, tm_v,
+                         ip) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
     check();
   }
   record(1);
@@ -541,8 +542,9 @@ int run_gdn(const Args& a, const DeviceInfo& di, cudaEvent_t* ev) {
   if (W > 0 && status == GLA_OK) {
     gla::IncParams ip{partial, wp, a.H, a.F, a.T, gla::RopeGeo{}, mpartial};
     using IC = gla::IncCfg<D, false, true>;
-    gla::gla_increment_kernel<D, false, true>
-        <<<G1, IC::kThreads, IC::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    if (launch_dependent(gla::gla_increment_kernel<D, false, true>, G1, IC::kThreads,
+                         IC::kSmemBytes, a.stream, tm_k, tm_v, ip) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
     check();
   }
   // the tail units' Gram partials -> one per unit
@@ -776,8 +778,9 @@ int run_backward(const BwdArgs& a, const DeviceInfo& di, cudaEvent_t* ev) {
   record(0);
   if (!saved && W > 0 && status == GLA_OK) {
     gla::IncParams ip{partial, wp, a.H, a.F};
-    gla::gla_increment_kernel<D>
-        <<<G1, gla::IncCfg<D>::kThreads, gla::IncCfg<D>::kSmemBytes, a.stream>>>(tm_k, tm_v, ip);
+    if (launch_dependent(gla::gla_increment_kernel<D>, G1, gla::IncCfg<D>::kThreads,
+                         gla::IncCfg<D>::kSmemBytes, a.stream, tm_k, tm_v, ip) != cudaSuccess)
+      status = GLA_ERR_LAUNCH;
     check();
   }
   record(1);

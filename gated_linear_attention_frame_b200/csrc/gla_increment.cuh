@@ -207,6 +207,11 @@ __global__ void __launch_bounds__(IncCfg<D, kRope, kGram>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent of whatever ran before it on the
+  // stream: every global read or write below comes after that grid has
+  // finished and its writes are visible (only the launch and this prologue
+  // overlap its last CTAs).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
