@@ -98,16 +98,16 @@ KERNEL_DEPS = {
 }
 NCU_TRAFFIC = {
     "720p-5s": {  # ncu, one kernel and one full-size launch per capture
-        "increment": (1899706880 + 66030592, "2dfd12f7c336bb5c"),
-        "scan": (76411136 + 8676608, "d1a81844eb801248"),
-        "output": (985627136 + 899218688, "a46f6cfd4c0fd9a9"),
-        "bwd_q": (1972530176 + 989206016, "6c473591c6b5c7d5"),
-        "bwd_kv": (1972743424 + 1851086336, "b368553cf092d91e"),
-        "gdn:increment": (1899702272 + 128526080, "2dfd12f7c336bb5c"),
-        "gdn:output": (985812992 + 898795520, "a46f6cfd4c0fd9a9"),
-        "rope:increment": (1899828736 + 65959680, "6b6f6cd52f009922"),
-        "rope:output": (986262016 + 900409600, "dd48f0563db5f644"),
-        "softmax:anchor": (8763404800 + 944289024, "09718e6ccbfd6386"),
+        "increment": (1899706880 + 65776896, "77706b5453f8c685"),
+        "scan": (76420096 + 9461760, "dc825921952c30f6"),
+        "output": (985888512 + 898614528, "ca0d25760e183b6d"),
+        "bwd_q": (1973153536 + 989409536, "b350490e812e8a26"),
+        "bwd_kv": (1972606464 + 1851236096, "482f220a22e6fbfc"),
+        "gdn:increment": (1899975680 + 130081536, "77706b5453f8c685"),
+        "gdn:output": (985748224 + 898199552, "ca0d25760e183b6d"),
+        "rope:increment": (1899834880 + 66113536, "57a13fddf495cfb7"),
+        "rope:output": (986200576 + 900601088, "8050e870a97585fa"),
+        "softmax:anchor": (8292931328 + 944969472, "4c96ba0ee6f65e3e"),
     },
 }
 
