@@ -228,7 +228,9 @@ int gla_softmax_anchor_step(const void* q, const void* k, const void* v, const v
  * beta_f ||phi(K_f)^T phi(K_f)|| < 2, e.g. k ~ N(0, 1/(d T)).
  * Arguments as gla_forward plus beta_logits fp32 [B, frames, H] (4-byte
  * aligned; must not be NULL when B * H * frames > 0).  Workspace: as
- * gla_forward plus 4 d^2 bytes per (batch, frame, head) and per SM.
+ * gla_forward plus 4 d^2 bytes per (batch, frame, head) and per SM (at
+ * d = 128 up to another 4 d^2 bytes per SM: the Gram matrices of the units
+ * that the tile schedule splits over several SMs).
  */
 int gla_forward_gdn(const void* q, const void* k, const void* v,
                     const float* gate_logits, const float* beta_logits,
