@@ -88,6 +88,7 @@ SMALL = [
     (1, 4, 6, 129, 32, True),
     (1, 37, 2, 400, 128, True),     # units split over two CTAs
     (2, 40, 3, 64, 128, False),     # more units than CTAs
+    (1, 1, 2, 5120, 128, True),     # each unit split over 40 CTAs (40 partials summed)
     (1, 3, 7, 255, 64, True),
 ]
 
